@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the block-quantized projection path on B200.
+
+One step = the paired Q8_0 decode projection workload: 64 back-to-back calls,
+each quantizing a fresh fp32 activation (1 x 4096) to Q8 and running the
+paired GEMV of two Q8_0 weights (8192 x 4096 each) against it.  Weights are
+rotated over enough copies that L2 (126 MB) cannot serve them.  The headline
+value is HBM GB/s of algorithmic bytes; the same JSON line also carries
+us/call, the roofline of the dominant kernel, an end-to-end figure through
+the public API with host buffers, the other decode workloads and the prefill
+dequant-GEMM TFLOP/s sweep, the CPU oracle baseline and clock samples.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import platform
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_PAIR, K_PAIR, CALLS = 8192, 4096, 64
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "decode GEMV HBM GB/s (% peak) and µs/call; prefill dequant-GEMM TFLOP/s"
+WORKLOAD = "paired Q8_0 decode projection: 2 x (8192 x 4096) weights, shared 1 x 4096 activation, 64 calls"
+
+
+def paired_bytes_per_call() -> dict:
+    """Algorithmic bytes of one call: the quantize step and the paired GEMV."""
+    rb = K_PAIR // 32 * 34
+    gemv = 2 * N_PAIR * rb + K_PAIR + (K_PAIR // 32) * 4 + 2 * N_PAIR * 4
+    quant = K_PAIR * 4 + K_PAIR + 2 * (K_PAIR // 32) * 4
+    return {"gemv": gemv, "quant": quant, "total": gemv + quant}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def traffic_record(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, or
+    None when the kernel source changed since the counters were taken."""
+    src = os.path.join(ROOT, "block_quantized_dsq_b200", "csrc", "gemv.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 4 and parts[0] == kernel and parts[1] == workload:
+            return int(parts[3]) if parts[2] == sha else None
+    return None
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler(threading.Thread):
+    """Polls SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, torch_device: int, period: float = 0.01):
+        super().__init__(daemon=True)
+        self.period = period
+        self.samples = []
+        self.error = None
+        self._stop = threading.Event()
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(torch_device)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report, do not fail the bench
+            self.error = f"{type(e).__name__}: {e}"
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return fn(self.handle)
+
+    def sample(self):
+        self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM), self._reasons()))
+
+    def run(self):
+        if self.handle is None:
+            return
+        while not self._stop.is_set():
+            try:
+                self.sample()
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self.is_alive():
+            self.join()
+        if self.handle is not None and not self.samples:
+            try:
+                self.sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if self.handle is None:
+            return {"error": self.error}
+        busy = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        reasons = set()
+        for _, r in busy:
+            for bit, name in self.REASONS.items():
+                if r & bit and bit != 0x1:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- helpers ----
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def quantized_weights(dsq, qtype, seed, N, K):
+    """Seeded N(0, 0.02^2) fp32 weights, quantized on the device by libdsq."""
+    import torch
+
+    from block_quantized_dsq_b200 import synth
+    w32 = torch.from_numpy(synth.weights(seed, N, K)).cuda()
+    w = torch.empty((N, dsq.dsq_row_bytes(qtype, K)), dtype=torch.uint8, device="cuda")
+    dsq.dsq_quantize_weights(qtype, w32, N, K, w)
+    del w32
+    return w
+
+
+def copies_for(nbytes: int, lo: int = 2) -> int:
+    """Enough copies that the others exceed 3x L2 between two uses of one."""
+    return max(lo, -(-3 * L2_BYTES // max(nbytes, 1)) + 1)
+
+
+def time_calls(fn, n_calls: int, warmup: int = 5):
+    """Device time per call (CUDA events around a batch of eager calls)."""
+    import torch
+    st = torch.cuda.current_stream().cuda_stream
+    for i in range(warmup):
+        fn(i, st)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n_calls):
+        fn(i, st)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / n_calls
+
+
+def time_graph(fn, calls_per_graph: int, replays: int = 5):
+    """Device time per call with the calls captured in a CUDA graph, so host
+    launch cost cannot hide in the figure (CUDA events around the replays)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for i in range(3):
+            fn(i, side.cuda_stream)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream().cuda_stream
+        for i in range(calls_per_graph):
+            fn(i, st)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / (replays * calls_per_graph)
+    del g
+    return t
+
+
+# ------------------------------------------------------------- the bench ---
+def run_dsq(args, world, rank):
+    import torch
+
+    import block_quantized_dsq_b200 as dsq
+    from block_quantized_dsq_b200 import synth
+    from block_quantized_dsq_b200.build import build
+    build()
+    stream = torch.cuda.current_stream().cuda_stream
+    L = dsq.lib()
+    hbm_peak, bf16_peak, bf16_sust, peak_src = measured_peaks()
+
+    # ---- paired workload: weights (rotated copies), 64 fresh activations
+    seeds = synth.SEEDS["paired_q8_0_2x8192x4096"]
+    W0 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w0"], N_PAIR, K_PAIR)
+    W1 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w1"], N_PAIR, K_PAIR)
+    bpc = paired_bytes_per_call()
+    R = copies_for(bpc["gemv"])
+    pairs = [(W0, W1)] + [(W0.clone(), W1.clone()) for _ in range(R - 1)]
+    X_host = __import__("numpy").concatenate(
+        [synth.activations(seeds["x_base"] + i, 1, K_PAIR) for i in range(CALLS)])
+    X = torch.from_numpy(X_host).cuda()
+    xq = torch.empty((CALLS, K_PAIR), dtype=torch.int8, device="cuda")
+    xd = torch.empty((CALLS, K_PAIR // 32), dtype=torch.float32, device="cuda")
+    xs = torch.empty((CALLS, K_PAIR // 32), dtype=torch.int32, device="cuda")
+    Y = torch.empty((CALLS, 2, N_PAIR), dtype=torch.float32, device="cuda")
+    p_x = [X[i].data_ptr() for i in range(CALLS)]
+    p_xq = [xq[i].data_ptr() for i in range(CALLS)]
+    p_xd = [xd[i].data_ptr() for i in range(CALLS)]
+    p_xs = [xs[i].data_ptr() for i in range(CALLS)]
+    p_y0 = [Y[i, 0].data_ptr() for i in range(CALLS)]
+    p_y1 = [Y[i, 1].data_ptr() for i in range(CALLS)]
+    p_w = [(a.data_ptr(), b.data_ptr()) for a, b in pairs]
+    quant, paired = L.dsq_quantize_act_q8, L.dsq_gemv_paired
+
+    def one_call(step, c, evs=None):
+        rc = quant(p_x[c], 1, K_PAIR, p_xq[c], p_xd[c], p_xs[c], stream)
+        w0, w1 = p_w[(step * CALLS + c) % R]
+        if evs is not None:
+            evs[0].record()
+        rc |= paired(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_xq[c], p_xd[c], p_xs[c], p_y0[c], p_y1[c], stream)
+        if evs is not None:
+            evs[1].record()
+        if rc:
+            raise RuntimeError(dsq.dsq_last_error())
+
+    for s in range(args.warmup):
+        for c in range(CALLS):
+            one_call(s, c)
+    torch.cuda.synchronize()
+    assert dsq.dsq_device_status() == 0
+
+    # per-launch events of the dominant kernel, on every 4th call of the
+    # timed region (cheap enough not to slow the launch stream)
+    EV_EVERY = 4
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps * CALLS // EV_EVERY)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = dsq.dsq_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for s in range(args.steps):
+        for c in range(CALLS):
+            one_call(s, c, ev_pairs[(s * CALLS + c) // EV_EVERY] if c % EV_EVERY == 0 else None)
+    t1.record()
+    torch.cuda.synchronize()
+    launches = dsq.dsq_launch_count() - launches0
+    barrier(world)
+    sampler.stop()
+    elapsed = max_over_ranks(world, t0.elapsed_time(t1) / 1e3)
+    assert dsq.dsq_device_status() == 0, "a device wait timed out during the bench"
+    gemv_durs = [a.elapsed_time(b) / 1e3 for a, b in ev_pairs]
+    gemv_avg = statistics.mean(gemv_durs)
+    ms_per_step = elapsed / args.steps * 1e3
+    value = world * args.steps * CALLS * bpc["total"] / elapsed / 1e9
+
+    # ---- end to end through the public API with host buffers
+    X_pin = torch.from_numpy(X_host).pin_memory()
+    Y_pin = torch.empty((CALLS, 2, N_PAIR), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 100))
+
+    def e2e_step(s):
+        X.copy_(X_pin, non_blocking=True)
+        for c in range(CALLS):
+            dsq.dsq_quantize_act_q8(p_x[c], 1, K_PAIR, p_xq[c], p_xd[c], p_xs[c], stream)
+            w0, w1 = p_w[(s * CALLS + c) % R]
+            dsq.dsq_gemv_paired(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_xq[c], p_xd[c], p_xs[c], p_y0[c], p_y1[c],
+                                stream)
+        Y_pin.copy_(Y, non_blocking=True)
+
+    e2e_t = time_calls(lambda s_, st_: e2e_step(s_), e2e_steps, warmup=2)
+    e2e_t = max_over_ranks(world, e2e_t)
+    e2e_value = world * CALLS * bpc["total"] / e2e_t / 1e9
+
+    # ---- the other rows of the path (each its own short timed loop)
+    rows = {}
+    if not args.skip_rows:
+        rows = measure_rows(dsq, L, stream, hbm_peak, bf16_peak)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "weights": "N(0,0.02^2) fp32 quantized to Q8_0 on device, seeds 1/2",
+                   "activations": "N(0,1) fp32, seeds 1000..1063, quantized to Q8 per call",
+                   "l2": f"weights rotated over {R} copies ({R * bpc['gemv'] / 1e6:.0f} MB > 3x L2)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "us_per_call": round(ms_per_step * 1e3 / CALLS, 3),
+        "hbm_frac": round(value / world / hbm_peak, 4),
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (paired Q8_0)",
+                     "achieved": round(bpc["gemv"] / gemv_avg / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(bpc["gemv"] / gemv_avg / 1e9 / hbm_peak, 4),
+                     "traffic": traffic_record("gemv_kernel", "paired_q8_0_2x8192x4096"),
+                     "algorithmic_bytes": bpc["gemv"], "avg_launch_us": round(gemv_avg * 1e6, 3),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                     else "fallback"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": CALLS * K_PAIR * 4,
+                "d2h_bytes_per_step": CALLS * 2 * N_PAIR * 4, "us_per_call": round(e2e_t / CALLS * 1e6, 3)},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(),
+        "rows": rows,
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        result["cpu_baseline"] = cpu_baseline(pairs[0], X_host, args.cpu_seconds)
+    return result
+
+
+def measure_rows(dsq, L, stream, hbm_peak, bf16_peak):
+    """µs/call and GB/s (or TFLOP/s) for every other step of the path."""
+    import torch
+
+    from block_quantized_dsq_b200 import synth
+    rows = {}
+
+    def act(seed, M, K):
+        x = torch.from_numpy(synth.activations(seed, M, K)).cuda()
+        xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        xd = torch.empty((M, K // 32), dtype=torch.float32, device="cuda")
+        xs = torch.empty((M, K // 32), dtype=torch.int32, device="cuda")
+        dsq.dsq_quantize_act_q8(x, M, K, xq, xd, xs)
+        return x, xq, xd, xs
+
+    # activation prequantization, one decode row of K = 4096
+    x, xq, xd, xs = act(101, 1, 4096)
+    px, pq, pd, ps = x.data_ptr(), xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
+    t = time_graph(lambda i, st: L.dsq_quantize_act_q8(px, 1, 4096, pq, pd, ps, st), 500)
+    rows["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 3),
+                                      "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 2)}
+
+    def gemv_row(name, qtype, N, K, seed, xseed, G=1):
+        w = quantized_weights(dsq, qtype, seed, G * N, K)
+        nbytes = w.numel()
+        R = copies_for(nbytes)
+        ws = [w] + [w.clone() for _ in range(R - 1)]
+        ptrs = [c.data_ptr() for c in ws]
+        x, xq, xd, xs = act(xseed, G, K)
+        y = torch.empty((G, N), dtype=torch.float32, device="cuda")
+        pq, pd, ps, py = xq.data_ptr(), xd.data_ptr(), xs.data_ptr(), y.data_ptr()
+        if G > 1:
+            fn = lambda i, st: L.dsq_gemv_grouped(qtype, ptrs[i % R], G, N, K, pq, pd, ps, py, st)  # noqa: E731
+        elif qtype == dsq.DSQ_Q8_0:
+            fn = lambda i, st: L.dsq_gemv_q8_0(ptrs[i % R], N, K, pq, pd, py, st)  # noqa: E731
+        else:
+            fn = lambda i, st: L.dsq_gemv_q4_k(ptrs[i % R], N, K, pq, pd, ps, py, st)  # noqa: E731
+        t = time_graph(fn, R * max(1, 200 // R))
+        alg = nbytes + G * (K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1)) + G * N * 4
+        gbs = alg / t / 1e9
+        rows[name] = {"us_per_call": round(t * 1e6, 3), "GB/s": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
+                      "algorithmic_bytes": alg, "weight_copies": R}
+        del ws
+
+    seeds = synth.SEEDS
+    gemv_row("gemv_q8_0_1024x1024", dsq.DSQ_Q8_0, 1024, 1024, seeds["gemv_q8_0_1024"]["w"],
+             seeds["gemv_q8_0_1024"]["x"])
+    gemv_row("gemv_q4_k_4096x4096", dsq.DSQ_Q4_K, 4096, 4096, seeds["gemv_q4_k_4096"]["w"],
+             seeds["gemv_q4_k_4096"]["x"])
+    gemv_row("grouped_q8_0_8x1024x4096", dsq.DSQ_Q8_0, 1024, 4096, seeds["grouped_q8_0_8x1024x4096"]["w_base"],
+             seeds["grouped_q8_0_8x1024x4096"]["x_base"], G=8)
+
+    # prefill dequant-GEMM sweep
+    K = 4096
+    for qtype, N, tag in ((dsq.DSQ_Q4_K, 4096, "q4_k_n4096"), (dsq.DSQ_Q8_0, 8192, "q8_0_n8192")):
+        w = quantized_weights(dsq, qtype, seeds["prefill"]["w_q4_k" if qtype == dsq.DSQ_Q4_K else "w_q8_0"], N, K)
+        ws = [w, w.clone()]
+        for M in (128, 512, 2048):
+            x = torch.from_numpy(synth.activations(seeds["prefill"]["x_base"] + M, M, K)).cuda()
+            y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+            nb = dsq.dsq_prefill_workspace_bytes(qtype, N, K, M)
+            wsp = torch.empty(nb, dtype=torch.uint8, device="cuda")
+            pw = [c.data_ptr() for c in ws]
+            px, py, pws = x.data_ptr(), y.data_ptr(), wsp.data_ptr()
+            t = time_graph(lambda i, st: L.dsq_gemm_prefill(qtype, pw[i % 2], N, K, px, M, py, pws, nb, st), 10, 3)
+            tf = 2.0 * M * N * K / t / 1e12
+            rows[f"prefill_{tag}_m{M}"] = {"us_per_call": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
+                                           "bf16_peak_frac": round(tf / bf16_peak, 4)}
+    assert dsq.dsq_device_status() == 0
+    return rows
+
+
+def cpu_baseline(pair, X_host, budget_s: float):
+    """The CPU oracle (single-threaded C) on a bounded sample of the workload:
+    as many of the 64 paired calls as fit in the time budget."""
+    import numpy as np
+
+    import oracle as ref
+    w0, w1 = pair[0].cpu().numpy(), pair[1].cpu().numpy()
+    bpc = paired_bytes_per_call()
+    t0 = time.perf_counter()
+    n = 0
+    while n < CALLS:
+        xq, xd, xs = ref.quantize_act_q8(X_host[n:n + 1])
+        ref.gemv(8, w0, K_PAIR, xq, xd, xs)
+        ref.gemv(8, w1, K_PAIR, xq, xd, xs)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(n * bpc["total"] / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of the 64 paired calls (oracle act-quantize + two integer-form GEMVs), {dt:.1f} s",
+            "cpu": platform.processor() or platform.machine(), "host_cores": os.cpu_count()}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: same metric and workload, a bounded
+    sample per step, host cores only (rank 0)."""
+    import numpy as np
+
+    import oracle as ref
+    from block_quantized_dsq_b200 import synth
+    seeds = synth.SEEDS["paired_q8_0_2x8192x4096"]
+    w0 = ref.quantize(8, synth.weights(seeds["w0"], N_PAIR, K_PAIR))
+    w1 = ref.quantize(8, synth.weights(seeds["w1"], N_PAIR, K_PAIR))
+    X = np.concatenate([synth.activations(seeds["x_base"] + i, 1, K_PAIR) for i in range(CALLS)])
+    per_step = 2      # calls per step: bounded so the whole run ends within minutes
+    bpc = paired_bytes_per_call()
+
+    def step(s):
+        for j in range(per_step):
+            c = (s * per_step + j) % CALLS
+            xq, xd, xs = ref.quantize_act_q8(X[c:c + 1])
+            ref.gemv(8, w0, K_PAIR, xq, xd, xs)
+            ref.gemv(8, w1, K_PAIR, xq, xd, xs)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(s)
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step * bpc["total"] / dt / 1e9
+    sample = f"{per_step} of the 64 paired calls per step (oracle act-quantize + two integer-form GEMVs)"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "host cores, rank 0"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["dsq", "reference"], default="dsq")
+    ap.add_argument("--skip-rows", action="store_true", help="only the headline workload")
+    ap.add_argument("--skip-cpu", action="store_true", help="no CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        args.steps = 5 if args.steps is None else args.steps
+        args.warmup = 1 if args.warmup is None else args.warmup
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        print(json.dumps(run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), 0)))
+        return 0
+    args.steps = 200 if args.steps is None else args.steps
+    args.warmup = 5 if args.warmup is None else args.warmup
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, _ = dist_setup()
+    try:
+        res = run_dsq(args, world, rank)
+        if rank == 0:
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,44 @@
+// dsq_host.h -- host-side plumbing shared by the libdsq entry points:
+// per-thread error text, argument checks, the per-device status word and the
+// launch counter.
+#pragma once
+
+#include <cstdint>
+#include <cstdio>
+#include <cuda_runtime.h>
+
+#include "../../include/dsq.h"
+#include "dsq_device.cuh"
+
+namespace dsq {
+
+// Records a message for dsq_last_error() and returns `code`.
+int fail(int code, const char *fmt, ...);
+
+// Checks the current device once (compute capability 10.0) and returns its
+// status-word pointer and SM count through the out-parameters.
+int device_ready(uint32_t **status_word, int *num_sms);
+
+// Wait control for kernels launched now (status word + current limit).
+int wait_ctl(WaitCtl *ctl, int *num_sms);
+
+// After a launch: maps a launch error to DSQ_ERR_LAUNCH and counts launches.
+int after_launch(const char *what, int n_kernels = 1);
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
+// the first call on a device configures it; later calls (for example inside
+// a CUDA graph capture) only launch.
+int set_smem_once(const void *kernel, int bytes, const char *what);
+
+inline bool aligned(const void *p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace dsq
+
+#define DSQ_REQUIRE(cond, code, ...)              \
+  do {                                            \
+    if (!(cond)) return ::dsq::fail((code), __VA_ARGS__); \
+  } while (0)

@@ -1,0 +1,458 @@
+// gemv.cu -- decode GEMV with the activation prequantized to Q8 per 32-block:
+// regular, paired (two weights sharing one activation) and grouped low-rank
+// attention-output (G independent weight/activation pairs), for Q8_0 and
+// Q4_K weights.
+//
+// Sources: "ROCm: restore DeepSeek V4 Flash decode performance and Q4 SSD
+// streaming" (antirez/ds4 PR #623) -- Summary (prequantized Q8 decode for
+// regular, paired and low-rank attention-output projections) and the
+// per-stage timing comment (matmul_q8_0_tensor, matmul_q8_0_pair_tensor,
+// attention_output_low_q8_tensor; the fast kernels run a warp per output
+// row, the slow ones a 256-thread block per row); "Support AProjQ4 GGUFs"
+// (antirez/ds4 PR #621) for the Q4_K projections; "DeepSeek V4"
+// (ggml-org/llama.cpp PR #24162) for the [4096, 1024, 8] grouped layout.
+//
+// B200 design (HBM-bound weight stream):
+//  * A CTA owns a contiguous, balanced range of weight rows.  Each warp runs
+//    its own ring of shared-memory slots, filled by cp.async.bulk (one
+//    elected lane, completion on an mbarrier, L2 evict-first): deep bytes
+//    in flight per SM without register staging, perfectly coalesced.
+//  * A row is split into 256-element units (8 Q8_0 blocks = 272 B, or one
+//    Q4_K super-block = 144 B, both 16-byte multiples).  G lanes share a row
+//    (G = units per row rounded up to a power of two, at most 32), so a warp
+//    holds 32/G rows per slot and lane j takes units j, j+G, ...
+//  * The lane's 256-element activation slice (xq, xd, xs) is cached in
+//    registers for as long as its (group, unit) does not change -- for
+//    K <= 8192 that is every row the warp touches.
+//  * Per 32-block: 8 dp4a give the exact int32 dot; the block term is
+//    (d_w * xd) * isum in fp32; lanes reduce with xor-shuffles; one store
+//    per row.  Rows whose byte length is not a multiple of 16 (Q8_0 with
+//    K % 256 != 0) take a plain warp-per-row kernel instead.
+#include "../../include/dsq_test.h"
+#include "dsq_host.h"
+
+namespace dsq {
+namespace {
+
+struct Seg {
+  const uint8_t *w;
+  float *y;
+  int64_t rows;
+};
+
+struct GemvArgs {
+  Seg seg[2];
+  int64_t rows0;        // rows of seg[0]; seg[1] follows in the virtual row space
+  int64_t total_rows;   // rows0 + rows of seg[1]
+  int64_t group_rows;   // rows per activation group inside a segment
+  const int8_t *xq;
+  const float *xd;
+  const int32_t *xs;
+  int64_t K;
+  int64_t row_bytes;
+  int nunits;           // K / 256 (fast kernel)
+  int warps;            // warps per CTA
+  int stages;           // ring slots per warp
+  int slot_bytes;       // rows-per-slot * row_bytes
+  WaitCtl wait;
+  int32_t *isum;        // test hook: per-block int32 sums (NULL in production)
+};
+
+template <int TYPE> struct Unit;
+template <> struct Unit<DSQ_Q8_0> { static constexpr int kBytes = 272; };
+template <> struct Unit<DSQ_Q4_K> { static constexpr int kBytes = 144; };
+
+__device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu))); }
+__device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))); }
+
+// Activation slice of one 256-element unit, held in registers.
+struct ActSlice {
+  uint32_t q[64];   // 256 int8 codes
+  float d[8];       // 8 block scales
+  int32_t s[8];     // 8 block code sums (Q4_K only)
+};
+
+template <int TYPE>
+__device__ __forceinline__ void load_act(ActSlice &act, const int8_t *xq, const float *xd, const int32_t *xs) {
+  const uint4 *q4 = reinterpret_cast<const uint4 *>(xq);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint4 v = __ldg(q4 + i);
+    act.q[4 * i + 0] = v.x; act.q[4 * i + 1] = v.y; act.q[4 * i + 2] = v.z; act.q[4 * i + 3] = v.w;
+  }
+  const float4 *d4 = reinterpret_cast<const float4 *>(xd);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float4 v = __ldg(d4 + i);
+    act.d[4 * i + 0] = v.x; act.d[4 * i + 1] = v.y; act.d[4 * i + 2] = v.z; act.d[4 * i + 3] = v.w;
+  }
+  if (TYPE == DSQ_Q4_K) {
+    const int4 *s4 = reinterpret_cast<const int4 *>(xs);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int4 v = __ldg(s4 + i);
+      act.s[4 * i + 0] = v.x; act.s[4 * i + 1] = v.y; act.s[4 * i + 2] = v.z; act.s[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// One Q8_0 unit (8 blocks, 272 bytes = 68 words) against its activation
+// slice.  Block b starts at byte 34b: for even b the scale is the low half of
+// word 17b/2 and the codes start two bytes later (realigned with a funnel
+// shift); for odd b the scale is the high half of word (17b-1)/2 and the
+// codes are word-aligned.
+template <bool ISUM>
+__device__ __forceinline__ float unit_q8_0(const uint8_t *p, const ActSlice &act, int32_t *isum_out) {
+  uint32_t w[68];
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < 17; ++i) {
+    const uint4 v = p4[i];
+    w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  float acc = 0.0f;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    int32_t s = 0;
+    float dw;
+    if ((b & 1) == 0) {
+      const int a = 17 * b / 2;
+      dw = half_lo(w[a]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s = __dp4a(static_cast<int>(__funnelshift_r(w[a + i], w[a + i + 1], 16)),
+                                             static_cast<int>(act.q[8 * b + i]), s);
+    } else {
+      const int a = (17 * b - 1) / 2;
+      dw = half_hi(w[a]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s = __dp4a(static_cast<int>(w[a + 1 + i]), static_cast<int>(act.q[8 * b + i]), s);
+    }
+    if (ISUM) isum_out[b] = s;
+    acc += __fmul_rn(__fmul_rn(dw, act.d[b]), static_cast<float>(s));
+  }
+  return acc;
+}
+
+// One Q4_K super-block (144 bytes = 36 words): word 0 = d | dmin << 16,
+// words 1..3 = the 12 scale bytes, words 4..35 = the 128 nibble bytes.
+template <bool ISUM>
+__device__ __forceinline__ float unit_q4_k(const uint8_t *p, const ActSlice &act, int32_t *isum_out) {
+  uint32_t w[36];
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < 9; ++i) {
+    const uint4 v = p4[i];
+    w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  const float d = half_lo(w[0]), dmin = half_hi(w[0]);
+  const uint32_t s0 = w[1], s1 = w[2], s2 = w[3];
+  // bytes j of (scA, mA) are (sc_j, m_j) for j < 4; of (scB, mB) for j >= 4
+  const uint32_t scA = s0 & 0x3f3f3f3fu;
+  const uint32_t mA = s1 & 0x3f3f3f3fu;
+  const uint32_t scB = (s2 & 0x0f0f0f0fu) | ((s0 >> 2) & 0x30303030u);
+  const uint32_t mB = ((s2 >> 4) & 0x0f0f0f0fu) | ((s1 >> 2) & 0x30303030u);
+  float acc = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t scw = j < 4 ? scA : scB, mw = j < 4 ? mA : mB;
+    const int sh = 8 * (j & 3);
+    const float sc = static_cast<float>((scw >> sh) & 0xffu);
+    const float m = static_cast<float>((mw >> sh) & 0xffu);
+    int32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t byte4 = w[4 + 8 * (j >> 1) + i];
+      const uint32_t nib = (j & 1) ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
+      s = __dp4a(static_cast<int>(nib), static_cast<int>(act.q[8 * j + i]), s);
+    }
+    if (ISUM) isum_out[j] = s;
+    const float t = __fmul_rn(__fmul_rn(d, sc), static_cast<float>(s));
+    const float u = __fmul_rn(__fmul_rn(dmin, m), static_cast<float>(act.s[j]));
+    acc += __fmul_rn(act.d[j], __fsub_rn(t, u));
+  }
+  return acc;
+}
+
+// Virtual row r -> (segment, row within segment).
+__device__ __forceinline__ void locate(const GemvArgs &a, int64_t r, int &seg, int64_t &local) {
+  if (r < a.rows0) { seg = 0; local = r; } else { seg = 1; local = r - a.rows0; }
+}
+
+// Issue the bulk copy of virtual rows [ra, rb) into a slot (split when the
+// range crosses from segment 0 into segment 1).
+__device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_t rb, uint8_t *dst, uint64_t *bar,
+                                           uint64_t policy) {
+  const uint32_t total = static_cast<uint32_t>((rb - ra) * a.row_bytes);
+  mbar_arrive_expect_tx(bar, total);
+  if (rb <= a.rows0) {
+    bulk_g2s(dst, a.seg[0].w + ra * a.row_bytes, total, bar, policy);
+  } else if (ra >= a.rows0) {
+    bulk_g2s(dst, a.seg[1].w + (ra - a.rows0) * a.row_bytes, total, bar, policy);
+  } else {
+    const uint32_t n0 = static_cast<uint32_t>((a.rows0 - ra) * a.row_bytes);
+    bulk_g2s(dst, a.seg[0].w + ra * a.row_bytes, n0, bar, policy);
+    bulk_g2s(dst + n0, a.seg[1].w, total - n0, bar, policy);
+  }
+}
+
+template <int TYPE, int G, bool ISUM>
+__global__ void __launch_bounds__(256, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
+  constexpr int RPC = 32 / G;  // rows per slot
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int W = a.warps, S = a.stages;
+  const int64_t r0 = a.total_rows * blockIdx.x / gridDim.x;
+  const int64_t r1 = a.total_rows * (blockIdx.x + 1) / gridDim.x;
+  const int64_t nchunks = (r1 - r0 + RPC - 1) / RPC;
+  const int64_t mine = nchunks > warp ? (nchunks - warp + W - 1) / W : 0;
+  uint8_t *ring = smem + static_cast<size_t>(warp) * S * a.slot_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + static_cast<size_t>(W) * S * a.slot_bytes) + warp * S;
+  if (mine == 0) return;
+
+  const uint64_t policy = l2_policy_evict_first();
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+    for (int64_t k = 0; k < mine && k < S; ++k) {
+      const int64_t c = warp + k * W;
+      const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
+      issue_rows(a, ra, rb, ring + k * a.slot_bytes, &bars[k], policy);
+    }
+  }
+  __syncwarp();
+
+  const int sub = lane / G, j = lane % G;
+  ActSlice act;
+  int64_t cached = -1;  // (group * nunits + unit) currently in registers
+  for (int64_t k = 0; k < mine; ++k) {
+    const int slot = static_cast<int>(k % S);
+    const uint32_t parity = static_cast<uint32_t>((k / S) & 1);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
+    if (!ok) {
+      if (lane == 0) {
+        record_timeout(a.wait);
+        for (int64_t kk = k; kk < mine && kk < k + S; ++kk)
+          mbar_wait_for(&bars[kk % S], static_cast<uint32_t>((kk / S) & 1), kDrainLimitNs);
+      }
+      __syncwarp();
+      return;
+    }
+    const int64_t c = warp + k * W;
+    const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
+    const int64_t row = ra + sub;
+    float acc = 0.0f;
+    if (row < rb) {
+      int seg;
+      int64_t local;
+      locate(a, row, seg, local);
+      const int64_t group = local / a.group_rows;
+      const uint8_t *rowp = ring + static_cast<size_t>(slot) * a.slot_bytes + static_cast<size_t>(sub) * a.row_bytes;
+      for (int u = j; u < a.nunits; u += G) {
+        const int64_t key = group * a.nunits + u;
+        if (key != cached) {
+          const int64_t e0 = group * a.K + static_cast<int64_t>(u) * 256;
+          load_act<TYPE>(act, a.xq + e0, a.xd + e0 / 32, TYPE == DSQ_Q4_K ? a.xs + e0 / 32 : nullptr);
+          cached = key;
+        }
+        int32_t is[8];
+        if (TYPE == DSQ_Q8_0)
+          acc += unit_q8_0<ISUM>(rowp + static_cast<size_t>(u) * Unit<TYPE>::kBytes, act, is);
+        else
+          acc += unit_q4_k<ISUM>(rowp + static_cast<size_t>(u) * Unit<TYPE>::kBytes, act, is);
+        if (ISUM) {
+#pragma unroll
+          for (int b = 0; b < 8; ++b) a.isum[row * (a.K / 32) + u * 8 + b] = is[b];
+        }
+      }
+    }
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (row < rb && j == 0) {
+      int seg;
+      int64_t local;
+      locate(a, row, seg, local);
+      a.seg[seg].y[local] = acc;
+    }
+    __syncwarp();
+    if (lane == 0 && k + S < mine) {
+      fence_proxy_async_smem();
+      const int64_t c2 = warp + (k + S) * W;
+      const int64_t ra2 = r0 + c2 * RPC, rb2 = min(ra2 + RPC, r1);
+      issue_rows(a, ra2, rb2, ring + static_cast<size_t>(slot) * a.slot_bytes, &bars[slot], policy);
+    }
+  }
+}
+
+// Rows whose length is not a multiple of 16 bytes (Q8_0, K % 256 != 0): one
+// warp per row, lanes over 34-byte blocks read with 16-bit loads.
+template <bool ISUM>
+__global__ void __launch_bounds__(256) gemv_q8_0_rowwise_kernel(const __grid_constant__ GemvArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nb = a.K / 32;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < a.total_rows;
+       row += static_cast<int64_t>(gridDim.x) * 8) {
+    int seg;
+    int64_t local;
+    locate(a, row, seg, local);
+    const int64_t group = local / a.group_rows;
+    const uint8_t *rowp = a.seg[seg].w + local * a.row_bytes;
+    float acc = 0.0f;
+    for (int64_t b = lane; b < nb; b += 32) {
+      const uint16_t *h = reinterpret_cast<const uint16_t *>(rowp + b * 34);
+      const float dw = __half2float(__ushort_as_half(h[0]));
+      const uint32_t *xq = reinterpret_cast<const uint32_t *>(a.xq + group * a.K + b * 32);
+      int32_t s = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t qw = static_cast<uint32_t>(h[1 + 2 * i]) | (static_cast<uint32_t>(h[2 + 2 * i]) << 16);
+        s = __dp4a(static_cast<int>(qw), static_cast<int>(__ldg(xq + i)), s);
+      }
+      if (ISUM) a.isum[row * nb + b] = s;
+      acc += __fmul_rn(__fmul_rn(dw, __ldg(a.xd + group * nb + b)), static_cast<float>(s));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) a.seg[seg].y[local] = acc;
+  }
+}
+
+constexpr int kMaxWarps = 8;
+constexpr size_t kSmemBudget = 220 * 1024;
+
+template <int TYPE, int G, bool ISUM>
+int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
+  constexpr int RPC = 32 / G;
+  const size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
+                      static_cast<size_t>(a.warps) * a.stages * sizeof(uint64_t);
+  auto kern = gemv_kernel<TYPE, G, ISUM>;
+  const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
+  if (rc != DSQ_OK) return rc;
+  const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
+  const unsigned grid = static_cast<unsigned>(chunks < num_sms ? chunks : num_sms);
+  kern<<<grid, a.warps * 32, smem, stream>>>(a);
+  return after_launch("gemv");
+}
+
+template <int TYPE, bool ISUM>
+int dispatch_g(GemvArgs &a, int G, int num_sms, cudaStream_t stream) {
+  switch (G) {
+    case 1: return launch_fast<TYPE, 1, ISUM>(a, num_sms, stream);
+    case 2: return launch_fast<TYPE, 2, ISUM>(a, num_sms, stream);
+    case 4: return launch_fast<TYPE, 4, ISUM>(a, num_sms, stream);
+    case 8: return launch_fast<TYPE, 8, ISUM>(a, num_sms, stream);
+    case 16: return launch_fast<TYPE, 16, ISUM>(a, num_sms, stream);
+    default: return launch_fast<TYPE, 32, ISUM>(a, num_sms, stream);
+  }
+}
+
+// Validates and launches one GEMV over up to two segments.
+int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int64_t groups, int64_t K,
+             const int8_t *xq, const float *xd, const int32_t *xs, int32_t *isum, cudaStream_t stream) {
+  DSQ_REQUIRE(type == DSQ_Q8_0 || type == DSQ_Q4_K, DSQ_ERR_INVALID_ARG, "%s: unsupported type %d", name, type);
+  DSQ_REQUIRE(K > 0 && s0.rows >= 0 && s1.rows >= 0, DSQ_ERR_INVALID_ARG, "%s: negative size", name);
+  const size_t rb = dsq_row_bytes(type, K);
+  DSQ_REQUIRE(rb != 0, DSQ_ERR_SHAPE, "%s: K=%lld is not a multiple of %d", name, (long long)K,
+              type == DSQ_Q8_0 ? 32 : 256);
+  DSQ_REQUIRE(K <= (int64_t(1) << 20) && s0.rows + s1.rows <= (int64_t(1) << 31), DSQ_ERR_SHAPE,
+              "%s: size out of range (K <= 2^20, rows <= 2^31)", name);
+  const int64_t total = s0.rows + s1.rows;
+  if (total == 0) return DSQ_OK;
+  DSQ_REQUIRE(xq && xd && (type == DSQ_Q8_0 || xs), DSQ_ERR_INVALID_ARG, "%s: null activation pointer", name);
+  DSQ_REQUIRE((s0.rows == 0 || (s0.w && s0.y)) && (s1.rows == 0 || (s1.w && s1.y)), DSQ_ERR_INVALID_ARG,
+              "%s: null weight/output pointer", name);
+  DSQ_REQUIRE(aligned(xq, 16) && aligned(xd, 16) && (!xs || aligned(xs, 16)), DSQ_ERR_ALIGNMENT,
+              "%s: xq/xd/xs must be 16-byte aligned", name);
+  DSQ_REQUIRE((s0.rows == 0 || (aligned(s0.w, 16) && aligned(s0.y, 4))) &&
+                  (s1.rows == 0 || (aligned(s1.w, 16) && aligned(s1.y, 4))),
+              DSQ_ERR_ALIGNMENT, "%s: weights must be 16-byte and outputs 4-byte aligned", name);
+  (void)groups;
+  WaitCtl ctl;
+  int num_sms = 0;
+  int rc = wait_ctl(&ctl, &num_sms);
+  if (rc != DSQ_OK) return rc;
+
+  GemvArgs a{};
+  a.seg[0] = s0;
+  a.seg[1] = s1;
+  a.rows0 = s0.rows;
+  a.total_rows = total;
+  a.group_rows = group_rows;
+  a.xq = xq;
+  a.xd = xd;
+  a.xs = xs;
+  a.K = K;
+  a.row_bytes = static_cast<int64_t>(rb);
+  a.wait = ctl;
+  a.isum = isum;
+
+  if (rb % 16 != 0) {  // Q8_0 with K % 256 != 0
+    const int64_t blocks = (total + 7) / 8;
+    const unsigned grid = static_cast<unsigned>(blocks < 4 * num_sms ? blocks : 4 * num_sms);
+    if (isum) gemv_q8_0_rowwise_kernel<true><<<grid, 256, 0, stream>>>(a);
+    else gemv_q8_0_rowwise_kernel<false><<<grid, 256, 0, stream>>>(a);
+    return after_launch(name);
+  }
+  a.nunits = static_cast<int>(K / 256);
+  int G = 1;
+  while (G < a.nunits && G < 32) G <<= 1;
+  a.slot_bytes = static_cast<int>((32 / G) * rb);
+  a.warps = kMaxWarps;
+  while (a.warps > 1 && static_cast<size_t>(a.warps) * 2 * a.slot_bytes > kSmemBudget) a.warps >>= 1;
+  DSQ_REQUIRE(static_cast<size_t>(a.warps) * 2 * a.slot_bytes <= kSmemBudget, DSQ_ERR_SHAPE,
+              "%s: K=%lld rows do not fit the shared-memory pipeline", name, (long long)K);
+  a.stages = static_cast<int>(kSmemBudget / (static_cast<size_t>(a.warps) * a.slot_bytes));
+  if (a.stages > 6) a.stages = 6;
+  if (type == DSQ_Q8_0)
+    return isum ? dispatch_g<DSQ_Q8_0, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q8_0, false>(a, G, num_sms, stream);
+  return isum ? dispatch_g<DSQ_Q4_K, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q4_K, false>(a, G, num_sms, stream);
+}
+
+constexpr int64_t kOneGroup = int64_t(1) << 62;
+
+}  // namespace
+}  // namespace dsq
+
+extern "C" {
+
+int dsq_gemv_q8_0(const void *w, int64_t N, int64_t K, const int8_t *xq, const float *xd, float *y, void *stream) {
+  using namespace dsq;
+  return run_gemv("dsq_gemv_q8_0", DSQ_Q8_0, Seg{static_cast<const uint8_t *>(w), y, N}, Seg{nullptr, nullptr, 0},
+                  kOneGroup, 1, K, xq, xd, nullptr, nullptr, as_stream(stream));
+}
+
+int dsq_gemv_q4_k(const void *w, int64_t N, int64_t K, const int8_t *xq, const float *xd, const int32_t *xs,
+                  float *y, void *stream) {
+  using namespace dsq;
+  return run_gemv("dsq_gemv_q4_k", DSQ_Q4_K, Seg{static_cast<const uint8_t *>(w), y, N}, Seg{nullptr, nullptr, 0},
+                  kOneGroup, 1, K, xq, xd, xs, nullptr, as_stream(stream));
+}
+
+int dsq_gemv_paired(int type, const void *w0, int64_t N0, const void *w1, int64_t N1, int64_t K, const int8_t *xq,
+                    const float *xd, const int32_t *xs, float *y0, float *y1, void *stream) {
+  using namespace dsq;
+  return run_gemv("dsq_gemv_paired", type, Seg{static_cast<const uint8_t *>(w0), y0, N0},
+                  Seg{static_cast<const uint8_t *>(w1), y1, N1}, kOneGroup, 1, K, xq, xd, xs, nullptr,
+                  as_stream(stream));
+}
+
+int dsq_gemv_grouped(int type, const void *w, int64_t G, int64_t N, int64_t K, const int8_t *xq, const float *xd,
+                     const int32_t *xs, float *y, void *stream) {
+  using namespace dsq;
+  DSQ_REQUIRE(G >= 0 && N >= 0, DSQ_ERR_INVALID_ARG, "dsq_gemv_grouped: G=%lld N=%lld", (long long)G, (long long)N);
+  DSQ_REQUIRE(G <= (int64_t(1) << 20), DSQ_ERR_SHAPE, "dsq_gemv_grouped: G out of range");
+  if (G == 0 || N == 0) return dsq::run_gemv("dsq_gemv_grouped", type, Seg{nullptr, nullptr, 0}, Seg{nullptr, nullptr, 0},
+                                             1, 0, K, xq, xd, xs, nullptr, as_stream(stream));
+  return run_gemv("dsq_gemv_grouped", type, Seg{static_cast<const uint8_t *>(w), y, G * N}, Seg{nullptr, nullptr, 0}, N,
+                  G, K, xq, xd, xs, nullptr, as_stream(stream));
+}
+
+int dsq_test_block_sums(int type, const void *w, int64_t N, int64_t K, const int8_t *xq, const float *xd,
+                        const int32_t *xs, float *y, int32_t *isum, void *stream) {
+  using namespace dsq;
+  DSQ_REQUIRE(isum != nullptr || N == 0, DSQ_ERR_INVALID_ARG, "dsq_test_block_sums: null isum");
+  DSQ_REQUIRE(aligned(isum, 4), DSQ_ERR_ALIGNMENT, "dsq_test_block_sums: isum alignment");
+  return run_gemv("dsq_test_block_sums", type, Seg{static_cast<const uint8_t *>(w), y, N}, Seg{nullptr, nullptr, 0},
+                  kOneGroup, 1, K, xq, xd, xs, isum, as_stream(stream));
+}
+
+}  // extern "C"

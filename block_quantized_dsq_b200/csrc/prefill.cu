@@ -1,0 +1,649 @@
+// prefill.cu -- prefill projection: dequantize Q8_0 / Q4_K weights into a
+// dense tensor-core GEMM, Y[M][N] = X[M][K] * deq(W)^T.
+//
+// Source: "Support AProjQ4 GGUFs: Q4_K dense attention projections"
+// (antirez/ds4 PR #621), GB10 test report (Q4_K prefill fell to 54.6 t/s
+// until a dequant + GEMM prefill path existed; the tester calls that path
+// the deciding factor) and the consolidated results (grouped attention-A
+// prefill).  The pages give no kernel; this is a B200-first design.
+//
+// Numerics: 16-bit float operands, fp32 accumulation.  Each activation row
+// is scaled by an exact power of two 2^s_m (its largest magnitude lands in
+// [2^14, 2^15)) and rounded to binary16; each weight element is dequantized
+// in fp32 ((d*q) for Q8_0, (d*sc)*q - dmin*m for Q4_K) and rounded to
+// binary16; the fp32 dot is scaled back by 2^-s_m.  binary16 (10 explicit
+// mantissa bits) keeps the operand rounding at ~3e-4 relative L2 on this
+// workload; bfloat16 operands would give ~2.3e-3, above the 2e-3 bar.
+//
+// Kernel (one CTA per 128 weight rows x TN tokens x K-split):
+//  * the weight tile is the MMA's A operand (M = 128 rows of W), the
+//    activation tile its B operand (N = TN tokens) -- "swap AB", so small
+//    token counts still use a full 128-row MMA and the weight stream stays
+//    HBM-efficient down to one token;
+//  * warp 0: TMA producer of the activation tiles (fp16, 128-byte swizzle);
+//  * warp 1: allocates TMEM and issues tcgen05.mma (kind::f16, fp32
+//    accumulate in TMEM), releasing smem stages with tcgen05.commit;
+//  * warps 2-5: each thread owns one weight row: it streams the row's raw
+//    blocks from global memory (one 256-element unit ahead), dequantizes 64
+//    elements per stage into the 128-byte-swizzled K-major layout the MMA
+//    reads, then runs the epilogue (tcgen05.ld -> scale by 2^-s_m -> global,
+//    coalesced across the 32 rows of a warp);
+//  * every wait is bounded; an expired wait records a timeout, stops every
+//    role, drains copies and MMAs in flight, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "../../include/dsq_test.h"
+#include "dsq_host.h"
+
+namespace dsq {
+namespace {
+
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBK = 64;           // K elements per pipeline stage
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kAStageBytes = kBM * kBK * 2;   // 16 KB
+
+struct PrefillArgs {
+  const uint8_t *w;
+  int64_t N, K, M;
+  int64_t row_bytes;
+  const int32_t *shift;   // [M] activation row shifts
+  float *y;               // [M][N], or [splits][M][N] partials
+  int units_per_split;    // 256-element units of K per split
+  int splits;
+  int tn;                 // tokens per tile (MMA N): 32..256, multiple of 32
+  int stages;
+  int tmem_cols;
+  WaitCtl wait;
+};
+
+// ---------------------------------------------------------------- dequant --
+// 256-element unit of one weight row in registers: Q8_0 = 8 blocks (272 B),
+// Q4_K = one super-block (144 B).
+template <int TYPE> struct RawUnit;
+template <> struct RawUnit<DSQ_Q8_0> { static constexpr int kVecs = 17; uint4 v[17]; };
+template <> struct RawUnit<DSQ_Q4_K> { static constexpr int kVecs = 9; uint4 v[9]; };
+
+template <int TYPE>
+__device__ __forceinline__ void load_unit(RawUnit<TYPE> &u, const uint8_t *p) {
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < RawUnit<TYPE>::kVecs; ++i) u.v[i] = __ldg(p4 + i);
+}
+
+template <int TYPE>
+__device__ __forceinline__ uint32_t word_of(const RawUnit<TYPE> &u, int i) {
+  const uint4 &v = u.v[i >> 2];
+  return (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t b) { return *reinterpret_cast<__half2 *>(&b); }
+
+// 4 int8 codes (one word) times an fp16 scale -> 4 binary16 values (2 words).
+// A biased byte u = q + 128 placed under exponent byte 0x64 is the half
+// 1024 + u; subtracting 1152 gives q exactly; the product d*q (exact in
+// fp32: 11 x 7 significant bits) is then rounded once to binary16 by the
+// half multiply -- the same value as fp16_rne(float(d) * q).
+__device__ __forceinline__ void q8x4_to_h(uint32_t qw, __half2 d2, uint32_t &o0, uint32_t &o1) {
+  const uint32_t b = qw ^ 0x80808080u;
+  const __half2 bias = __half2half2(__ushort_as_half(0x6480));   // 1152.0
+  const __half2 lo = __hsub2(bits_h2(__byte_perm(b, 0x64646464u, 0x5140)), bias);
+  const __half2 hi = __hsub2(bits_h2(__byte_perm(b, 0x64646464u, 0x7362)), bias);
+  o0 = h2_bits(__hmul2_rn(lo, d2));
+  o1 = h2_bits(__hmul2_rn(hi, d2));
+}
+
+// Q8_0: piece p (64 elements = blocks 2p, 2p+1) as 8 chunks of 8 halves.
+__device__ __forceinline__ void piece_q8_0(const RawUnit<DSQ_Q8_0> &u, int p, uint32_t (&out)[32]) {
+#pragma unroll
+  for (int half_ = 0; half_ < 2; ++half_) {
+    const int b = 2 * p + half_;
+    // block b starts at byte 34b; see gemv.cu for the word alignment rule
+    uint32_t qwd[8];
+    __half dh;
+    if ((b & 1) == 0) {
+      const int a = 17 * b / 2;
+      dh = __ushort_as_half(static_cast<unsigned short>(word_of(u, a) & 0xffffu));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qwd[i] = __funnelshift_r(word_of(u, a + i), word_of(u, a + i + 1), 16);
+    } else {
+      const int a = (17 * b - 1) / 2;
+      dh = __ushort_as_half(static_cast<unsigned short>(word_of(u, a) >> 16));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qwd[i] = word_of(u, a + 1 + i);
+    }
+    const __half2 d2 = __half2half2(dh);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q8x4_to_h(qwd[i], d2, out[16 * half_ + 2 * i], out[16 * half_ + 2 * i + 1]);
+  }
+}
+
+// Q4_K: piece p (64 elements = sub-blocks 2p (low nibbles) and 2p+1 (high
+// nibbles) of bytes qs[32p .. 32p+31]).  Each value is fp32 (d*sc)*q - dmin*m
+// (one rounding: (d*sc)*q and dmin*m are exact), then binary16 RNE.
+__device__ __forceinline__ void piece_q4_k(const RawUnit<DSQ_Q4_K> &u, int p, uint32_t (&out)[32]) {
+  const uint32_t w0 = word_of(u, 0);
+  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(w0 & 0xffffu)));
+  const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(w0 >> 16)));
+  const uint32_t s0 = word_of(u, 1), s1 = word_of(u, 2), s2 = word_of(u, 3);
+#pragma unroll
+  for (int half_ = 0; half_ < 2; ++half_) {
+    const int j = 2 * p + half_;
+    uint32_t scw, mw;
+    if (j < 4) {
+      scw = s0 & 0x3f3f3f3fu;
+      mw = s1 & 0x3f3f3f3fu;
+    } else {
+      scw = (s2 & 0x0f0f0f0fu) | ((s0 >> 2) & 0x30303030u);
+      mw = ((s2 >> 4) & 0x0f0f0f0fu) | ((s1 >> 2) & 0x30303030u);
+    }
+    const int sh = 8 * (j & 3);
+    const float a = __fmul_rn(d, static_cast<float>((scw >> sh) & 0xffu));
+    const float nb = -__fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t byte4 = word_of(u, 4 + 8 * p + i);
+      const uint32_t nib = half_ ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        // 0x4B000000 | q is the float 2^23 + q; subtracting 2^23 is exact
+        const float f = __uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7540 + e));
+        v[e] = __fmaf_rn(__fsub_rn(f, 8388608.0f), a, nb);
+      }
+      out[16 * half_ + 2 * i] = h2_bits(__floats2half2_rn(v[0], v[1]));
+      out[16 * half_ + 2 * i + 1] = h2_bits(__floats2half2_rn(v[2], v[3]));
+    }
+  }
+}
+
+template <int TYPE>
+__device__ __forceinline__ void dequant_piece(const RawUnit<TYPE> &u, int p, uint32_t (&out)[32]) {
+  if constexpr (TYPE == DSQ_Q8_0) piece_q8_0(u, p, out);
+  else piece_q4_k(u, p, out);
+}
+
+// Store one row's 64-element piece into a 128B-swizzled K-major stage:
+// row r at r*128, 16-byte chunk c at chunk position c ^ (r & 7).
+__device__ __forceinline__ void store_piece_sw128(uint8_t *stage, int r, const uint32_t (&v)[32]) {
+  uint8_t *row = stage + r * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 q = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = q;
+  }
+}
+
+// ------------------------------------------------------------------ GEMM ---
+struct Smem {
+  uint8_t *a;         // stages x 16 KB
+  uint8_t *b;         // stages x tn*128
+  uint64_t *afull;    // converters arrived (count 4)
+  uint64_t *bfull;    // TMA bytes landed (count 1 + tx)
+  uint64_t *empty;    // MMA finished reading the stage (commit)
+  uint64_t *acc;      // accumulator complete (commit)
+  uint64_t *drain;    // MMA drain after an abort
+  uint32_t *tmem;     // TMEM base address
+  volatile int *abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t *base, int stages, int tn) {
+  Smem s;
+  s.a = base;
+  s.b = base + static_cast<size_t>(stages) * kAStageBytes;
+  uint8_t *p = s.b + static_cast<size_t>(stages) * tn * 128;
+  s.afull = reinterpret_cast<uint64_t *>(p);
+  s.bfull = s.afull + stages;
+  s.empty = s.bfull + stages;
+  s.acc = s.empty + stages;
+  s.drain = s.acc + 1;
+  s.tmem = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.abort = reinterpret_cast<volatile int *>(s.tmem + 1);
+  return s;
+}
+
+__device__ __forceinline__ bool aborted(const Smem &s) { return *s.abort != 0; }
+__device__ __forceinline__ void set_abort(const Smem &s, const WaitCtl &w) {
+  *s.abort = 1;
+  record_timeout(w);
+}
+
+template <int TYPE>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Smem s = carve(base, a.stages, a.tn);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * a.tn;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kBM;
+  const int split = blockIdx.z;
+  const int u_begin = split * a.units_per_split;
+  const int units_total = static_cast<int>(a.K / 256);
+  const int u_end = min(u_begin + a.units_per_split, units_total);
+  const int iters = 4 * (u_end - u_begin);
+  const int S = a.stages;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&s.afull[i], 4);
+      mbar_init(&s.bfull[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    mbar_init(s.acc, 1);
+    mbar_init(s.drain, 1);
+    *s.abort = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmap_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(s.tmem, static_cast<uint32_t>(a.tmem_cols));
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_d = *s.tmem;
+  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (X tiles)
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < iters; ++it) {
+        const int st = it % S;
+        if (it >= S) {
+          if (aborted(s)) break;
+          if (!mbar_wait_for(&s.empty[st], static_cast<uint32_t>((it / S - 1) & 1), a.wait.limit_ns)) {
+            set_abort(s, a.wait);
+            break;
+          }
+        }
+        mbar_arrive_expect_tx(&s.bfull[st], stage_b_bytes);
+        const int32_t kx = (u_begin * 4 + it) * kBK;
+        tma_load_2d(s.b + static_cast<size_t>(st) * stage_b_bytes, &tmap_x, kx, static_cast<int32_t>(m0),
+                    &s.bfull[st]);
+        ++issued;
+      }
+      if (aborted(s)) {  // drain our copies still in flight
+        for (int it = (issued > S ? issued - S : 0); it < issued; ++it)
+          mbar_wait_for(&s.bfull[it % S], static_cast<uint32_t>((it / S) & 1), kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(kBM, static_cast<uint32_t>(a.tn), 0);
+      const uint32_t a_base = smem_u32(s.a), b_base = smem_u32(s.b);
+      bool ok = true;
+      for (int it = 0; it < iters && ok; ++it) {
+        const int st = it % S;
+        const uint32_t par = static_cast<uint32_t>((it / S) & 1);
+        if (aborted(s) || !mbar_wait_for(&s.bfull[st], par, a.wait.limit_ns) ||
+            !mbar_wait_for(&s.afull[st], par, a.wait.limit_ns)) {
+          if (!aborted(s)) set_abort(s, a.wait);
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = a_base + static_cast<uint32_t>(st) * kAStageBytes;
+        const uint32_t b_addr = b_base + static_cast<uint32_t>(st) * stage_b_bytes;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          umma_f16(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
+                   (it > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&s.empty[st]);
+      }
+      if (ok) {
+        umma_commit(s.acc);
+      } else {
+        umma_commit(s.drain);
+        mbar_wait_for(s.drain, 0, kDrainLimitNs);
+      }
+    }
+  } else {
+    // ------------------------------------- converters, then the epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = 32 * q + lane;            // weight row within the tile
+    const int64_t n = n0 + r;
+    const bool live = n < a.N;
+    const uint8_t *rowp = a.w + (live ? n : 0) * a.row_bytes;
+    RawUnit<TYPE> cur, nxt;
+    if (live && u_begin < u_end) load_unit<TYPE>(cur, rowp + static_cast<size_t>(u_begin) * (TYPE == DSQ_Q8_0 ? 272 : 144));
+    bool ok = true;
+    for (int u = u_begin; u < u_end && ok; ++u) {
+      if (live && u + 1 < u_end) load_unit<TYPE>(nxt, rowp + static_cast<size_t>(u + 1) * (TYPE == DSQ_Q8_0 ? 272 : 144));
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int it = 4 * (u - u_begin) + p;
+        const int st = it % S;
+        if (it >= S) {
+          const bool got = mbar_wait_for(&s.empty[st], static_cast<uint32_t>((it / S - 1) & 1), a.wait.limit_ns);
+          if (__any_sync(0xffffffffu, !got) || aborted(s)) {
+            if (lane == 0 && !aborted(s)) set_abort(s, a.wait);
+            ok = false;
+            break;
+          }
+        }
+        uint32_t v[32];
+        if (live) {
+          dequant_piece<TYPE>(cur, p, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        store_piece_sw128(s.a + static_cast<size_t>(st) * kAStageBytes, r, v);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.afull[st]);
+      }
+      cur = nxt;
+    }
+    // epilogue: D[r][token] -> y[m][n] * 2^-s_m
+    if (ok && !aborted(s)) {
+      const bool got = mbar_wait_for(s.acc, 0, a.wait.limit_ns);
+      if (__any_sync(0xffffffffu, !got)) {
+        if (lane == 0) set_abort(s, a.wait);
+      } else {
+        tc_fence_after_sync();
+        float *y = a.y + static_cast<int64_t>(split) * a.M * a.N;
+        for (int c = 0; c < a.tn / 32; ++c) {
+          uint32_t acc[32];
+          tmem_ld_32cols(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), acc);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int64_t m = m0 + 32 * c + i;
+            if (m < a.M && live) {
+              const int sft = __ldg(a.shift + m);
+              const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
+              y[m * a.N + n] = __fmul_rn(__uint_as_float(acc[i]), scale);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_d, static_cast<uint32_t>(a.tmem_cols));
+  }
+}
+
+// --------------------------------------------------- activation rounding --
+// One CTA per activation row: row max -> shift s (max |x| * 2^s in
+// [2^14, 2^15), 0 for a zero row, clamped to [-64, 64]) -> binary16 RNE of
+// x * 2^s (an exact scaling unless the product is an fp32 subnormal).
+// Rows m >= M (padding up to whole token tiles) are written as zeros.
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__ x, int64_t M, int64_t K,
+                                                       __half *__restrict__ x16, int32_t *__restrict__ shift) {
+  __shared__ float red[8];
+  const int64_t m = blockIdx.x;
+  if (m >= M) {
+    uint4 *out = reinterpret_cast<uint4 *>(x16 + m * K);
+    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) out[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x == 0) shift[m] = 0;
+    return;
+  }
+  const float4 *row = reinterpret_cast<const float4 *>(x + m * K);
+  const int64_t nv = K / 4;
+  float amax = 0.0f;
+  for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
+    const float4 v = __ldg(row + i);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  int s = 0;
+  if (amax > 0.0f && !isinf(amax)) {
+    int e;
+    frexpf(amax, &e);
+    s = min(64, max(-64, 15 - e));
+  }
+  const float scale = __int_as_float((127 + s) << 23);
+  if (threadIdx.x == 0) shift[m] = s;
+  uint2 *out = reinterpret_cast<uint2 *>(x16 + m * K);
+  for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
+    const float4 v = __ldg(row + i);
+    const __half2 lo = __floats2half2_rn(__fmul_rn(v.x, scale), __fmul_rn(v.y, scale));
+    const __half2 hi = __floats2half2_rn(__fmul_rn(v.z, scale), __fmul_rn(v.w, scale));
+    out[i] = make_uint2(h2_bits(lo), h2_bits(hi));
+  }
+}
+
+// Split-K partials -> output, summed in split order (deterministic).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ part, int64_t total, int splits,
+                                                            float *__restrict__ y) {
+  const int64_t n4 = total / 4;
+  const float4 *p4 = reinterpret_cast<const float4 *>(part);
+  float4 *y4 = reinterpret_cast<float4 *>(y);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 acc = __ldg(p4 + i);
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = __ldg(p4 + static_cast<int64_t>(s) * n4 + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    y4[i] = acc;
+  }
+  for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    float acc = part[i];
+    for (int s = 1; s < splits; ++s) acc += part[static_cast<int64_t>(s) * total + i];
+    y[i] = acc;
+  }
+}
+
+// Test hook: the whole dequantized weight matrix in binary16, produced by the
+// same device functions as the GEMM's converter warps.
+template <int TYPE>
+__global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict__ w, int64_t N, int64_t K,
+                                                       int64_t row_bytes, uint16_t *__restrict__ w16) {
+  const int64_t units = K / 256;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= N * units) return;
+  const int64_t n = idx / units, u = idx % units;
+  RawUnit<TYPE> ru;
+  load_unit<TYPE>(ru, w + n * row_bytes + u * (TYPE == DSQ_Q8_0 ? 272 : 144));
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    uint32_t v[32];
+    dequant_piece<TYPE>(ru, p, v);
+    uint4 *dst = reinterpret_cast<uint4 *>(w16 + n * K + u * 256 + p * 64);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
+}
+
+// ------------------------------------------------------------------- host --
+struct Plan {
+  int tn, stages, splits, units_per_split, tmem_cols;
+  int64_t tiles_m, tiles_n, m_pad;
+  size_t x16_bytes, shift_off, part_off, total;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
+  Plan p{};
+  const int64_t tiles_n = (N + kBM - 1) / kBM;
+  // tokens per tile: small M takes the smallest multiple of 32 that covers
+  // it; larger M picks 128 or 256 by a waves x per-tile-cost model (the +64
+  // stands for the per-tile weight dequantization, which does not shrink
+  // with the tile's token count)
+  if (M <= 128) {
+    p.tn = static_cast<int>((M + 31) / 32 * 32);
+  } else {
+    double best = 1e30;
+    for (int tn : {256, 128}) {
+      const int64_t ctas = (M + tn - 1) / tn * tiles_n;
+      const double waves = static_cast<double>((ctas + num_sms - 1) / num_sms);
+      const double cost = waves * (tn + 64);
+      if (cost < best - 1e-9) { best = cost; p.tn = tn; }
+    }
+  }
+  p.tiles_m = (M + p.tn - 1) / p.tn;
+  p.tiles_n = tiles_n;
+  const int units = static_cast<int>(K / 256);
+  const int64_t tiles = p.tiles_m * p.tiles_n;
+  // split K only when the tiles leave more than half the SMs idle
+  p.splits = 1;
+  while (tiles * p.splits * 2 <= num_sms && p.splits * 2 <= 16 && p.splits * 2 <= units) p.splits *= 2;
+  p.units_per_split = (units + p.splits - 1) / p.splits;
+  p.splits = (units + p.units_per_split - 1) / p.units_per_split;
+  const int stage_bytes = kAStageBytes + p.tn * 128;
+  p.stages = static_cast<int>((200 * 1024) / stage_bytes);
+  if (p.stages > 8) p.stages = 8;
+  p.tmem_cols = 32;
+  while (p.tmem_cols < p.tn) p.tmem_cols *= 2;   // TMEM allocations are powers of two
+  // the fp16 activation buffer is padded with zero rows to whole token tiles,
+  // so every TMA box lies inside the tensor
+  p.m_pad = p.tiles_m * p.tn;
+  p.x16_bytes = align_up(static_cast<size_t>(p.m_pad) * K * 2, 1024);
+  p.shift_off = p.x16_bytes;
+  p.part_off = align_up(p.shift_off + static_cast<size_t>(p.m_pad) * 4, 1024);
+  p.total = p.part_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * 4 : 0);
+  return p;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+int validate(const char *name, int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M) {
+  DSQ_REQUIRE(type == DSQ_Q8_0 || type == DSQ_Q4_K, DSQ_ERR_INVALID_ARG, "%s: unsupported type %d", name, type);
+  DSQ_REQUIRE(N >= 1 && M >= 1 && K >= 1, DSQ_ERR_INVALID_ARG, "%s: N, M, K must be >= 1", name);
+  DSQ_REQUIRE(K % 256 == 0, DSQ_ERR_SHAPE, "%s: K=%lld must be a multiple of 256", name, (long long)K);
+  DSQ_REQUIRE(K <= 65536 && N <= (int64_t(1) << 24) && M <= (int64_t(1) << 24), DSQ_ERR_SHAPE,
+              "%s: size out of range (K <= 65536, M, N <= 2^24)", name);
+  DSQ_REQUIRE(w && x, DSQ_ERR_INVALID_ARG, "%s: null pointer", name);
+  DSQ_REQUIRE(aligned(w, 16) && aligned(x, 16), DSQ_ERR_ALIGNMENT, "%s: w and x must be 16-byte aligned", name);
+  return DSQ_OK;
+}
+
+template <int TYPE>
+int launch_gemm(const PrefillArgs &args, const CUtensorMap &map, const Plan &p, cudaStream_t stream) {
+  const size_t smem = 1024 + static_cast<size_t>(p.stages) * (kAStageBytes + p.tn * 128) +
+                      (3 * p.stages + 2) * sizeof(uint64_t) + 16;
+  auto kern = prefill_kernel<TYPE>;
+  const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "prefill");
+  if (rc != DSQ_OK) return rc;
+  dim3 grid(static_cast<unsigned>(p.tiles_m), static_cast<unsigned>(p.tiles_n), static_cast<unsigned>(p.splits));
+  kern<<<grid, kThreads, smem, stream>>>(map, args);
+  return after_launch("dsq_gemm_prefill: gemm");
+}
+
+}  // namespace
+}  // namespace dsq
+
+extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M) {
+  using namespace dsq;
+  if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
+  int sms = 148;
+  if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
+  return make_plan(N, K, M, sms).total;
+}
+
+extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+  using namespace dsq;
+  int rc = validate("dsq_gemm_prefill", type, w, N, K, x, M);
+  if (rc != DSQ_OK) return rc;
+  DSQ_REQUIRE(y != nullptr, DSQ_ERR_INVALID_ARG, "dsq_gemm_prefill: null output");
+  DSQ_REQUIRE(aligned(y, 16), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: y must be 16-byte aligned");
+  WaitCtl ctl;
+  int sms = 0;
+  rc = wait_ctl(&ctl, &sms);
+  if (rc != DSQ_OK) return rc;
+  const Plan p = make_plan(N, K, M, sms);
+  DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
+              "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
+  DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
+  auto enc = encode_fn();
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  __half *x16 = reinterpret_cast<__half *>(ws);
+  int32_t *shift = reinterpret_cast<int32_t *>(ws + p.shift_off);
+  float *part = reinterpret_cast<float *>(ws + p.part_off);
+
+  CUtensorMap map;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(p.m_pad)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.tn)};
+  const cuuint32_t estride[2] = {1u, 1u};
+  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: tensor map encode failed (%d)", (int)cr);
+
+  cudaStream_t st = as_stream(stream);
+  x_to_f16_kernel<<<static_cast<unsigned>(p.m_pad), 256, 0, st>>>(x, M, K, x16, shift);
+  rc = after_launch("dsq_gemm_prefill: x_to_f16");
+  if (rc != DSQ_OK) return rc;
+
+  PrefillArgs args{};
+  args.w = static_cast<const uint8_t *>(w);
+  args.N = N;
+  args.K = K;
+  args.M = M;
+  args.row_bytes = static_cast<int64_t>(dsq_row_bytes(type, K));
+  args.shift = shift;
+  args.y = p.splits > 1 ? part : y;
+  args.units_per_split = p.units_per_split;
+  args.splits = p.splits;
+  args.tn = p.tn;
+  args.stages = p.stages;
+  args.tmem_cols = p.tmem_cols;
+  args.wait = ctl;
+  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, map, p, st) : launch_gemm<DSQ_Q4_K>(args, map, p, st);
+  if (rc != DSQ_OK) return rc;
+  if (p.splits > 1) {
+    const int64_t total = M * N;
+    const int64_t blocks = (total / 4 + 255) / 256 + 1;
+    const unsigned grid = static_cast<unsigned>(blocks < 8 * sms ? blocks : 8 * sms);
+    splitk_reduce_kernel<<<grid, 256, 0, st>>>(part, total, p.splits, y);
+    rc = after_launch("dsq_gemm_prefill: split-k reduce");
+  }
+  return rc;
+}
+
+extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M,
+                                         uint16_t *x16, int32_t *shift, uint16_t *w16, void *stream) {
+  using namespace dsq;
+  int rc = validate("dsq_test_prefill_operands", type, w, N, K, x, M);
+  if (rc != DSQ_OK) return rc;
+  DSQ_REQUIRE(x16 && shift && w16, DSQ_ERR_INVALID_ARG, "dsq_test_prefill_operands: null output");
+  DSQ_REQUIRE(aligned(x16, 16) && aligned(w16, 16) && aligned(shift, 4), DSQ_ERR_ALIGNMENT,
+              "dsq_test_prefill_operands: output alignment");
+  rc = device_ready(nullptr, nullptr);
+  if (rc != DSQ_OK) return rc;
+  cudaStream_t st = as_stream(stream);
+  x_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, reinterpret_cast<__half *>(x16), shift);
+  rc = after_launch("dsq_test_prefill_operands: x");
+  if (rc != DSQ_OK) return rc;
+  const int64_t work = N * (K / 256);
+  const unsigned grid = static_cast<unsigned>((work + 127) / 128);
+  const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  if (type == DSQ_Q8_0)
+    w_to_f16_kernel<DSQ_Q8_0><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16);
+  else
+    w_to_f16_kernel<DSQ_Q4_K><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16);
+  return after_launch("dsq_test_prefill_operands: w");
+}

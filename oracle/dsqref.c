@@ -433,33 +433,46 @@ int dsqref_row_shift(const float *row, int64_t K)
     return s;
 }
 
-static double round16(int op16, float v)
+static uint16_t round16_bits(int op16, float v)
 {
-    return op16 ? (double)dsqref_bf16_to_f32(dsqref_f32_to_bf16(v))
-                : (double)dsqref_f16_to_f32(dsqref_f32_to_f16(v));
+    return op16 ? dsqref_f32_to_bf16(v) : dsqref_f32_to_f16(v);
+}
+
+static double bits16_value(int op16, uint16_t h)
+{
+    return op16 ? (double)dsqref_bf16_to_f32(h) : (double)dsqref_f16_to_f32(h);
+}
+
+void dsqref_prefill_operands(int type, int op16, const uint8_t *w, int64_t N,
+                             int64_t K, const float *x, int64_t M,
+                             uint16_t *x16, int32_t *shift, uint16_t *w16)
+{
+    float *wf = (float *)malloc((size_t)K * sizeof(float));
+    for (int64_t n = 0; n < N; ++n) {
+        dsqref_dequantize(type, w + n * dsqref_row_bytes(type, K), 1, K, wf);
+        for (int64_t k = 0; k < K; ++k) w16[n * K + k] = round16_bits(op16, wf[k]);
+    }
+    for (int64_t m = 0; m < M; ++m) {
+        shift[m] = dsqref_row_shift(x + m * K, K);
+        for (int64_t k = 0; k < K; ++k)
+            x16[m * K + k] = round16_bits(op16, ldexpf(x[m * K + k], shift[m]));
+    }
+    free(wf);
 }
 
 void dsqref_prefill_rounded(int type, int op16, const uint8_t *w, int64_t N,
                             int64_t K, const float *x, int64_t M, double *y)
 {
-    float *wf = (float *)malloc((size_t)K * sizeof(float));
-    double *wr = (double *)malloc((size_t)N * (size_t)K * sizeof(double));
-    double *xr = (double *)malloc((size_t)M * (size_t)K * sizeof(double));
-    int *shift = (int *)malloc((size_t)(M > 0 ? M : 1) * sizeof(int));
-    for (int64_t n = 0; n < N; ++n) {
-        dsqref_dequantize(type, w + n * dsqref_row_bytes(type, K), 1, K, wf);
-        for (int64_t k = 0; k < K; ++k) wr[n * K + k] = round16(op16, wf[k]);
-    }
-    for (int64_t m = 0; m < M; ++m) {
-        shift[m] = dsqref_row_shift(x + m * K, K);
-        for (int64_t k = 0; k < K; ++k)
-            xr[m * K + k] = round16(op16, ldexpf(x[m * K + k], shift[m]));
-    }
+    uint16_t *w16 = (uint16_t *)malloc((size_t)N * (size_t)K * sizeof(uint16_t));
+    uint16_t *x16 = (uint16_t *)malloc((size_t)(M > 0 ? M : 1) * (size_t)K * sizeof(uint16_t));
+    int32_t *shift = (int32_t *)malloc((size_t)(M > 0 ? M : 1) * sizeof(int32_t));
+    dsqref_prefill_operands(type, op16, w, N, K, x, M, x16, shift, w16);
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double acc = 0.0;
-            for (int64_t k = 0; k < K; ++k) acc += xr[m * K + k] * wr[n * K + k];
+            for (int64_t k = 0; k < K; ++k)
+                acc += bits16_value(op16, x16[m * K + k]) * bits16_value(op16, w16[n * K + k]);
             y[m * N + n] = ldexp(acc, -shift[m]);
         }
-    free(wf); free(wr); free(xr); free(shift);
+    free(w16); free(x16); free(shift);
 }

@@ -111,6 +111,12 @@ int dsqref_row_shift(const float *row, int64_t K);
 void dsqref_prefill_rounded(int type, int op16, const uint8_t *w, int64_t N,
                             int64_t K, const float *x, int64_t M, double *y);
 
+/* The rounded operands of dsqref_prefill_rounded as bit patterns:
+ * x16[m][k] = r(x[m][k] * 2^shift[m]), w16[n][k] = r(fp32 dequant). */
+void dsqref_prefill_operands(int type, int op16, const uint8_t *w, int64_t N,
+                             int64_t K, const float *x, int64_t M,
+                             uint16_t *x16, int32_t *shift, uint16_t *w16);
+
 #ifdef __cplusplus
 }
 #endif

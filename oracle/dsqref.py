@@ -73,6 +73,7 @@ def _declare(L):
         "dsqref_prefill_f64": (None, [_INT, _P, _I64, _I64, _P, _I64, _P]),
         "dsqref_row_shift": (_INT, [_P, _I64]),
         "dsqref_prefill_rounded": (None, [_INT, _INT, _P, _I64, _I64, _P, _I64, _P]),
+        "dsqref_prefill_operands": (None, [_INT, _INT, _P, _I64, _I64, _P, _I64, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -214,3 +215,16 @@ def prefill_rounded(qtype: int, w: np.ndarray, K: int, x: np.ndarray, op16: str 
     lib().dsqref_prefill_rounded(qtype, 0 if op16 == "f16" else 1, _ptr(w), N, K,
                                  _ptr(x), M, _ptr(y))
     return y
+
+
+def prefill_operands(qtype: int, w: np.ndarray, K: int, x: np.ndarray, op16: str = "f16"):
+    """(x16 bits [M, K], shift [M], w16 bits [N, K]) as the rounded reference forms them."""
+    w = _c(w, np.uint8)
+    x = _c(x, np.float32)
+    M, N = x.shape[0], w.shape[0]
+    x16 = np.zeros((M, K), np.uint16)
+    sh = np.zeros(M, np.int32)
+    w16 = np.zeros((N, K), np.uint16)
+    lib().dsqref_prefill_operands(qtype, 0 if op16 == "f16" else 1, _ptr(w), N, K, _ptr(x), M,
+                                  _ptr(x16), _ptr(sh), _ptr(w16))
+    return x16, sh, w16
