@@ -78,7 +78,7 @@ class ClockSampler(threading.Thread):
         self.period = period
         self.samples = []
         self.error = None
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         self.handle = None
         try:
             import pynvml
@@ -104,7 +104,7 @@ class ClockSampler(threading.Thread):
     def run(self):
         if self.handle is None:
             return
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 self.sample()
             except Exception as e:
@@ -113,7 +113,7 @@ class ClockSampler(threading.Thread):
             time.sleep(self.period)
 
     def stop(self):
-        self._stop.set()
+        self._halt.set()
         if self.is_alive():
             self.join()
         if self.handle is not None and not self.samples:
@@ -186,9 +186,24 @@ def copies_for(nbytes: int, lo: int = 2) -> int:
     return max(lo, -(-3 * L2_BYTES // max(nbytes, 1)) + 1)
 
 
+PROFILE = False   # --profile: run each selected workload a few times, untimed
+
+
+def profile_calls(fn, n: int = 3):
+    """Profile mode: n eager calls, no timing (for ncu captures)."""
+    import torch
+    st = torch.cuda.current_stream().cuda_stream
+    for i in range(n):
+        fn(i, st)
+    torch.cuda.synchronize()
+    return float("nan")
+
+
 def time_calls(fn, n_calls: int, warmup: int = 5):
     """Device time per call (CUDA events around a batch of eager calls)."""
     import torch
+    if PROFILE:
+        return profile_calls(fn)
     st = torch.cuda.current_stream().cuda_stream
     for i in range(warmup):
         fn(i, st)
@@ -206,6 +221,8 @@ def time_graph(fn, calls_per_graph: int, replays: int = 5):
     """Device time per call with the calls captured in a CUDA graph, so host
     launch cost cannot hide in the figure (CUDA events around the replays)."""
     import torch
+    if PROFILE:
+        return profile_calls(fn)
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -331,7 +348,8 @@ def run_dsq(args, world, rank):
     # ---- the other rows of the path (each its own short timed loop)
     rows = {}
     if not args.skip_rows:
-        rows = measure_rows(dsq, L, stream, hbm_peak, bf16_peak)
+        rows = measure_rows(dsq, L, stream, hbm_peak, bf16_peak,
+                            only=set(args.rows.split(",")) if args.rows else None)
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -361,12 +379,16 @@ def run_dsq(args, world, rank):
     return result
 
 
-def measure_rows(dsq, L, stream, hbm_peak, bf16_peak):
-    """µs/call and GB/s (or TFLOP/s) for every other step of the path."""
+def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
+    """µs/call and GB/s (or TFLOP/s) for every other step of the path;
+    `only` restricts the run to the named rows."""
     import torch
 
     from block_quantized_dsq_b200 import synth
     rows = {}
+
+    def want(name):
+        return only is None or name in only
 
     def act(seed, M, K):
         x = torch.from_numpy(synth.activations(seed, M, K)).cuda()
@@ -377,13 +399,16 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak):
         return x, xq, xd, xs
 
     # activation prequantization, one decode row of K = 4096
-    x, xq, xd, xs = act(101, 1, 4096)
-    px, pq, pd, ps = x.data_ptr(), xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
-    t = time_graph(lambda i, st: L.dsq_quantize_act_q8(px, 1, 4096, pq, pd, ps, st), 500)
-    rows["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 3),
-                                      "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 2)}
+    if want("quantize_act_q8_1x4096"):
+        x, xq, xd, xs = act(101, 1, 4096)
+        px, pq, pd, ps = x.data_ptr(), xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
+        t = time_graph(lambda i, st: L.dsq_quantize_act_q8(px, 1, 4096, pq, pd, ps, st), 500)
+        rows["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 3),
+                                          "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 2)}
 
     def gemv_row(name, qtype, N, K, seed, xseed, G=1):
+        if not want(name):
+            return
         w = quantized_weights(dsq, qtype, seed, G * N, K)
         nbytes = w.numel()
         R = copies_for(nbytes)
@@ -416,9 +441,12 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak):
     # prefill dequant-GEMM sweep
     K = 4096
     for qtype, N, tag in ((dsq.DSQ_Q4_K, 4096, "q4_k_n4096"), (dsq.DSQ_Q8_0, 8192, "q8_0_n8192")):
+        Ms = [M for M in (128, 512, 2048) if want(f"prefill_{tag}_m{M}")]
+        if not Ms:
+            continue
         w = quantized_weights(dsq, qtype, seeds["prefill"]["w_q4_k" if qtype == dsq.DSQ_Q4_K else "w_q8_0"], N, K)
         ws = [w, w.clone()]
-        for M in (128, 512, 2048):
+        for M in Ms:
             x = torch.from_numpy(synth.activations(seeds["prefill"]["x_base"] + M, M, K)).cuda()
             y = torch.empty((M, N), dtype=torch.float32, device="cuda")
             nb = dsq.dsq_prefill_workspace_bytes(qtype, N, K, M)
@@ -429,8 +457,41 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak):
             tf = 2.0 * M * N * K / t / 1e12
             rows[f"prefill_{tag}_m{M}"] = {"us_per_call": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
                                            "bf16_peak_frac": round(tf / bf16_peak, 4)}
+            del x, y, wsp
     assert dsq.dsq_device_status() == 0
     return rows
+
+
+def run_profile(args):
+    """Untimed runs of selected workloads for ncu (committed so that every
+    profile summary names a command over committed files only)."""
+    global PROFILE
+    PROFILE = True
+    import torch
+
+    import block_quantized_dsq_b200 as dsq
+    from block_quantized_dsq_b200.build import build
+    build()
+    L = dsq.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    if not args.skip_headline:
+        from block_quantized_dsq_b200 import synth
+        seeds = synth.SEEDS["paired_q8_0_2x8192x4096"]
+        W0 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w0"], N_PAIR, K_PAIR)
+        W1 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w1"], N_PAIR, K_PAIR)
+        x = torch.from_numpy(synth.activations(seeds["x_base"], 1, K_PAIR)).cuda()
+        xq = torch.empty(K_PAIR, dtype=torch.int8, device="cuda")
+        xd = torch.empty(K_PAIR // 32, dtype=torch.float32, device="cuda")
+        xs = torch.empty(K_PAIR // 32, dtype=torch.int32, device="cuda")
+        y = torch.empty((2, N_PAIR), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            dsq.dsq_quantize_act_q8(x, 1, K_PAIR, xq, xd, xs, stream)
+            dsq.dsq_gemv_paired(8, W0, N_PAIR, W1, N_PAIR, K_PAIR, xq, xd, xs, y[0], y[1], stream)
+        torch.cuda.synchronize()
+    hbm_peak, bf16_peak, _, _ = measured_peaks()
+    if args.rows:
+        measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=set(args.rows.split(",")))
+    assert dsq.dsq_device_status() == 0
 
 
 def cpu_baseline(pair, X_host, budget_s: float):
@@ -503,6 +564,12 @@ def main():
     ap.add_argument("--skip-rows", action="store_true", help="only the headline workload")
     ap.add_argument("--skip-cpu", action="store_true", help="no CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--rows", default=None,
+                    help="comma-separated row names to run (e.g. prefill_q8_0_n8192_m2048)")
+    ap.add_argument("--profile", action="store_true",
+                    help="for ncu: run the selected rows (and, unless --skip-headline, one headline "
+                         "step) a few times untimed and print nothing")
+    ap.add_argument("--skip-headline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         args.steps = 5 if args.steps is None else args.steps
@@ -517,6 +584,9 @@ def main():
         args.warmup = 3
     world, rank, _ = dist_setup()
     try:
+        if args.profile:
+            run_profile(args)
+            return 0
         res = run_dsq(args, world, rank)
         if rank == 0:
             print(json.dumps(res))
