@@ -16,7 +16,7 @@ import threading
 __all__ = [
     "DSQ_Q8_0", "DSQ_Q4_K", "DsqError", "lib", "dsq_row_bytes", "dsq_quantize_act_q8",
     "dsq_gemv_q8_0", "dsq_gemv_q4_k", "dsq_gemv_paired", "dsq_gemv_grouped", "dsq_gemm_prefill",
-    "dsq_prefill_workspace_bytes", "dsq_quantize_weights", "dsq_device_status", "dsq_last_error",
+    "dsq_prefill_workspace_bytes", "dsq_gemm_prefill_noalloc", "dsq_quantize_weights", "dsq_device_status", "dsq_last_error",
     "dsq_version", "dsq_launch_count", "dsq_test_block_sums", "dsq_test_set_wait_limit_ns",
     "dsq_test_prefill_operands", "LIB_PATH",
 ]
@@ -45,6 +45,7 @@ _SIGS = {
     "dsq_gemv_grouped": (_INT, [_INT, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "dsq_gemm_prefill": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "dsq_prefill_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64]),
+    "dsq_gemm_prefill_noalloc": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P]),
     "dsq_quantize_weights": (_INT, [_INT, _P, _I64, _I64, _P, _P]),
     "dsq_device_status": (_INT, [_P]),
     "dsq_last_error": (ctypes.c_char_p, []),
@@ -143,6 +144,19 @@ def dsq_gemm_prefill(qtype, w, N, K, x, M, y, workspace, workspace_bytes, stream
 
 def dsq_prefill_workspace_bytes(qtype: int, N: int, K: int, M: int) -> int:
     return lib().dsq_prefill_workspace_bytes(qtype, N, K, M)
+
+
+DSQ_PREFILL_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def dsq_gemm_prefill_noalloc(qtype, w, N, K, x, M, y, stream=None):
+    """dsq_gemm_prefill for callers that cannot allocate device memory at
+    call time: scratch comes from a fixed 32 MiB array inside the library.
+    The first call on a device does a one-time set-up (make it before any
+    stream capture); calls that may overlap on the GPU race on the shared
+    scratch and must be serialized by the caller."""
+    _check("dsq_gemm_prefill_noalloc",
+           lib().dsq_gemm_prefill_noalloc(qtype, _ptr(w), N, K, _ptr(x), M, _ptr(y), _stream(stream)))
 
 
 def dsq_quantize_weights(qtype, x, N, K, w, stream=None):

@@ -32,6 +32,8 @@
 //    role, drains copies and MMAs in flight, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "../../include/dsq_test.h"
 #include "dsq_host.h"
 
@@ -646,4 +648,51 @@ extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int
   else
     w_to_f16_kernel<DSQ_Q4_K><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16);
   return after_launch("dsq_test_prefill_operands: w");
+}
+
+// ------------------------------------------------ allocation-free variant --
+// Scratch for dsq_gemm_prefill_noalloc: a fixed array in device global
+// memory, reserved once per device when the module loads (every device that
+// loads the library holds these 32 MiB until the process exits).  The
+// prefill kernels write every byte of it they later read in the same call,
+// so nothing has to be cleared between calls.
+static __device__ __align__(256) uint8_t g_prefill_scratch[DSQ_PREFILL_NOALLOC_SCRATCH_BYTES];
+
+namespace dsq {
+namespace {
+std::mutex g_scratch_mu;
+void *g_scratch_addr[64] = {};   // device address of g_prefill_scratch, per device
+}  // namespace
+}  // namespace dsq
+
+extern "C" int dsq_gemm_prefill_noalloc(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M,
+                                        float *y, void *stream) {
+  using namespace dsq;
+  const size_t need = dsq_prefill_workspace_bytes(type, N, K, M);
+  if (need == 0)  // invalid type or shape: let the regular entry point name it
+    return dsq_gemm_prefill(type, w, N, K, x, M, y, nullptr, 0, stream);
+  DSQ_REQUIRE(need <= DSQ_PREFILL_NOALLOC_SCRATCH_BYTES, DSQ_ERR_WORKSPACE,
+              "dsq_gemm_prefill_noalloc: this problem needs %zu bytes of scratch but the built-in scratch holds "
+              "%llu bytes (M x K x 2 bytes of fp16 activations plus split-K partials must fit); use "
+              "dsq_gemm_prefill with a caller-provided workspace",
+              need, (unsigned long long)DSQ_PREFILL_NOALLOC_SCRATCH_BYTES);
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  DSQ_REQUIRE(e == cudaSuccess && dev >= 0 && dev < 64, DSQ_ERR_CUDA, "dsq_gemm_prefill_noalloc: no current device");
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+      // One-time set-up on this device (the device is current): the host
+      // name of the array is only a stand-in, so fetch its device address.
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+      DSQ_REQUIRE(e == cudaSuccess && p != nullptr, DSQ_ERR_CUDA,
+                  "dsq_gemm_prefill_noalloc: cudaGetSymbolAddress of the scratch failed: %s", cudaGetErrorString(e));
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  return dsq_gemm_prefill(type, w, N, K, x, M, y, scratch, static_cast<size_t>(DSQ_PREFILL_NOALLOC_SCRATCH_BYTES),
+                          stream);
 }

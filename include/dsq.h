@@ -154,6 +154,34 @@ int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K,
 size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M);
 
 /*
+ * Allocation-free prefill: dsq_gemm_prefill without a workspace argument.
+ * The paper has no counterpart; this entry point exists for callers that
+ * cannot allocate device memory when they call -- for example code that
+ * runs under a fixed device-memory budget reserved up front, a plugin that
+ * is handed only its input and output buffers by a host framework with no
+ * workspace hook, or a caller inside a region where cudaMalloc is not
+ * allowed (such as a global-mode stream capture).
+ *
+ * Scratch lives in a fixed 32 MiB array in device memory that every device
+ * loading libdsq reserves until the process exits.  Problems whose
+ * dsq_prefill_workspace_bytes(type, N, K, M) exceeds
+ * DSQ_PREFILL_NOALLOC_SCRATCH_BYTES are rejected with DSQ_ERR_WORKSPACE and
+ * nothing is launched; otherwise arguments, layout, numerics and errors are
+ * those of dsq_gemm_prefill.  No call allocates or frees device memory.
+ *
+ * The first call on a device performs a one-time set-up (it looks up the
+ * device address of the scratch array); make that first call before any
+ * stream capture.  All calls on a device share the one scratch array, so
+ * calls that may overlap on the GPU (different streams without ordering,
+ * or concurrent host threads) race and must be serialized by the caller.
+ * Nothing in the array needs to be cleared between calls: each call writes
+ * every scratch byte it later reads.
+ */
+#define DSQ_PREFILL_NOALLOC_SCRATCH_BYTES (32ull * 1024ull * 1024ull)
+int dsq_gemm_prefill_noalloc(int type, const void *w, int64_t N, int64_t K,
+                             const float *x, int64_t M, float *y, void *stream);
+
+/*
  * Offline weight quantizer (device): fp32 rows x [N][K] -> packed rows in w
  * (N * dsq_row_bytes bytes).  Q8_0: d = fp16(amax/127), q from the fp32
  * scale, round half away from zero.  Q4_K (the pages give no quantizer; a
