@@ -34,6 +34,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------ programmatic launch ------
+// Kernels launched with programmatic stream serialization may start while
+// the previous kernel on the stream is still running.  pdl_wait() blocks
+// until that kernel has completed and its memory is visible: every read of
+// data a predecessor may have produced (and every write a predecessor may
+// still read) comes after it.  pdl_trigger() lets the next kernel launch
+// early.  Both are no-ops when the launch had no programmatic dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Hint: bring [src, src+bytes) into L2 (16-byte aligned, multiple of 16).
+// Safe before pdl_wait(): L2 is the point of coherence, so a prefetched line
+// can never be older than a predecessor's completed writes.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
@@ -122,6 +139,13 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Hint: bring one 2-D tile of a tensor map into L2 (same coordinate rules as
+// tma_load_2d).
+__device__ __forceinline__ void prefetch_l2_tile_2d(const CUtensorMap *map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {

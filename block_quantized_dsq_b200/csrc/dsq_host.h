@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "../../include/dsq.h"
@@ -29,6 +30,25 @@ int after_launch(const char *what, int n_kernels = 1);
 // the first call on a device configures it; later calls (for example inside
 // a CUDA graph capture) only launch.
 int set_smem_once(const void *kernel, int bytes, const char *what);
+
+// Launches `kern` on `stream` with programmatic stream serialization, so it
+// may start before the previous kernel on the stream has finished (the
+// kernel itself orders its dependent accesses with pdl_wait()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 inline bool aligned(const void *p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;

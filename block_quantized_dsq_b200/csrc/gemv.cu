@@ -31,6 +31,20 @@
 #include "../../include/dsq_test.h"
 #include "dsq_host.h"
 
+// Launch shape (compile-time constants; the defaults are the tuned values).
+#ifndef DSQ_GEMV_MAX_WARPS
+#define DSQ_GEMV_MAX_WARPS 8
+#endif
+#ifndef DSQ_GEMV_SMEM_KB
+#define DSQ_GEMV_SMEM_KB 220
+#endif
+#ifndef DSQ_GEMV_MAX_STAGES
+#define DSQ_GEMV_MAX_STAGES 2
+#endif
+#ifndef DSQ_GEMV_CTAS_PER_SM
+#define DSQ_GEMV_CTAS_PER_SM 1
+#endif
+
 namespace dsq {
 namespace {
 
@@ -196,7 +210,7 @@ __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_
 }
 
 template <int TYPE, int G, bool ISUM>
-__global__ void __launch_bounds__(256, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
+__global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
   constexpr int RPC = 32 / G;  // rows per slot
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -207,6 +221,23 @@ __global__ void __launch_bounds__(256, 1) gemv_kernel(const __grid_constant__ Ge
   const int64_t mine = nchunks > warp ? (nchunks - warp + W - 1) / W : 0;
   uint8_t *ring = smem + static_cast<size_t>(warp) * S * a.slot_bytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + static_cast<size_t>(W) * S * a.slot_bytes) + warp * S;
+
+  // Weights are read-only parameters: start pulling this warp's first slots
+  // into L2 while the previous kernel (usually the activation quantizer)
+  // finishes, then let the next kernel launch, then wait for our inputs.
+  if (lane == 0) {
+    for (int64_t k = 0; k < mine && k < S; ++k) {
+      const int64_t c = warp + k * W;
+      const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
+      if (rb <= a.rows0) {
+        prefetch_l2(a.seg[0].w + ra * a.row_bytes, static_cast<uint32_t>((rb - ra) * a.row_bytes));
+      } else if (ra >= a.rows0) {
+        prefetch_l2(a.seg[1].w + (ra - a.rows0) * a.row_bytes, static_cast<uint32_t>((rb - ra) * a.row_bytes));
+      }
+    }
+  }
+  pdl_trigger();
+  pdl_wait();
   if (mine == 0) return;
 
   const uint64_t policy = l2_policy_evict_first();
@@ -287,6 +318,8 @@ __global__ void __launch_bounds__(256, 1) gemv_kernel(const __grid_constant__ Ge
 // warp per row, lanes over 34-byte blocks read with 16-bit loads.
 template <bool ISUM>
 __global__ void __launch_bounds__(256) gemv_q8_0_rowwise_kernel(const __grid_constant__ GemvArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t nb = a.K / 32;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < a.total_rows;
@@ -316,8 +349,8 @@ __global__ void __launch_bounds__(256) gemv_q8_0_rowwise_kernel(const __grid_con
   }
 }
 
-constexpr int kMaxWarps = 8;
-constexpr size_t kSmemBudget = 220 * 1024;
+constexpr int kMaxWarps = DSQ_GEMV_MAX_WARPS;
+constexpr size_t kSmemBudget = DSQ_GEMV_SMEM_KB * 1024;
 
 template <int TYPE, int G, bool ISUM>
 int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
@@ -328,8 +361,10 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
   if (rc != DSQ_OK) return rc;
   const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
-  const unsigned grid = static_cast<unsigned>(chunks < num_sms ? chunks : num_sms);
-  kern<<<grid, a.warps * 32, smem, stream>>>(a);
+  const int64_t slots = static_cast<int64_t>(num_sms) * DSQ_GEMV_CTAS_PER_SM;
+  const unsigned grid = static_cast<unsigned>(chunks < slots ? chunks : slots);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(a.warps * 32), smem, stream, a);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "gemv: %s", cudaGetErrorString(e));
   return after_launch("gemv");
 }
 
@@ -388,8 +423,9 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   if (rb % 16 != 0) {  // Q8_0 with K % 256 != 0
     const int64_t blocks = (total + 7) / 8;
     const unsigned grid = static_cast<unsigned>(blocks < 4 * num_sms ? blocks : 4 * num_sms);
-    if (isum) gemv_q8_0_rowwise_kernel<true><<<grid, 256, 0, stream>>>(a);
-    else gemv_q8_0_rowwise_kernel<false><<<grid, 256, 0, stream>>>(a);
+    const cudaError_t e = isum ? launch_pdl(gemv_q8_0_rowwise_kernel<true>, dim3(grid), dim3(256), 0, stream, a)
+                               : launch_pdl(gemv_q8_0_rowwise_kernel<false>, dim3(grid), dim3(256), 0, stream, a);
+    if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: %s", name, cudaGetErrorString(e));
     return after_launch(name);
   }
   a.nunits = static_cast<int>(K / 256);
@@ -401,7 +437,7 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   DSQ_REQUIRE(static_cast<size_t>(a.warps) * 2 * a.slot_bytes <= kSmemBudget, DSQ_ERR_SHAPE,
               "%s: K=%lld rows do not fit the shared-memory pipeline", name, (long long)K);
   a.stages = static_cast<int>(kSmemBudget / (static_cast<size_t>(a.warps) * a.slot_bytes));
-  if (a.stages > 6) a.stages = 6;
+  if (a.stages > DSQ_GEMV_MAX_STAGES) a.stages = DSQ_GEMV_MAX_STAGES;
   if (type == DSQ_Q8_0)
     return isum ? dispatch_g<DSQ_Q8_0, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q8_0, false>(a, G, num_sms, stream);
   return isum ? dispatch_g<DSQ_Q4_K, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q4_K, false>(a, G, num_sms, stream);

@@ -42,20 +42,26 @@ namespace {
 
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // K elements per pipeline stage
-constexpr int kThreads = 192;     // 6 warps
 constexpr int kAStageBytes = kBM * kBK * 2;   // 16 KB
+// warp roles
+constexpr int kWarpX = 0;         // TMA producer: fp16 activation tiles
+constexpr int kWarpW = 1;         // TMA producer: raw weight units
+constexpr int kWarpMma = 2;       // TMEM owner, tcgen05.mma issuer
+constexpr int kWarpConv0 = 3;     // warps 3..6: dequantize raw units into A stages
+constexpr int kWarpEpi0 = 7;      // warps 7..10: TMEM -> global epilogue
+constexpr int kThreads = 11 * 32;
 
 struct PrefillArgs {
-  const uint8_t *w;
   int64_t N, K, M;
-  int64_t row_bytes;
   const int32_t *shift;   // [M] activation row shifts
   float *y;               // [M][N], or [splits][M][N] partials
   int units_per_split;    // 256-element units of K per split
   int splits;
   int tn;                 // tokens per tile (MMA N): 32..256, multiple of 32
-  int stages;
-  int tmem_cols;
+  int stages;             // A/B pipeline stages
+  int raw_stages;         // raw weight unit slots
+  int tmem_cols;          // two accumulators of tn columns
+  int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
 };
 
@@ -65,6 +71,7 @@ struct PrefillArgs {
 template <int TYPE> struct RawUnit;
 template <> struct RawUnit<DSQ_Q8_0> { static constexpr int kVecs = 17; uint4 v[17]; };
 template <> struct RawUnit<DSQ_Q4_K> { static constexpr int kVecs = 9; uint4 v[9]; };
+template <int TYPE> __host__ __device__ constexpr int unit_bytes() { return TYPE == DSQ_Q8_0 ? 272 : 144; }
 
 template <int TYPE>
 __device__ __forceinline__ void load_unit(RawUnit<TYPE> &u, const uint8_t *p) {
@@ -179,27 +186,35 @@ __device__ __forceinline__ void store_piece_sw128(uint8_t *stage, int r, const u
 
 // ------------------------------------------------------------------ GEMM ---
 struct Smem {
-  uint8_t *a;         // stages x 16 KB
-  uint8_t *b;         // stages x tn*128
-  uint64_t *afull;    // converters arrived (count 4)
-  uint64_t *bfull;    // TMA bytes landed (count 1 + tx)
-  uint64_t *empty;    // MMA finished reading the stage (commit)
-  uint64_t *acc;      // accumulator complete (commit)
-  uint64_t *drain;    // MMA drain after an abort
-  uint32_t *tmem;     // TMEM base address
+  uint8_t *a;          // stages x 16 KB: dequantized weight tiles (MMA A)
+  uint8_t *b;          // stages x tn*128: activation tiles (MMA B)
+  uint8_t *raw;        // raw_stages x 128 rows x unit bytes: raw weight units
+  uint64_t *afull;     // converters stored a stage (count 4)
+  uint64_t *bfull;     // activation tile landed (1 + tx)
+  uint64_t *sempty;    // MMA finished reading a stage (commit)
+  uint64_t *rfull;     // raw unit landed (1 + tx)
+  uint64_t *rempty;    // converters copied a raw unit out (count 4)
+  uint64_t *accfull;   // accumulator complete (commit), x2
+  uint64_t *accempty;  // epilogue drained an accumulator (count 4), x2
+  uint64_t *drain;     // MMA drain after an abort
+  uint32_t *tmem;      // TMEM base address
   volatile int *abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int stages, int tn) {
+__device__ __forceinline__ Smem carve(uint8_t *base, int stages, int tn, int raw_stages, int raw_bytes) {
   Smem s;
   s.a = base;
-  s.b = base + static_cast<size_t>(stages) * kAStageBytes;
-  uint8_t *p = s.b + static_cast<size_t>(stages) * tn * 128;
-  s.afull = reinterpret_cast<uint64_t *>(p);
+  s.b = s.a + static_cast<size_t>(stages) * kAStageBytes;
+  s.raw = s.b + static_cast<size_t>(stages) * tn * 128;
+  uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(raw_stages) * raw_bytes);
+  s.afull = p;
   s.bfull = s.afull + stages;
-  s.empty = s.bfull + stages;
-  s.acc = s.empty + stages;
-  s.drain = s.acc + 1;
+  s.sempty = s.bfull + stages;
+  s.rfull = s.sempty + stages;
+  s.rempty = s.rfull + raw_stages;
+  s.accfull = s.rempty + raw_stages;
+  s.accempty = s.accfull + 2;
+  s.drain = s.accempty + 2;
   s.tmem = reinterpret_cast<uint32_t *>(s.drain + 1);
   s.abort = reinterpret_cast<volatile int *>(s.tmem + 1);
   return s;
@@ -211,167 +226,240 @@ __device__ __forceinline__ void set_abort(const Smem &s, const WaitCtl &w) {
   record_timeout(w);
 }
 
+// One thread's bounded wait; on expiry (or an abort raised elsewhere) it
+// raises the CTA abort flag and returns false.
+__device__ __forceinline__ bool wait_or_abort(const Smem &s, uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+  if (aborted(s)) return false;
+  if (mbar_wait_for(bar, parity, w.limit_ns)) return true;
+  set_abort(s, w);
+  return false;
+}
+
+// Tile t -> (first token, first weight row, K split); consecutive tiles
+// share a weight tile, so CTAs running side by side reuse it from L2.
+struct Tile {
+  int64_t m0, n0;
+  int u0, u1;
+  int split;
+};
+__device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
+  Tile tl;
+  const int64_t m = t % a.tiles_m;
+  const int64_t rest = t / a.tiles_m;
+  tl.split = static_cast<int>(rest % a.splits);
+  tl.m0 = m * a.tn;
+  tl.n0 = (rest / a.splits) * kBM;
+  tl.u0 = tl.split * a.units_per_split;
+  tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
+  return tl;
+}
+
+// Persistent CTA: tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Every role
+// walks the same tile sequence; the A/B ring, the raw ring and the two TMEM
+// accumulators carry their phases across tiles.
 template <int TYPE>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ PrefillArgs a) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ PrefillArgs a) {
+  constexpr int UB = unit_bytes<TYPE>();
+  constexpr int RAW_BYTES = kBM * UB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Smem s = carve(base, a.stages, a.tn);
+  const Smem s = carve(base, a.stages, a.tn, a.raw_stages, RAW_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * a.tn;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kBM;
-  const int split = blockIdx.z;
-  const int u_begin = split * a.units_per_split;
-  const int units_total = static_cast<int>(a.K / 256);
-  const int u_end = min(u_begin + a.units_per_split, units_total);
-  const int iters = 4 * (u_end - u_begin);
-  const int S = a.stages;
+  const int S = a.stages, R = a.raw_stages;
+  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&s.afull[i], 4);
       mbar_init(&s.bfull[i], 1);
-      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.sempty[i], 1);
     }
-    mbar_init(s.acc, 1);
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&s.rfull[i], 1);
+      mbar_init(&s.rempty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.accfull[i], 1);
+      mbar_init(&s.accempty[i], 4);
+    }
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmap_x);
+    prefetch_tensormap(&tmap_w);
   }
-  if (warp == 1) {
+  if (warp == kWarpW && lane == 0 && blockIdx.x < a.total_tiles) {
+    // weights are read-only: start their first units toward L2 while the
+    // activation-rounding kernel before us finishes
+    const Tile tl = tile_of(a, blockIdx.x);
+    for (int u = tl.u0; u < tl.u1 && u < tl.u0 + R; ++u)
+      prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0));
+  }
+  if (warp == kWarpMma) {
     tmem_alloc(s.tmem, static_cast<uint32_t>(a.tmem_cols));
     tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_d = *s.tmem;
-  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;
+  pdl_trigger();
+  pdl_wait();
+  const uint32_t tmem_base = *s.tmem;
 
-  if (warp == 0) {
-    // ---------------------------------------------- TMA producer (X tiles)
+  if (warp == kWarpX) {
+    // ---------------------------------------------- activation tiles (TMA)
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < iters; ++it) {
-        const int st = it % S;
-        if (it >= S) {
-          if (aborted(s)) break;
-          if (!mbar_wait_for(&s.empty[st], static_cast<uint32_t>((it / S - 1) & 1), a.wait.limit_ns)) {
-            set_abort(s, a.wait);
-            break;
-          }
+      int64_t gs = 0;
+      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
+        const Tile tl = tile_of(a, t);
+        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it, ++gs) {
+          const int st = static_cast<int>(gs % S);
+          if (gs >= S && !wait_or_abort(s, &s.sempty[st], static_cast<uint32_t>((gs / S - 1) & 1), a.wait)) break;
+          mbar_arrive_expect_tx(&s.bfull[st], stage_b_bytes);
+          tma_load_2d(s.b + static_cast<size_t>(st) * stage_b_bytes, &tmap_x, (tl.u0 * 4 + it) * kBK,
+                      static_cast<int32_t>(tl.m0), &s.bfull[st]);
         }
-        mbar_arrive_expect_tx(&s.bfull[st], stage_b_bytes);
-        const int32_t kx = (u_begin * 4 + it) * kBK;
-        tma_load_2d(s.b + static_cast<size_t>(st) * stage_b_bytes, &tmap_x, kx, static_cast<int32_t>(m0),
-                    &s.bfull[st]);
-        ++issued;
       }
-      if (aborted(s)) {  // drain our copies still in flight
-        for (int it = (issued > S ? issued - S : 0); it < issued; ++it)
-          mbar_wait_for(&s.bfull[it % S], static_cast<uint32_t>((it / S) & 1), kDrainLimitNs);
-      }
+      if (aborted(s))
+        for (int64_t g = (gs > S ? gs - S : 0); g < gs; ++g)
+          mbar_wait_for(&s.bfull[g % S], static_cast<uint32_t>((g / S) & 1), kDrainLimitNs);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpW) {
+    // ------------------------------------------- raw weight units (TMA)
+    if (lane == 0) {
+      int64_t gu = 0;
+      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
+        const Tile tl = tile_of(a, t);
+        for (int u = tl.u0; u < tl.u1; ++u, ++gu) {
+          const int rs = static_cast<int>(gu % R);
+          if (gu >= R && !wait_or_abort(s, &s.rempty[rs], static_cast<uint32_t>((gu / R - 1) & 1), a.wait)) break;
+          mbar_arrive_expect_tx(&s.rfull[rs], static_cast<uint32_t>(RAW_BYTES));
+          tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &tmap_w, u * (UB / 4),
+                      static_cast<int32_t>(tl.n0), &s.rfull[rs]);
+        }
+      }
+      if (aborted(s))
+        for (int64_t g = (gu > R ? gu - R : 0); g < gu; ++g)
+          mbar_wait_for(&s.rfull[g % R], static_cast<uint32_t>((g / R) & 1), kDrainLimitNs);
+    }
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(kBM, static_cast<uint32_t>(a.tn), 0);
       const uint32_t a_base = smem_u32(s.a), b_base = smem_u32(s.b);
+      int64_t gs = 0, i = 0;
       bool ok = true;
-      for (int it = 0; it < iters && ok; ++it) {
-        const int st = it % S;
-        const uint32_t par = static_cast<uint32_t>((it / S) & 1);
-        if (aborted(s) || !mbar_wait_for(&s.bfull[st], par, a.wait.limit_ns) ||
-            !mbar_wait_for(&s.afull[st], par, a.wait.limit_ns)) {
-          if (!aborted(s)) set_abort(s, a.wait);
+      for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x, ++i) {
+        const Tile tl = tile_of(a, t);
+        const int acc = static_cast<int>(i & 1);
+        if (i >= 2 && !wait_or_abort(s, &s.accempty[acc], static_cast<uint32_t>((i / 2 - 1) & 1), a.wait)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a_addr = a_base + static_cast<uint32_t>(st) * kAStageBytes;
-        const uint32_t b_addr = b_base + static_cast<uint32_t>(st) * stage_b_bytes;
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * a.tn);
+        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it, ++gs) {
+          const int st = static_cast<int>(gs % S);
+          const uint32_t par = static_cast<uint32_t>((gs / S) & 1);
+          if (!wait_or_abort(s, &s.bfull[st], par, a.wait) || !wait_or_abort(s, &s.afull[st], par, a.wait)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = a_base + static_cast<uint32_t>(st) * kAStageBytes;
+          const uint32_t b_addr = b_base + static_cast<uint32_t>(st) * stage_b_bytes;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          umma_f16(tmem_d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
-                   (it > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&s.empty[st]);
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_f16(d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
+                     (it > 0 || k > 0) ? 1u : 0u);
+          umma_commit(&s.sempty[st]);
+        }
+        if (ok) umma_commit(&s.accfull[acc]);
       }
-      if (ok) {
-        umma_commit(s.acc);
-      } else {
+      if (!ok) {
         umma_commit(s.drain);
         mbar_wait_for(s.drain, 0, kDrainLimitNs);
       }
     }
-  } else {
-    // ------------------------------------- converters, then the epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = 32 * q + lane;            // weight row within the tile
-    const int64_t n = n0 + r;
-    const bool live = n < a.N;
-    const uint8_t *rowp = a.w + (live ? n : 0) * a.row_bytes;
-    RawUnit<TYPE> cur, nxt;
-    if (live && u_begin < u_end) load_unit<TYPE>(cur, rowp + static_cast<size_t>(u_begin) * (TYPE == DSQ_Q8_0 ? 272 : 144));
+  } else if (warp < kWarpEpi0) {
+    // ------------------------------------------ converters (dequantize)
+    const int r = 32 * (warp - kWarpConv0) + lane;   // weight row within the tile
+    int64_t gs = 0, gu = 0;
     bool ok = true;
-    for (int u = u_begin; u < u_end && ok; ++u) {
-      if (live && u + 1 < u_end) load_unit<TYPE>(nxt, rowp + static_cast<size_t>(u + 1) * (TYPE == DSQ_Q8_0 ? 272 : 144));
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int it = 4 * (u - u_begin) + p;
-        const int st = it % S;
-        if (it >= S) {
-          const bool got = mbar_wait_for(&s.empty[st], static_cast<uint32_t>((it / S - 1) & 1), a.wait.limit_ns);
-          if (__any_sync(0xffffffffu, !got) || aborted(s)) {
-            if (lane == 0 && !aborted(s)) set_abort(s, a.wait);
-            ok = false;
-            break;
-          }
+    for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x) {
+      const Tile tl = tile_of(a, t);
+      for (int u = tl.u0; u < tl.u1 && ok; ++u, ++gu) {
+        const int rs = static_cast<int>(gu % R);
+        const bool got = wait_or_abort(s, &s.rfull[rs], static_cast<uint32_t>((gu / R) & 1), a.wait);
+        if (__any_sync(0xffffffffu, !got)) {
+          ok = false;
+          break;
         }
-        uint32_t v[32];
-        if (live) {
-          dequant_piece<TYPE>(cur, p, v);
-        } else {
+        RawUnit<TYPE> ru;
+        const uint4 *src = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES + r * UB);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
-        }
-        store_piece_sw128(s.a + static_cast<size_t>(st) * kAStageBytes, r, v);
-        fence_proxy_async_smem();
+        for (int v = 0; v < RawUnit<TYPE>::kVecs; ++v) ru.v[v] = src[v];
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.afull[st]);
-      }
-      cur = nxt;
-    }
-    // epilogue: D[r][token] -> y[m][n] * 2^-s_m
-    if (ok && !aborted(s)) {
-      const bool got = mbar_wait_for(s.acc, 0, a.wait.limit_ns);
-      if (__any_sync(0xffffffffu, !got)) {
-        if (lane == 0) set_abort(s, a.wait);
-      } else {
-        tc_fence_after_sync();
-        float *y = a.y + static_cast<int64_t>(split) * a.M * a.N;
-        for (int c = 0; c < a.tn / 32; ++c) {
-          uint32_t acc[32];
-          tmem_ld_32cols(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), acc);
-          tmem_ld_wait();
+        if (lane == 0) mbar_arrive(&s.rempty[rs]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int64_t m = m0 + 32 * c + i;
-            if (m < a.M && live) {
-              const int sft = __ldg(a.shift + m);
-              const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
-              y[m * a.N + n] = __fmul_rn(__uint_as_float(acc[i]), scale);
+        for (int p = 0; p < 4; ++p, ++gs) {
+          const int st = static_cast<int>(gs % S);
+          if (gs >= S) {
+            const bool free_ = wait_or_abort(s, &s.sempty[st], static_cast<uint32_t>((gs / S - 1) & 1), a.wait);
+            if (__any_sync(0xffffffffu, !free_)) {
+              ok = false;
+              break;
             }
           }
+          uint32_t v[32];
+          dequant_piece<TYPE>(ru, p, v);
+          store_piece_sw128(s.a + static_cast<size_t>(st) * kAStageBytes, r, v);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.afull[st]);
         }
       }
+    }
+  } else {
+    // ------------------------------- epilogue: TMEM -> y * 2^-s_m
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int r = 32 * q + lane;            // weight row within the tile
+    int64_t i = 0;
+    for (int64_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x, ++i) {
+      const Tile tl = tile_of(a, t);
+      const int acc = static_cast<int>(i & 1);
+      const bool got = wait_or_abort(s, &s.accfull[acc], static_cast<uint32_t>((i / 2) & 1), a.wait);
+      if (__any_sync(0xffffffffu, !got)) break;
+      tc_fence_after_sync();
+      const int64_t n = tl.n0 + r;
+      float *y = a.y + static_cast<int64_t>(tl.split) * a.M * a.N;
+      for (int c = 0; c < a.tn / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * a.tn + 32 * c),
+                       v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int64_t m = tl.m0 + 32 * c + j;
+          if (m < a.M && n < a.N) {
+            const int sft = __ldg(a.shift + m);
+            const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
+            y[m * a.N + n] = __fmul_rn(__uint_as_float(v[j]), scale);
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.accempty[acc]);
     }
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_d, static_cast<uint32_t>(a.tmem_cols));
+    tmem_dealloc(tmem_base, static_cast<uint32_t>(a.tmem_cols));
   }
 }
 
@@ -383,6 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__ x, int64_t M, int64_t K,
                                                        __half *__restrict__ x16, int32_t *__restrict__ shift) {
   __shared__ float red[8];
+  pdl_trigger();
+  pdl_wait();
   const int64_t m = blockIdx.x;
   if (m >= M) {
     uint4 *out = reinterpret_cast<uint4 *>(x16 + m * K);
@@ -424,6 +514,8 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__
 // Split-K partials -> output, summed in split order (deterministic).
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ part, int64_t total, int splits,
                                                             float *__restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n4 = total / 4;
   const float4 *p4 = reinterpret_cast<const float4 *>(part);
   float4 *y4 = reinterpret_cast<float4 *>(y);
@@ -466,14 +558,17 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, stages, splits, units_per_split, tmem_cols;
-  int64_t tiles_m, tiles_n, m_pad;
-  size_t x16_bytes, shift_off, part_off, total;
+  int tn, stages, raw_stages, splits, units_per_split, tmem_cols;
+  int64_t tiles_m, tiles_n, total_tiles, m_pad;
+  unsigned grid;
+  size_t smem, x16_bytes, shift_off, part_off, total;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
+constexpr size_t kSmemLimit = 227 * 1024;
+
+Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int num_sms) {
   Plan p{};
   const int64_t tiles_n = (N + kBM - 1) / kBM;
   // tokens per tile: small M takes the smallest multiple of 32 that covers
@@ -485,8 +580,8 @@ Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
   } else {
     double best = 1e30;
     for (int tn : {256, 128}) {
-      const int64_t ctas = (M + tn - 1) / tn * tiles_n;
-      const double waves = static_cast<double>((ctas + num_sms - 1) / num_sms);
+      const int64_t tiles = (M + tn - 1) / tn * tiles_n;
+      const double waves = static_cast<double>((tiles + num_sms - 1) / num_sms);
       const double cost = waves * (tn + 64);
       if (cost < best - 1e-9) { best = cost; p.tn = tn; }
     }
@@ -500,11 +595,19 @@ Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
   while (tiles * p.splits * 2 <= num_sms && p.splits * 2 <= 16 && p.splits * 2 <= units) p.splits *= 2;
   p.units_per_split = (units + p.splits - 1) / p.splits;
   p.splits = (units + p.units_per_split - 1) / p.units_per_split;
+  p.total_tiles = tiles * p.splits;
+  p.grid = static_cast<unsigned>(p.total_tiles < num_sms ? p.total_tiles : num_sms);
+  // shared memory: raw weight ring (2 units) + as many A/B stages as fit
+  const int raw_bytes = kBM * (type == DSQ_Q8_0 ? 272 : 144);
+  p.raw_stages = 2;
   const int stage_bytes = kAStageBytes + p.tn * 128;
-  p.stages = static_cast<int>((200 * 1024) / stage_bytes);
+  const size_t fixed = 1024 + static_cast<size_t>(p.raw_stages) * raw_bytes + 512;
+  p.stages = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
   if (p.stages > 8) p.stages = 8;
+  p.smem = 1024 + static_cast<size_t>(p.stages) * stage_bytes + static_cast<size_t>(p.raw_stages) * raw_bytes +
+           (3 * p.stages + 2 * p.raw_stages + 5) * sizeof(uint64_t) + 16;
   p.tmem_cols = 32;
-  while (p.tmem_cols < p.tn) p.tmem_cols *= 2;   // TMEM allocations are powers of two
+  while (p.tmem_cols < 2 * p.tn) p.tmem_cols *= 2;   // two accumulators; powers of two
   // the fp16 activation buffer is padded with zero rows to whole token tiles,
   // so every TMA box lies inside the tensor
   p.m_pad = p.tiles_m * p.tn;
@@ -540,14 +643,13 @@ int validate(const char *name, int type, const void *w, int64_t N, int64_t K, co
 }
 
 template <int TYPE>
-int launch_gemm(const PrefillArgs &args, const CUtensorMap &map, const Plan &p, cudaStream_t stream) {
-  const size_t smem = 1024 + static_cast<size_t>(p.stages) * (kAStageBytes + p.tn * 128) +
-                      (3 * p.stages + 2) * sizeof(uint64_t) + 16;
+int launch_gemm(const PrefillArgs &args, const CUtensorMap &map_x, const CUtensorMap &map_w, const Plan &p,
+                cudaStream_t stream) {
   auto kern = prefill_kernel<TYPE>;
-  const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "prefill");
+  const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  dim3 grid(static_cast<unsigned>(p.tiles_m), static_cast<unsigned>(p.tiles_n), static_cast<unsigned>(p.splits));
-  kern<<<grid, kThreads, smem, stream>>>(map, args);
+  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, map_x, map_w, args);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
 
@@ -559,7 +661,7 @@ extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, in
   if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
-  return make_plan(N, K, M, sms).total;
+  return make_plan(type, N, K, M, sms).total;
 }
 
 extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
@@ -573,10 +675,11 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int sms = 0;
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
-  const Plan p = make_plan(N, K, M, sms);
+  const Plan p = make_plan(type, N, K, M, sms);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.stages >= 2, DSQ_ERR_SHAPE, "dsq_gemm_prefill: no pipeline fits");
   auto enc = encode_fn();
   DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
 
@@ -585,42 +688,67 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int32_t *shift = reinterpret_cast<int32_t *>(ws + p.shift_off);
   float *part = reinterpret_cast<float *>(ws + p.part_off);
 
-  CUtensorMap map;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(p.m_pad)};
-  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.tn)};
-  const cuuint32_t estride[2] = {1u, 1u};
-  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, gdim, gstride, box, estride,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: tensor map encode failed (%d)", (int)cr);
+  // activation tiles: fp16 [m_pad][K], 64 x tn boxes, 128-byte swizzle
+  CUtensorMap map_x, map_w;
+  {
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(p.m_pad)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.tn)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, gdim, gstride, box, estride,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: activation tensor map (%d)", (int)cr);
+  }
+  // raw weight units: the packed rows viewed as uint32 [N][row_bytes/4],
+  // one 256-element unit (68 or 36 words) x 128 rows per box, rows past N
+  // read as zero (a zero block dequantizes to zero)
+  {
+    const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+    const cuuint32_t unit_words = type == DSQ_Q8_0 ? 68u : 36u;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kBM)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box,
+                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: weight tensor map (%d)", (int)cr);
+  }
 
   cudaStream_t st = as_stream(stream);
-  x_to_f16_kernel<<<static_cast<unsigned>(p.m_pad), 256, 0, st>>>(x, M, K, x16, shift);
+  cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K, x16,
+                             shift);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: x_to_f16: %s", cudaGetErrorString(e));
   rc = after_launch("dsq_gemm_prefill: x_to_f16");
   if (rc != DSQ_OK) return rc;
 
   PrefillArgs args{};
-  args.w = static_cast<const uint8_t *>(w);
   args.N = N;
   args.K = K;
   args.M = M;
-  args.row_bytes = static_cast<int64_t>(dsq_row_bytes(type, K));
   args.shift = shift;
   args.y = p.splits > 1 ? part : y;
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
   args.stages = p.stages;
+  args.raw_stages = p.raw_stages;
   args.tmem_cols = p.tmem_cols;
+  args.tiles_m = p.tiles_m;
+  args.tiles_n = p.tiles_n;
+  args.total_tiles = p.total_tiles;
   args.wait = ctl;
-  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, map, p, st) : launch_gemm<DSQ_Q4_K>(args, map, p, st);
+  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, map_x, map_w, p, st)
+                        : launch_gemm<DSQ_Q4_K>(args, map_x, map_w, p, st);
   if (rc != DSQ_OK) return rc;
   if (p.splits > 1) {
     const int64_t total = M * N;
     const int64_t blocks = (total / 4 + 255) / 256 + 1;
     const unsigned grid = static_cast<unsigned>(blocks < 8 * sms ? blocks : 8 * sms);
-    splitk_reduce_kernel<<<grid, 256, 0, st>>>(part, total, p.splits, y);
+    e = launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(256), 0, st, static_cast<const float *>(part), total,
+                   p.splits, y);
+    if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: reduce: %s", cudaGetErrorString(e));
     rc = after_launch("dsq_gemm_prefill: split-k reduce");
   }
   return rc;

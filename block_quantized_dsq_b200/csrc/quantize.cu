@@ -23,6 +23,8 @@ __device__ __forceinline__ float q8_code(float x, float d) {
 __global__ void __launch_bounds__(256) act_q8_kernel(const float4 *__restrict__ x, int64_t nblocks,
                                                      int8_t *__restrict__ xq, float *__restrict__ xd,
                                                      int32_t *__restrict__ xs) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t blk = tid >> 3;
   const int sub = threadIdx.x & 7;
@@ -155,7 +157,9 @@ extern "C" int dsq_quantize_act_q8(const float *x, int64_t M, int64_t K, int8_t 
   const int64_t nblocks = M * (K / 32);
   const int64_t threads = nblocks * 8;
   const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
-  act_q8_kernel<<<grid, 256, 0, as_stream(stream)>>>(reinterpret_cast<const float4 *>(x), nblocks, xq, xd, xs);
+  const cudaError_t e = launch_pdl(act_q8_kernel, dim3(grid), dim3(256), 0, as_stream(stream),
+                                   reinterpret_cast<const float4 *>(x), nblocks, xq, xd, xs);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_quantize_act_q8: %s", cudaGetErrorString(e));
   return after_launch("dsq_quantize_act_q8");
 }
 
