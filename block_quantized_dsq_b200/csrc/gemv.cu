@@ -255,9 +255,9 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   const int sub = lane / G, j = lane % G;
   ActSlice act;
   int64_t cached = -1;  // (group * nunits + unit) currently in registers
+  int slot = 0;         // ring position kept incrementally (no division per chunk)
+  uint32_t parity = 0;
   for (int64_t k = 0; k < mine; ++k) {
-    const int slot = static_cast<int>(k % S);
-    const uint32_t parity = static_cast<uint32_t>((k / S) & 1);
     const bool ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
     if (!ok) {
       if (lane == 0) {
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       int seg;
       int64_t local;
       locate(a, row, seg, local);
-      const int64_t group = local / a.group_rows;
+      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
       const uint8_t *rowp = ring + static_cast<size_t>(slot) * a.slot_bytes + static_cast<size_t>(sub) * a.row_bytes;
       for (int u = j; u < a.nunits; u += G) {
         const int64_t key = group * a.nunits + u;
@@ -310,6 +310,10 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       const int64_t c2 = warp + (k + S) * W;
       const int64_t ra2 = r0 + c2 * RPC, rb2 = min(ra2 + RPC, r1);
       issue_rows(a, ra2, rb2, ring + static_cast<size_t>(slot) * a.slot_bytes, &bars[slot], policy);
+    }
+    if (++slot == S) {
+      slot = 0;
+      parity ^= 1u;
     }
   }
 }

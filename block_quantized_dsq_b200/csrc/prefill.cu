@@ -30,8 +30,6 @@
 //    coalesced across the 32 rows of a warp);
 //  * every wait is bounded; an expired wait records a timeout, stops every
 //    role, drains copies and MMAs in flight, frees TMEM and returns.
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "../../include/dsq_test.h"
@@ -40,27 +38,34 @@
 namespace dsq {
 namespace {
 
-constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBM = 128;          // weight rows per MMA (the MMA's M)
+constexpr int kHalves = 2;        // a CTA tile holds 2 x 128 weight rows sharing each activation stage
+constexpr int kTileN = kBM * kHalves;   // weight rows per CTA tile
 constexpr int kBK = 64;           // K elements per pipeline stage
-constexpr int kAStageBytes = kBM * kBK * 2;   // 16 KB
+constexpr int kAColsHalf = kBK / 2;     // TMEM columns of one half's A stage (2 fp16 per column)
+constexpr int kAColsStage = kHalves * kAColsHalf;   // 64
+constexpr int kTmemCols = 512;    // the CTA owns all of TMEM (1 CTA per SM)
 // warp roles
-constexpr int kWarpX = 0;         // TMA producer: fp16 activation tiles
-constexpr int kWarpW = 1;         // TMA producer: raw weight units
-constexpr int kWarpMma = 2;       // TMEM owner, tcgen05.mma issuer
-constexpr int kWarpConv0 = 3;     // warps 3..6: dequantize raw units into A stages
-constexpr int kWarpEpi0 = 7;      // warps 7..10: TMEM -> global epilogue
-constexpr int kThreads = 11 * 32;
+constexpr int kWarpX = 0;         // bulk-copy producer: fp16 activation stages
+constexpr int kWarpMma = 1;       // TMEM owner, tcgen05.mma issuer
+constexpr int kWarpConv0 = 2;     // warps 2..9: one weight row per thread, dequantize into TMEM
+constexpr int kConvWarps = 8;
+constexpr int kWarpEpi0 = kWarpConv0 + kConvWarps;   // warps 10..13: TMEM -> global epilogue
+constexpr int kThreads = (kWarpEpi0 + 4) * 32;
 
 struct PrefillArgs {
+  const uint8_t *w;       // packed weight rows
+  int64_t row_bytes;
   int64_t N, K, M;
+  const __half *x16;      // fp16 activations, K-blocked and swizzled (see x_to_f16_kernel)
+  int64_t m_pad;          // rows of x16 (whole token tiles)
   const int32_t *shift;   // [M] activation row shifts
   float *y;               // [M][N], or [splits][M][N] partials
   int units_per_split;    // 256-element units of K per split
   int splits;
   int tn;                 // tokens per tile (MMA N): 32..256, multiple of 32
-  int stages;             // A/B pipeline stages
-  int raw_stages;         // raw weight unit slots
-  int tmem_cols;          // two accumulators of tn columns
+  int stages_b;           // activation stages in shared memory
+  int stages_a;           // dequantized weight stages in TMEM
   int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
 };
@@ -173,48 +178,38 @@ __device__ __forceinline__ void dequant_piece(const RawUnit<TYPE> &u, int p, uin
   else piece_q4_k(u, p, out);
 }
 
-// Store one row's 64-element piece into a 128B-swizzled K-major stage:
-// row r at r*128, 16-byte chunk c at chunk position c ^ (r & 7).
-__device__ __forceinline__ void store_piece_sw128(uint8_t *stage, int r, const uint32_t (&v)[32]) {
-  uint8_t *row = stage + r * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 q = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-    *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = q;
-  }
-}
 
 // ------------------------------------------------------------------ GEMM ---
+// TMEM map (512 columns x 128 lanes): [0, 2*tn) the fp32 accumulators of the
+// two halves (half h at h*tn); then stages_a dequantized-weight stages of
+// 64 columns each (half h at +32h), lane = row of the half, each column two
+// consecutive fp16 K elements.  The MMA reads A from TMEM and B (the
+// activation tile) from shared memory, so shared memory carries only the
+// activation stream.
 struct Smem {
-  uint8_t *a;          // stages x 16 KB: dequantized weight tiles (MMA A)
-  uint8_t *b;          // stages x tn*128: activation tiles (MMA B)
-  uint8_t *raw;        // raw_stages x 128 rows x unit bytes: raw weight units
-  uint64_t *afull;     // converters stored a stage (count 4)
-  uint64_t *bfull;     // activation tile landed (1 + tx)
-  uint64_t *sempty;    // MMA finished reading a stage (commit)
-  uint64_t *rfull;     // raw unit landed (1 + tx)
-  uint64_t *rempty;    // converters copied a raw unit out (count 4)
-  uint64_t *accfull;   // accumulator complete (commit), x2
-  uint64_t *accempty;  // epilogue drained an accumulator (count 4), x2
+  uint8_t *b;          // stages_b x tn*128: activation tiles (MMA B)
+  uint64_t *bfull;     // activation stage landed (1 + tx)
+  uint64_t *bempty;    // MMA finished reading an activation stage (commit)
+  uint64_t *afull;     // converters stored a TMEM weight stage (count 8 warps)
+  uint64_t *aempty;    // MMA finished reading a TMEM weight stage (commit)
+  uint64_t *accfull;   // accumulators complete (commit)
+  uint64_t *accempty;  // epilogue drained the accumulators (count 4)
   uint64_t *drain;     // MMA drain after an abort
   uint32_t *tmem;      // TMEM base address
   volatile int *abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int stages, int tn, int raw_stages, int raw_bytes) {
+__device__ __forceinline__ Smem carve(uint8_t *base, int stages_b, int stages_a, int tn) {
   Smem s;
-  s.a = base;
-  s.b = s.a + static_cast<size_t>(stages) * kAStageBytes;
-  s.raw = s.b + static_cast<size_t>(stages) * tn * 128;
-  uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(raw_stages) * raw_bytes);
-  s.afull = p;
-  s.bfull = s.afull + stages;
-  s.sempty = s.bfull + stages;
-  s.rfull = s.sempty + stages;
-  s.rempty = s.rfull + raw_stages;
-  s.accfull = s.rempty + raw_stages;
-  s.accempty = s.accfull + 2;
-  s.drain = s.accempty + 2;
+  s.b = base;
+  uint64_t *p = reinterpret_cast<uint64_t *>(s.b + static_cast<size_t>(stages_b) * tn * 128);
+  s.bfull = p;
+  s.bempty = s.bfull + stages_b;
+  s.afull = s.bempty + stages_b;
+  s.aempty = s.afull + stages_a;
+  s.accfull = s.aempty + stages_a;
+  s.accempty = s.accfull + 1;
+  s.drain = s.accempty + 1;
   s.tmem = reinterpret_cast<uint32_t *>(s.drain + 1);
   s.abort = reinterpret_cast<volatile int *>(s.tmem + 1);
   return s;
@@ -227,10 +222,12 @@ __device__ __forceinline__ void set_abort(const Smem &s, const WaitCtl &w) {
 }
 
 // One thread's bounded wait; on expiry (or an abort raised elsewhere) it
-// raises the CTA abort flag and returns false.
-__device__ __forceinline__ bool wait_or_abort(const Smem &s, uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+// raises the CTA abort flag and returns false.  sleep_ns: poll back-off for
+// waiters off the critical path.
+__device__ __forceinline__ bool wait_or_abort(const Smem &s, uint64_t *bar, uint32_t parity, const WaitCtl &w,
+                                              uint32_t sleep_ns = 0) {
   if (aborted(s)) return false;
-  if (mbar_wait_for(bar, parity, w.limit_ns)) return true;
+  if (mbar_wait_for(bar, parity, w.limit_ns, sleep_ns)) return true;
   set_abort(s, w);
   return false;
 }
@@ -248,57 +245,54 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   const int64_t rest = t / a.tiles_m;
   tl.split = static_cast<int>(rest % a.splits);
   tl.m0 = m * a.tn;
-  tl.n0 = (rest / a.splits) * kBM;
+  tl.n0 = (rest / a.splits) * kTileN;
   tl.u0 = tl.split * a.units_per_split;
   tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
   return tl;
 }
 
-// Persistent CTA: tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Every role
-// walks the same tile sequence; the A/B ring, the raw ring and the two TMEM
-// accumulators carry their phases across tiles.
+// Persistent CTA over tiles of 256 weight rows x tn tokens x one K split:
+// tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Each 64-K stage holds the
+// activation tile once (shared memory) and the two 128-row weight halves
+// (TMEM); the MMA warp issues both halves against the same activation tile.
 template <int TYPE>
-__global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
-  constexpr int RAW_BYTES = kBM * UB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Smem s = carve(base, a.stages, a.tn, a.raw_stages, RAW_BYTES);
+  const Smem s = carve(base, a.stages_b, a.stages_a, a.tn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = a.stages, R = a.raw_stages;
+  const int SB = a.stages_b, SA = a.stages_a;
   const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&s.afull[i], 4);
+    for (int i = 0; i < SB; ++i) {
       mbar_init(&s.bfull[i], 1);
-      mbar_init(&s.sempty[i], 1);
+      mbar_init(&s.bempty[i], 1);
     }
-    for (int i = 0; i < R; ++i) {
-      mbar_init(&s.rfull[i], 1);
-      mbar_init(&s.rempty[i], 4);
+    for (int i = 0; i < SA; ++i) {
+      mbar_init(&s.afull[i], kConvWarps);
+      mbar_init(&s.aempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.accfull[i], 1);
-      mbar_init(&s.accempty[i], 4);
-    }
+    mbar_init(s.accfull, 1);
+    mbar_init(s.accempty, 4);
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
-    prefetch_tensormap(&tmap_x);
-    prefetch_tensormap(&tmap_w);
   }
-  if (warp == kWarpW && lane == 0 && blockIdx.x < a.total_tiles) {
-    // weights are read-only: start their first units toward L2 while the
+  const int conv = (warp >= kWarpConv0 && warp < kWarpEpi0) ? warp - kWarpConv0 : -1;
+  // converter warp c: half c / 4, TMEM lane quadrant warp % 4 (a warp may only
+  // touch its own quadrant), so its row within the half is 32 * (warp % 4) + lane
+  const int conv_half = conv / 4, conv_rr = 32 * (warp & 3) + lane;
+  if (conv >= 0 && blockIdx.x < a.total_tiles) {
+    // weights are read-only: start this row's first unit toward L2 while the
     // activation-rounding kernel before us finishes
     const Tile tl = tile_of(a, blockIdx.x);
-    for (int u = tl.u0; u < tl.u1 && u < tl.u0 + R; ++u)
-      prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0));
+    const int64_t n = tl.n0 + conv_half * kBM + conv_rr;
+    if (n < a.N) prefetch_l2(a.w + n * a.row_bytes + static_cast<int64_t>(tl.u0) * UB, UB);
   }
   if (warp == kWarpMma) {
-    tmem_alloc(s.tmem, static_cast<uint32_t>(a.tmem_cols));
+    tmem_alloc(s.tmem, static_cast<uint32_t>(kTmemCols));
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -307,159 +301,181 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   pdl_wait();
   const uint32_t tmem_base = *s.tmem;
+  const uint32_t a_col0 = static_cast<uint32_t>(kHalves * a.tn);   // first weight-stage column
 
   if (warp == kWarpX) {
-    // ---------------------------------------------- activation tiles (TMA)
+    // ---------------------------------------- activation stages (bulk copy)
     if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();   // every weight tile re-reads these
+      // ring position kept incrementally (no integer division on this path):
+      // slot sb of round rnd; round r >= 1 first waits for the MMA's release
+      // of that slot in round r - 1
       int64_t gs = 0;
+      int sb = 0;
+      uint32_t rnd = 0;
       for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
         const Tile tl = tile_of(a, t);
         for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it, ++gs) {
-          const int st = static_cast<int>(gs % S);
-          if (gs >= S && !wait_or_abort(s, &s.sempty[st], static_cast<uint32_t>((gs / S - 1) & 1), a.wait)) break;
-          mbar_arrive_expect_tx(&s.bfull[st], stage_b_bytes);
-          tma_load_2d(s.b + static_cast<size_t>(st) * stage_b_bytes, &tmap_x, (tl.u0 * 4 + it) * kBK,
-                      static_cast<int32_t>(tl.m0), &s.bfull[st]);
+          if (rnd > 0 && !wait_or_abort(s, &s.bempty[sb], (rnd - 1) & 1u, a.wait, 64)) break;
+          mbar_arrive_expect_tx(&s.bfull[sb], stage_b_bytes);
+          const int64_t kb = static_cast<int64_t>(tl.u0) * 4 + it;   // 64-element K block
+          bulk_g2s(s.b + static_cast<size_t>(sb) * stage_b_bytes,
+                   reinterpret_cast<const uint8_t *>(a.x16) + (kb * a.m_pad + tl.m0) * 128, stage_b_bytes, &s.bfull[sb],
+                   keep);
+          if (++sb == SB) {
+            sb = 0;
+            ++rnd;
+          }
         }
       }
       if (aborted(s))
-        for (int64_t g = (gs > S ? gs - S : 0); g < gs; ++g)
-          mbar_wait_for(&s.bfull[g % S], static_cast<uint32_t>((g / S) & 1), kDrainLimitNs);
-    }
-  } else if (warp == kWarpW) {
-    // ------------------------------------------- raw weight units (TMA)
-    if (lane == 0) {
-      int64_t gu = 0;
-      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
-        const Tile tl = tile_of(a, t);
-        for (int u = tl.u0; u < tl.u1; ++u, ++gu) {
-          const int rs = static_cast<int>(gu % R);
-          if (gu >= R && !wait_or_abort(s, &s.rempty[rs], static_cast<uint32_t>((gu / R - 1) & 1), a.wait)) break;
-          mbar_arrive_expect_tx(&s.rfull[rs], static_cast<uint32_t>(RAW_BYTES));
-          tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &tmap_w, u * (UB / 4),
-                      static_cast<int32_t>(tl.n0), &s.rfull[rs]);
-        }
-      }
-      if (aborted(s))
-        for (int64_t g = (gu > R ? gu - R : 0); g < gu; ++g)
-          mbar_wait_for(&s.rfull[g % R], static_cast<uint32_t>((g / R) & 1), kDrainLimitNs);
+        for (int64_t g = (gs > SB ? gs - SB : 0); g < gs; ++g)
+          mbar_wait_for(&s.bfull[g % SB], static_cast<uint32_t>((g / SB) & 1), kDrainLimitNs);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(kBM, static_cast<uint32_t>(a.tn), 0);
-      const uint32_t a_base = smem_u32(s.a), b_base = smem_u32(s.b);
-      int64_t gs = 0, i = 0;
+      const uint32_t b_base = smem_u32(s.b);
+      int64_t i = 0;
+      int sb = 0, sa = 0;
+      uint32_t pb = 0, pa = 0;   // phase parity of the current round of each ring
       bool ok = true;
       for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x, ++i) {
         const Tile tl = tile_of(a, t);
-        const int acc = static_cast<int>(i & 1);
-        if (i >= 2 && !wait_or_abort(s, &s.accempty[acc], static_cast<uint32_t>((i / 2 - 1) & 1), a.wait)) {
+        if (i >= 1 && !wait_or_abort(s, s.accempty, static_cast<uint32_t>((i - 1) & 1), a.wait)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * a.tn);
-        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it, ++gs) {
-          const int st = static_cast<int>(gs % S);
-          const uint32_t par = static_cast<uint32_t>((gs / S) & 1);
-          if (!wait_or_abort(s, &s.bfull[st], par, a.wait) || !wait_or_abort(s, &s.afull[st], par, a.wait)) {
+        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it) {
+          if (!wait_or_abort(s, &s.bfull[sb], pb, a.wait) || !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = a_base + static_cast<uint32_t>(st) * kAStageBytes;
-          const uint32_t b_addr = b_base + static_cast<uint32_t>(st) * stage_b_bytes;
+          const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * stage_b_bytes;
+          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_f16(d, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
-                     (it > 0 || k > 0) ? 1u : 0u);
-          umma_commit(&s.sempty[st]);
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bdesc = umma_desc_sw128(b_addr + 32 * k);
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h)
+              umma_f16_ts(tmem_base + static_cast<uint32_t>(h * a.tn),
+                          a_tmem + static_cast<uint32_t>(h * kAColsHalf + 8 * k), bdesc, idesc,
+                          (it > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&s.bempty[sb]);
+          umma_commit(&s.aempty[sa]);
+          if (++sb == SB) {
+            sb = 0;
+            pb ^= 1u;
+          }
+          if (++sa == SA) {
+            sa = 0;
+            pa ^= 1u;
+          }
         }
-        if (ok) umma_commit(&s.accfull[acc]);
+        if (ok) umma_commit(s.accfull);
       }
       if (!ok) {
         umma_commit(s.drain);
         mbar_wait_for(s.drain, 0, kDrainLimitNs);
       }
     }
-  } else if (warp < kWarpEpi0) {
+  } else if (conv >= 0) {
     // ------------------------------------------ converters (dequantize)
-    const int r = 32 * (warp - kWarpConv0) + lane;   // weight row within the tile
-    int64_t gs = 0, gu = 0;
+    // Thread (half h, row rr) owns weight row 128h + rr of the tile.  It
+    // reads the row's raw 256-element units from global memory (the next
+    // unit is prefetched into L2 while this one is converted) and writes 64
+    // dequantized fp16 per stage into its TMEM lane with one store.
+    const int h = conv_half, rr = conv_rr;
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    int sa = 0;
+    uint32_t rnd = 0;   // ring round; round r >= 1 waits for the release from round r - 1
     bool ok = true;
     for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x) {
       const Tile tl = tile_of(a, t);
-      for (int u = tl.u0; u < tl.u1 && ok; ++u, ++gu) {
-        const int rs = static_cast<int>(gu % R);
-        const bool got = wait_or_abort(s, &s.rfull[rs], static_cast<uint32_t>((gu / R) & 1), a.wait);
-        if (__any_sync(0xffffffffu, !got)) {
-          ok = false;
-          break;
-        }
+      const int64_t n = tl.n0 + h * kBM + rr;
+      const bool live = n < a.N;
+      const uint8_t *rowp = a.w + (live ? n : 0) * a.row_bytes;
+      for (int u = tl.u0; u < tl.u1 && ok; ++u) {
         RawUnit<TYPE> ru;
-        const uint4 *src = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES + r * UB);
+        if (live) {
+          load_unit<TYPE>(ru, rowp + static_cast<int64_t>(u) * UB);
+          if (u + 1 < tl.u1) prefetch_l2(rowp + static_cast<int64_t>(u + 1) * UB, UB);
+        }
 #pragma unroll
-        for (int v = 0; v < RawUnit<TYPE>::kVecs; ++v) ru.v[v] = src[v];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.rempty[rs]);
-#pragma unroll
-        for (int p = 0; p < 4; ++p, ++gs) {
-          const int st = static_cast<int>(gs % S);
-          if (gs >= S) {
-            const bool free_ = wait_or_abort(s, &s.sempty[st], static_cast<uint32_t>((gs / S - 1) & 1), a.wait);
+        for (int p = 0; p < 4; ++p) {
+          if (rnd > 0) {
+            const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
             if (__any_sync(0xffffffffu, !free_)) {
               ok = false;
               break;
             }
           }
           uint32_t v[32];
-          dequant_piece<TYPE>(ru, p, v);
-          store_piece_sw128(s.a + static_cast<size_t>(st) * kAStageBytes, r, v);
-          fence_proxy_async_smem();
+          if (live) {
+            dequant_piece<TYPE>(ru, p, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          tc_fence_after_sync();
+          tmem_st_32cols(tmem_base + lane_addr + a_col0 + static_cast<uint32_t>(sa * kAColsStage + h * kAColsHalf), v);
+          tmem_st_wait();
+          tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s.afull[st]);
+          if (lane == 0) mbar_arrive(&s.afull[sa]);
+          if (++sa == SA) {
+            sa = 0;
+            ++rnd;
+          }
         }
       }
     }
   } else {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = 32 * q + lane;            // weight row within the tile
+    const int r = 32 * q + lane;            // row within each 128-row half
     int64_t i = 0;
     for (int64_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x, ++i) {
       const Tile tl = tile_of(a, t);
-      const int acc = static_cast<int>(i & 1);
-      const bool got = wait_or_abort(s, &s.accfull[acc], static_cast<uint32_t>((i / 2) & 1), a.wait);
+      const bool got = wait_or_abort(s, s.accfull, static_cast<uint32_t>(i & 1), a.wait, 256);
       if (__any_sync(0xffffffffu, !got)) break;
       tc_fence_after_sync();
-      const int64_t n = tl.n0 + r;
       float *y = a.y + static_cast<int64_t>(tl.split) * a.M * a.N;
-      for (int c = 0; c < a.tn / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * a.tn + 32 * c),
-                       v);
-        tmem_ld_wait();
+      for (int hh = 0; hh < kHalves; ++hh) {
+        const int64_t n = tl.n0 + hh * kBM + r;
+        for (int c = 0; c < a.tn / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(hh * a.tn + 32 * c),
+                         v);
+          tmem_ld_wait();
+          if (hh == kHalves - 1 && c == a.tn / 32 - 1) {
+            // every accumulator column is in registers: let the next tile start
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s.accempty);
+          }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int64_t m = tl.m0 + 32 * c + j;
-          if (m < a.M && n < a.N) {
-            const int sft = __ldg(a.shift + m);
-            const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
-            y[m * a.N + n] = __fmul_rn(__uint_as_float(v[j]), scale);
+          for (int j = 0; j < 32; ++j) {
+            const int64_t m = tl.m0 + 32 * c + j;
+            if (m < a.M && n < a.N) {
+              const int sft = __ldg(a.shift + m);
+              const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
+              y[m * a.N + n] = __fmul_rn(__uint_as_float(v[j]), scale);
+            }
           }
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.accempty[acc]);
     }
   }
   tc_fence_before_sync();
   __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, static_cast<uint32_t>(a.tmem_cols));
+    tmem_dealloc(tmem_base, static_cast<uint32_t>(kTmemCols));
   }
 }
 
@@ -467,16 +483,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One CTA per activation row: row max -> shift s (max |x| * 2^s in
 // [2^14, 2^15), 0 for a zero row, clamped to [-64, 64]) -> binary16 RNE of
 // x * 2^s (an exact scaling unless the product is an fp32 subnormal).
-// Rows m >= M (padding up to whole token tiles) are written as zeros.
+// BLOCKED = true writes the layout the MMA reads, so one pipeline stage of
+// activations is a single contiguous bulk copy: K-blocks of 64 elements,
+// block kb of row m at byte ((kb * m_pad + m) * 128), and inside those 128
+// bytes the 16-byte chunk c stored at position c ^ (m & 7) (the 128-byte
+// swizzle).  BLOCKED = false writes plain row-major [M][K].  Rows m >= M
+// (padding up to whole token tiles) are written as zeros.
+template <bool BLOCKED>
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__ x, int64_t M, int64_t K,
-                                                       __half *__restrict__ x16, int32_t *__restrict__ shift) {
+                                                       int64_t m_pad, __half *__restrict__ x16,
+                                                       int32_t *__restrict__ shift) {
   __shared__ float red[8];
   pdl_trigger();
   pdl_wait();
   const int64_t m = blockIdx.x;
+  const int64_t nchunks = K / 8;   // 16-byte chunks of 8 halves per row
+  auto chunk_ptr = [&](int64_t c) -> uint4 * {
+    if (BLOCKED) {
+      const int64_t kb = c / 8, cc = c % 8;
+      return reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(x16) + (kb * m_pad + m) * 128 +
+                                       ((cc ^ (m & 7)) << 4));
+    }
+    return reinterpret_cast<uint4 *>(x16 + m * K) + c;
+  };
   if (m >= M) {
-    uint4 *out = reinterpret_cast<uint4 *>(x16 + m * K);
-    for (int64_t i = threadIdx.x; i < K / 8; i += blockDim.x) out[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) *chunk_ptr(c) = make_uint4(0u, 0u, 0u, 0u);
     if (threadIdx.x == 0) shift[m] = 0;
     return;
   }
@@ -502,12 +533,13 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__
   }
   const float scale = __int_as_float((127 + s) << 23);
   if (threadIdx.x == 0) shift[m] = s;
-  uint2 *out = reinterpret_cast<uint2 *>(x16 + m * K);
-  for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
-    const float4 v = __ldg(row + i);
-    const __half2 lo = __floats2half2_rn(__fmul_rn(v.x, scale), __fmul_rn(v.y, scale));
-    const __half2 hi = __floats2half2_rn(__fmul_rn(v.z, scale), __fmul_rn(v.w, scale));
-    out[i] = make_uint2(h2_bits(lo), h2_bits(hi));
+  for (int64_t c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    const float4 a = __ldg(row + 2 * c), b = __ldg(row + 2 * c + 1);
+    const __half2 h0 = __floats2half2_rn(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale));
+    const __half2 h1 = __floats2half2_rn(__fmul_rn(a.z, scale), __fmul_rn(a.w, scale));
+    const __half2 h2 = __floats2half2_rn(__fmul_rn(b.x, scale), __fmul_rn(b.y, scale));
+    const __half2 h3 = __floats2half2_rn(__fmul_rn(b.z, scale), __fmul_rn(b.w, scale));
+    *chunk_ptr(c) = make_uint4(h2_bits(h0), h2_bits(h1), h2_bits(h2), h2_bits(h3));
   }
 }
 
@@ -558,7 +590,7 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, stages, raw_stages, splits, units_per_split, tmem_cols;
+  int tn, stages_b, stages_a, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
   unsigned grid;
   size_t smem, x16_bytes, shift_off, part_off, total;
@@ -568,24 +600,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int num_sms) {
+Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
   Plan p{};
-  const int64_t tiles_n = (N + kBM - 1) / kBM;
-  // tokens per tile: small M takes the smallest multiple of 32 that covers
-  // it; larger M picks 128 or 256 by a waves x per-tile-cost model (the +64
-  // stands for the per-tile weight dequantization, which does not shrink
-  // with the tile's token count)
-  if (M <= 128) {
-    p.tn = static_cast<int>((M + 31) / 32 * 32);
-  } else {
-    double best = 1e30;
-    for (int tn : {256, 128}) {
-      const int64_t tiles = (M + tn - 1) / tn * tiles_n;
-      const double waves = static_cast<double>((tiles + num_sms - 1) / num_sms);
-      const double cost = waves * (tn + 64);
-      if (cost < best - 1e-9) { best = cost; p.tn = tn; }
-    }
-  }
+  const int64_t tiles_n = (N + kTileN - 1) / kTileN;
+  // tokens per tile: the smallest multiple of 32 that covers M, at most 128
+  // (TMEM holds 2 x tn accumulator columns plus the weight stages, so tn <= 128)
+  p.tn = M <= 128 ? static_cast<int>((M + 31) / 32 * 32) : 128;
   p.tiles_m = (M + p.tn - 1) / p.tn;
   p.tiles_n = tiles_n;
   const int units = static_cast<int>(K / 256);
@@ -597,38 +617,24 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int num_sms) {
   p.splits = (units + p.units_per_split - 1) / p.units_per_split;
   p.total_tiles = tiles * p.splits;
   p.grid = static_cast<unsigned>(p.total_tiles < num_sms ? p.total_tiles : num_sms);
-  // shared memory: raw weight ring (2 units) + as many A/B stages as fit
-  const int raw_bytes = kBM * (type == DSQ_Q8_0 ? 272 : 144);
-  p.raw_stages = 2;
-  const int stage_bytes = kAStageBytes + p.tn * 128;
-  const size_t fixed = 1024 + static_cast<size_t>(p.raw_stages) * raw_bytes + 512;
-  p.stages = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
-  if (p.stages > 8) p.stages = 8;
-  p.smem = 1024 + static_cast<size_t>(p.stages) * stage_bytes + static_cast<size_t>(p.raw_stages) * raw_bytes +
-           (3 * p.stages + 2 * p.raw_stages + 5) * sizeof(uint64_t) + 16;
-  p.tmem_cols = 32;
-  while (p.tmem_cols < 2 * p.tn) p.tmem_cols *= 2;   // two accumulators; powers of two
-  // the fp16 activation buffer is padded with zero rows to whole token tiles,
-  // so every TMA box lies inside the tensor
+  // TMEM: the accumulators (2 halves x tn fp32 columns), then as many
+  // 64-column weight stages as fit (at most 6)
+  p.stages_a = (kTmemCols - kHalves * p.tn) / kAColsStage;
+  if (p.stages_a > 6) p.stages_a = 6;
+  // shared memory: activation stages only (at most 12)
+  const int stage_bytes = p.tn * 128;
+  const size_t fixed = 1024 + 512;
+  p.stages_b = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
+  if (p.stages_b > 12) p.stages_b = 12;
+  p.smem = 1024 + static_cast<size_t>(p.stages_b) * stage_bytes +
+           (2 * p.stages_b + 2 * p.stages_a + 3) * sizeof(uint64_t) + 16;
+  // the fp16 activation buffer is padded with zero rows to whole token tiles
   p.m_pad = p.tiles_m * p.tn;
   p.x16_bytes = align_up(static_cast<size_t>(p.m_pad) * K * 2, 1024);
   p.shift_off = p.x16_bytes;
   p.part_off = align_up(p.shift_off + static_cast<size_t>(p.m_pad) * 4, 1024);
   p.total = p.part_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * 4 : 0);
   return p;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
 }
 
 int validate(const char *name, int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M) {
@@ -643,12 +649,11 @@ int validate(const char *name, int type, const void *w, int64_t N, int64_t K, co
 }
 
 template <int TYPE>
-int launch_gemm(const PrefillArgs &args, const CUtensorMap &map_x, const CUtensorMap &map_w, const Plan &p,
-                cudaStream_t stream) {
+int launch_gemm(const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
   auto kern = prefill_kernel<TYPE>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, map_x, map_w, args);
+  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, args);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
@@ -661,7 +666,7 @@ extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, in
   if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
-  return make_plan(type, N, K, M, sms).total;
+  return make_plan(N, K, M, sms).total;
 }
 
 extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
@@ -675,72 +680,45 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int sms = 0;
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
-  const Plan p = make_plan(type, N, K, M, sms);
+  const Plan p = make_plan(N, K, M, sms);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.stages >= 2, DSQ_ERR_SHAPE, "dsq_gemm_prefill: no pipeline fits");
-  auto enc = encode_fn();
-  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.stages_b >= 2 && p.stages_a >= 2, DSQ_ERR_SHAPE,
+              "dsq_gemm_prefill: no pipeline fits");
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   __half *x16 = reinterpret_cast<__half *>(ws);
   int32_t *shift = reinterpret_cast<int32_t *>(ws + p.shift_off);
   float *part = reinterpret_cast<float *>(ws + p.part_off);
 
-  // activation tiles: fp16 [m_pad][K], 64 x tn boxes, 128-byte swizzle
-  CUtensorMap map_x, map_w;
-  {
-    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(p.m_pad)};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(p.tn)};
-    const cuuint32_t estride[2] = {1u, 1u};
-    const CUresult cr = enc(&map_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, gdim, gstride, box, estride,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: activation tensor map (%d)", (int)cr);
-  }
-  // raw weight units: the packed rows viewed as uint32 [N][row_bytes/4],
-  // one 256-element unit (68 or 36 words) x 128 rows per box, rows past N
-  // read as zero (a zero block dequantizes to zero)
-  {
-    const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
-    const cuuint32_t unit_words = type == DSQ_Q8_0 ? 68u : 36u;
-    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
-    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
-    const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kBM)};
-    const cuuint32_t estride[2] = {1u, 1u};
-    const CUresult cr = enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box,
-                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: weight tensor map (%d)", (int)cr);
-  }
-
   cudaStream_t st = as_stream(stream);
-  cudaError_t e = launch_pdl(x_to_f16_kernel, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K, x16,
-                             shift);
+  cudaError_t e = launch_pdl(x_to_f16_kernel<true>, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K,
+                             static_cast<int64_t>(p.m_pad), x16, shift);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: x_to_f16: %s", cudaGetErrorString(e));
   rc = after_launch("dsq_gemm_prefill: x_to_f16");
   if (rc != DSQ_OK) return rc;
 
   PrefillArgs args{};
+  args.w = static_cast<const uint8_t *>(w);
+  args.row_bytes = static_cast<int64_t>(dsq_row_bytes(type, K));
   args.N = N;
   args.K = K;
   args.M = M;
+  args.x16 = x16;
+  args.m_pad = p.m_pad;
   args.shift = shift;
   args.y = p.splits > 1 ? part : y;
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
-  args.stages = p.stages;
-  args.raw_stages = p.raw_stages;
-  args.tmem_cols = p.tmem_cols;
+  args.stages_b = p.stages_b;
+  args.stages_a = p.stages_a;
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
   args.wait = ctl;
-  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, map_x, map_w, p, st)
-                        : launch_gemm<DSQ_Q4_K>(args, map_x, map_w, p, st);
+  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, p, st) : launch_gemm<DSQ_Q4_K>(args, p, st);
   if (rc != DSQ_OK) return rc;
   if (p.splits > 1) {
     const int64_t total = M * N;
@@ -765,7 +743,7 @@ extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int
   rc = device_ready(nullptr, nullptr);
   if (rc != DSQ_OK) return rc;
   cudaStream_t st = as_stream(stream);
-  x_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, reinterpret_cast<__half *>(x16), shift);
+  x_to_f16_kernel<false><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, M, reinterpret_cast<__half *>(x16), shift);
   rc = after_launch("dsq_test_prefill_operands: x");
   if (rc != DSQ_OK) return rc;
   const int64_t work = N * (K / 256);
