@@ -30,6 +30,7 @@
 //    coalesced across the 32 rows of a warp);
 //  * every wait is bounded; an expired wait records a timeout, stops every
 //    role, drains copies and MMAs in flight, frees TMEM and returns.
+#include <cudaTypedefs.h>
 #include <mutex>
 
 #include "../../include/dsq_test.h"
@@ -51,20 +52,21 @@ constexpr int kWarpMma = 1;       // TMEM owner, tcgen05.mma issuer
 constexpr int kWarpConv0 = 2;     // warps 2..9: one weight row per thread, dequantize into TMEM
 constexpr int kConvWarps = 8;
 constexpr int kWarpEpi0 = kWarpConv0 + kConvWarps;   // warps 10..13: TMEM -> global epilogue
-constexpr int kThreads = (kWarpEpi0 + 4) * 32;
+constexpr int kWarpW = kWarpEpi0 + 4;                 // warp 14: TMA producer of raw weight units
+constexpr int kThreads = (kWarpW + 1) * 32;
 
 struct PrefillArgs {
   const uint8_t *w;       // packed weight rows
   int64_t row_bytes;
   int64_t N, K, M;
-  const __half *x16;      // fp16 activations, K-blocked and swizzled (see x_to_f16_kernel)
-  int64_t m_pad;          // rows of x16 (whole token tiles)
+  const __half *x16;      // fp16 activations, tile-major and swizzled (see x_to_f16_kernel)
   const int32_t *shift;   // [M] activation row shifts
   float *y;               // [M][N], or [splits][M][N] partials
   int units_per_split;    // 256-element units of K per split
   int splits;
   int tn;                 // tokens per tile (MMA N): 32..256, multiple of 32
-  int stages_b;           // activation stages in shared memory
+  int groups_b;           // activation slots in shared memory (one 256-element unit of K each)
+  int raw_slots;          // raw weight unit slots in shared memory (256 rows x unit bytes each)
   int stages_a;           // dequantized weight stages in TMEM
   int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
@@ -187,11 +189,14 @@ __device__ __forceinline__ void dequant_piece(const RawUnit<TYPE> &u, int p, uin
 // activation tile) from shared memory, so shared memory carries only the
 // activation stream.
 struct Smem {
-  uint8_t *b;          // stages_b x tn*128: activation tiles (MMA B)
-  uint64_t *bfull;     // activation stage landed (1 + tx)
-  uint64_t *bempty;    // MMA finished reading an activation stage (commit)
+  uint8_t *b;          // groups_b x 4 x tn*128: activation tiles of one K unit each (MMA B)
+  uint64_t *bfull;     // activation unit landed (1 + tx)
+  uint64_t *bempty;    // MMA finished reading an activation unit (commit)
   uint64_t *afull;     // converters stored a TMEM weight stage (count 8 warps)
   uint64_t *aempty;    // MMA finished reading a TMEM weight stage (commit)
+  uint8_t *raw;        // raw_slots x 256 rows x unit bytes: raw weight units (TMA)
+  uint64_t *rfull;     // raw unit landed (1 + tx)
+  uint64_t *rempty;    // converters copied a raw unit into registers (count 8 warps)
   uint64_t *accfull;   // accumulators complete (commit)
   uint64_t *accempty;  // epilogue drained the accumulators (count 4)
   uint64_t *drain;     // MMA drain after an abort
@@ -199,15 +204,18 @@ struct Smem {
   volatile int *abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int stages_b, int stages_a, int tn) {
+__device__ __forceinline__ Smem carve(uint8_t *base, int groups_b, int stages_a, int tn, int raw_slots, int raw_bytes) {
   Smem s;
   s.b = base;
-  uint64_t *p = reinterpret_cast<uint64_t *>(s.b + static_cast<size_t>(stages_b) * tn * 128);
+  s.raw = s.b + static_cast<size_t>(groups_b) * 4 * tn * 128;
+  uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(raw_slots) * raw_bytes);
   s.bfull = p;
-  s.bempty = s.bfull + stages_b;
-  s.afull = s.bempty + stages_b;
+  s.bempty = s.bfull + groups_b;
+  s.afull = s.bempty + groups_b;
   s.aempty = s.afull + stages_a;
-  s.accfull = s.aempty + stages_a;
+  s.rfull = s.aempty + stages_a;
+  s.rempty = s.rfull + raw_slots;
+  s.accfull = s.rempty + raw_slots;
   s.accempty = s.accfull + 1;
   s.drain = s.accempty + 1;
   s.tmem = reinterpret_cast<uint32_t *>(s.drain + 1);
@@ -256,14 +264,18 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
 // activation tile once (shared memory) and the two 128-row weight halves
 // (TMEM); the MMA warp issues both halves against the same activation tile.
 template <int TYPE>
-__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ PrefillArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
+  constexpr int RAW_BYTES = kTileN * UB;   // one unit of the tile's 256 rows
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Smem s = carve(base, a.stages_b, a.stages_a, a.tn);
+  const Smem s = carve(base, a.groups_b, a.stages_a, a.tn, a.raw_slots, RAW_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int SB = a.stages_b, SA = a.stages_a;
-  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;
+  const int SB = a.groups_b, SA = a.stages_a, SR = a.raw_slots;
+  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;   // one 64-K activation tile
+  const uint32_t group_b_bytes = 4u * stage_b_bytes;                    // one 256-K unit
+  const int units = static_cast<int>(a.K / 256);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SB; ++i) {
@@ -274,22 +286,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       mbar_init(&s.afull[i], kConvWarps);
       mbar_init(&s.aempty[i], 1);
     }
+    for (int i = 0; i < SR; ++i) {
+      mbar_init(&s.rfull[i], 1);
+      mbar_init(&s.rempty[i], kConvWarps);
+    }
     mbar_init(s.accfull, 1);
     mbar_init(s.accempty, 4);
     mbar_init(s.drain, 1);
     *s.abort = 0;
     fence_barrier_init();
+    prefetch_tensormap(&tmap_w);
   }
   const int conv = (warp >= kWarpConv0 && warp < kWarpEpi0) ? warp - kWarpConv0 : -1;
   // converter warp c: half c / 4, TMEM lane quadrant warp % 4 (a warp may only
   // touch its own quadrant), so its row within the half is 32 * (warp % 4) + lane
   const int conv_half = conv / 4, conv_rr = 32 * (warp & 3) + lane;
-  if (conv >= 0 && blockIdx.x < a.total_tiles) {
-    // weights are read-only: start this row's first unit toward L2 while the
+  if (warp == kWarpW && lane == 0 && blockIdx.x < a.total_tiles) {
+    // weights are read-only: start the first units toward L2 while the
     // activation-rounding kernel before us finishes
     const Tile tl = tile_of(a, blockIdx.x);
-    const int64_t n = tl.n0 + conv_half * kBM + conv_rr;
-    if (n < a.N) prefetch_l2(a.w + n * a.row_bytes + static_cast<int64_t>(tl.u0) * UB, UB);
+    for (int u = tl.u0; u < tl.u1 && u < tl.u0 + 2; ++u)
+      for (int h = 0; h < kHalves; ++h)
+        prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0 + h * kBM));
   }
   if (warp == kWarpMma) {
     tmem_alloc(s.tmem, static_cast<uint32_t>(kTmemCols));
@@ -307,21 +325,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // ---------------------------------------- activation stages (bulk copy)
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();   // every weight tile re-reads these
-      // ring position kept incrementally (no integer division on this path):
-      // slot sb of round rnd; round r >= 1 first waits for the MMA's release
-      // of that slot in round r - 1
+      // One bulk copy per 256-element K unit: the activation tile of the
+      // unit is contiguous in the tile-major layout.  Ring position kept
+      // incrementally (no integer division on this path): slot sb of round
+      // rnd; round r >= 1 first waits for the MMA's release from round r - 1.
       int64_t gs = 0;
       int sb = 0;
       uint32_t rnd = 0;
       for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
         const Tile tl = tile_of(a, t);
-        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it, ++gs) {
+        const int64_t mt = tl.m0 / a.tn;
+        for (int u = tl.u0; u < tl.u1; ++u, ++gs) {
           if (rnd > 0 && !wait_or_abort(s, &s.bempty[sb], (rnd - 1) & 1u, a.wait, 64)) break;
-          mbar_arrive_expect_tx(&s.bfull[sb], stage_b_bytes);
-          const int64_t kb = static_cast<int64_t>(tl.u0) * 4 + it;   // 64-element K block
-          bulk_g2s(s.b + static_cast<size_t>(sb) * stage_b_bytes,
-                   reinterpret_cast<const uint8_t *>(a.x16) + (kb * a.m_pad + tl.m0) * 128, stage_b_bytes, &s.bfull[sb],
-                   keep);
+          mbar_arrive_expect_tx(&s.bfull[sb], group_b_bytes);
+          bulk_g2s(s.b + static_cast<size_t>(sb) * group_b_bytes,
+                   reinterpret_cast<const uint8_t *>(a.x16) + (mt * units + u) * static_cast<int64_t>(group_b_bytes),
+                   group_b_bytes, &s.bfull[sb], keep);
           if (++sb == SB) {
             sb = 0;
             ++rnd;
@@ -348,32 +367,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           break;
         }
         tc_fence_after_sync();
-        for (int it = 0; it < 4 * (tl.u1 - tl.u0); ++it) {
-          if (!wait_or_abort(s, &s.bfull[sb], pb, a.wait) || !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
+        for (int u = tl.u0; u < tl.u1 && ok; ++u) {
+          if (!wait_or_abort(s, &s.bfull[sb], pb, a.wait)) {
             ok = false;
             break;
           }
-          tc_fence_after_sync();
-          const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * stage_b_bytes;
-          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
+          for (int kb4 = 0; kb4 < 4; ++kb4) {
+            if (!wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * group_b_bytes + static_cast<uint32_t>(kb4) * stage_b_bytes;
+            const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
+            const bool first = (u == tl.u0 && kb4 == 0);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t bdesc = umma_desc_sw128(b_addr + 32 * k);
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t bdesc = umma_desc_sw128(b_addr + 32 * k);
 #pragma unroll
-            for (int h = 0; h < kHalves; ++h)
-              umma_f16_ts(tmem_base + static_cast<uint32_t>(h * a.tn),
-                          a_tmem + static_cast<uint32_t>(h * kAColsHalf + 8 * k), bdesc, idesc,
-                          (it > 0 || k > 0) ? 1u : 0u);
+              for (int h = 0; h < kHalves; ++h)
+                umma_f16_ts(tmem_base + static_cast<uint32_t>(h * a.tn),
+                            a_tmem + static_cast<uint32_t>(h * kAColsHalf + 8 * k), bdesc, idesc,
+                            (!first || k > 0) ? 1u : 0u);
+            }
+            umma_commit(&s.aempty[sa]);
+            if (++sa == SA) {
+              sa = 0;
+              pa ^= 1u;
+            }
           }
+          if (!ok) break;
           umma_commit(&s.bempty[sb]);
-          umma_commit(&s.aempty[sa]);
           if (++sb == SB) {
             sb = 0;
             pb ^= 1u;
-          }
-          if (++sa == SA) {
-            sa = 0;
-            pa ^= 1u;
           }
         }
         if (ok) umma_commit(s.accfull);
@@ -382,6 +409,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         umma_commit(s.drain);
         mbar_wait_for(s.drain, 0, kDrainLimitNs);
       }
+    }
+  } else if (warp == kWarpW) {
+    // ------------------------------------------- raw weight units (TMA)
+    if (lane == 0) {
+      int64_t gu = 0;
+      int rs = 0;
+      uint32_t rnd = 0;
+      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
+        const Tile tl = tile_of(a, t);
+        for (int u = tl.u0; u < tl.u1; ++u, ++gu) {
+          if (rnd > 0 && !wait_or_abort(s, &s.rempty[rs], (rnd - 1) & 1u, a.wait, 64)) break;
+          mbar_arrive_expect_tx(&s.rfull[rs], static_cast<uint32_t>(RAW_BYTES));
+          for (int h = 0; h < kHalves; ++h)
+            tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES + static_cast<size_t>(h) * kBM * UB, &tmap_w,
+                        u * (UB / 4), static_cast<int32_t>(tl.n0 + h * kBM), &s.rfull[rs]);
+          if (++rs == SR) {
+            rs = 0;
+            ++rnd;
+          }
+        }
+      }
+      if (aborted(s))
+        for (int64_t g = (gu > SR ? gu - SR : 0); g < gu; ++g)
+          mbar_wait_for(&s.rfull[g % SR], static_cast<uint32_t>((g / SR) & 1), kDrainLimitNs);
     }
   } else if (conv >= 0) {
     // ------------------------------------------ converters (dequantize)
@@ -393,17 +444,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     int sa = 0;
     uint32_t rnd = 0;   // ring round; round r >= 1 waits for the release from round r - 1
+    int rs = 0;         // raw unit slot and its phase parity
+    uint32_t rpar = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x) {
       const Tile tl = tile_of(a, t);
-      const int64_t n = tl.n0 + h * kBM + rr;
-      const bool live = n < a.N;
-      const uint8_t *rowp = a.w + (live ? n : 0) * a.row_bytes;
       for (int u = tl.u0; u < tl.u1 && ok; ++u) {
+        const bool got = wait_or_abort(s, &s.rfull[rs], rpar, a.wait);
+        if (__any_sync(0xffffffffu, !got)) {
+          ok = false;
+          break;
+        }
         RawUnit<TYPE> ru;
-        if (live) {
-          load_unit<TYPE>(ru, rowp + static_cast<int64_t>(u) * UB);
-          if (u + 1 < tl.u1) prefetch_l2(rowp + static_cast<int64_t>(u + 1) * UB, UB);
+        const uint4 *src = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES +
+                                                           static_cast<size_t>(h * kBM + rr) * UB);
+#pragma unroll
+        for (int v = 0; v < RawUnit<TYPE>::kVecs; ++v) ru.v[v] = src[v];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.rempty[rs]);
+        if (++rs == SR) {
+          rs = 0;
+          rpar ^= 1u;
         }
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -415,12 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
           }
           uint32_t v[32];
-          if (live) {
-            dequant_piece<TYPE>(ru, p, v);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
+          dequant_piece<TYPE>(ru, p, v);   // rows past N arrive as zero blocks: zeros
           tc_fence_after_sync();
           tmem_st_32cols(tmem_base + lane_addr + a_col0 + static_cast<uint32_t>(sa * kAColsStage + h * kAColsHalf), v);
           tmem_st_wait();
@@ -434,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         }
       }
     }
-  } else {
+  } else if (warp >= kWarpEpi0) {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int r = 32 * q + lane;            // row within each 128-row half
@@ -483,26 +539,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 // One CTA per activation row: row max -> shift s (max |x| * 2^s in
 // [2^14, 2^15), 0 for a zero row, clamped to [-64, 64]) -> binary16 RNE of
 // x * 2^s (an exact scaling unless the product is an fp32 subnormal).
-// BLOCKED = true writes the layout the MMA reads, so one pipeline stage of
-// activations is a single contiguous bulk copy: K-blocks of 64 elements,
-// block kb of row m at byte ((kb * m_pad + m) * 128), and inside those 128
-// bytes the 16-byte chunk c stored at position c ^ (m & 7) (the 128-byte
-// swizzle).  BLOCKED = false writes plain row-major [M][K].  Rows m >= M
-// (padding up to whole token tiles) are written as zeros.
+// BLOCKED = true writes the tile-major layout the MMA reads, so the
+// activations of one token tile for one 256-element unit of K are a single
+// contiguous block (one bulk copy): for token tile mt = m / tn, unit ub and
+// 64-element sub-block kb4, the 128 bytes of row m start at
+//   (((mt * units + ub) * 4 + kb4) * tn + m % tn) * 128,
+// and inside them the 16-byte chunk c sits at position c ^ (m & 7) (the
+// 128-byte swizzle).  BLOCKED = false writes plain row-major [M][K].  Rows
+// m >= M (padding up to whole token tiles) are written as zeros.
 template <bool BLOCKED>
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__ x, int64_t M, int64_t K,
-                                                       int64_t m_pad, __half *__restrict__ x16,
+                                                       int64_t tn, __half *__restrict__ x16,
                                                        int32_t *__restrict__ shift) {
   __shared__ float red[8];
   pdl_trigger();
   pdl_wait();
   const int64_t m = blockIdx.x;
   const int64_t nchunks = K / 8;   // 16-byte chunks of 8 halves per row
+  const int64_t units = K / 256;
   auto chunk_ptr = [&](int64_t c) -> uint4 * {
     if (BLOCKED) {
       const int64_t kb = c / 8, cc = c % 8;
-      return reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(x16) + (kb * m_pad + m) * 128 +
-                                       ((cc ^ (m & 7)) << 4));
+      const int64_t off = ((((m / tn) * units + kb / 4) * 4 + kb % 4) * tn + m % tn) * 128 + ((cc ^ (m & 7)) << 4);
+      return reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(x16) + off);
     }
     return reinterpret_cast<uint4 *>(x16 + m * K) + c;
   };
@@ -590,7 +649,7 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, stages_b, stages_a, splits, units_per_split;
+  int tn, groups_b, stages_a, raw_slots, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
   unsigned grid;
   size_t smem, x16_bytes, shift_off, part_off, total;
@@ -600,7 +659,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
+Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int num_sms) {
   Plan p{};
   const int64_t tiles_n = (N + kTileN - 1) / kTileN;
   // tokens per tile: the smallest multiple of 32 that covers M, at most 128
@@ -621,13 +680,17 @@ Plan make_plan(int64_t N, int64_t K, int64_t M, int num_sms) {
   // 64-column weight stages as fit (at most 6)
   p.stages_a = (kTmemCols - kHalves * p.tn) / kAColsStage;
   if (p.stages_a > 6) p.stages_a = 6;
-  // shared memory: activation stages only (at most 12)
-  const int stage_bytes = p.tn * 128;
+  // shared memory: raw weight slots (one 256-element unit of the tile's 256
+  // rows each; two when they fit, else one) and activation slots (one unit
+  // of K each; two or more)
+  const int group_bytes = 4 * p.tn * 128;
+  const int raw_bytes = kTileN * (type == DSQ_Q8_0 ? 272 : 144);
   const size_t fixed = 1024 + 512;
-  p.stages_b = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
-  if (p.stages_b > 12) p.stages_b = 12;
-  p.smem = 1024 + static_cast<size_t>(p.stages_b) * stage_bytes +
-           (2 * p.stages_b + 2 * p.stages_a + 3) * sizeof(uint64_t) + 16;
+  p.raw_slots = (fixed + 2 * static_cast<size_t>(raw_bytes) + 2 * group_bytes <= kSmemLimit) ? 2 : 1;
+  p.groups_b = static_cast<int>((kSmemLimit - fixed - static_cast<size_t>(p.raw_slots) * raw_bytes) / group_bytes);
+  if (p.groups_b > 6) p.groups_b = 6;
+  p.smem = 1024 + static_cast<size_t>(p.groups_b) * group_bytes + static_cast<size_t>(p.raw_slots) * raw_bytes +
+           (2 * p.groups_b + 2 * p.stages_a + 2 * p.raw_slots + 3) * sizeof(uint64_t) + 16;
   // the fp16 activation buffer is padded with zero rows to whole token tiles
   p.m_pad = p.tiles_m * p.tn;
   p.x16_bytes = align_up(static_cast<size_t>(p.m_pad) * K * 2, 1024);
@@ -648,12 +711,28 @@ int validate(const char *name, int type, const void *w, int64_t N, int64_t K, co
   return DSQ_OK;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
 template <int TYPE>
-int launch_gemm(const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
+int launch_gemm(const CUtensorMap &map_w, const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
   auto kern = prefill_kernel<TYPE>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, args);
+  // ask for no more shared-memory carveout than the kernel uses: the rest is L1
+  const int carve = static_cast<int>((p.smem * 100 + 228 * 1024 - 1) / (228 * 1024));
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
+  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, map_w, args);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
@@ -666,7 +745,7 @@ extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, in
   if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
-  return make_plan(N, K, M, sms).total;
+  return make_plan(type, N, K, M, sms).total;
 }
 
 extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
@@ -680,11 +759,11 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int sms = 0;
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
-  const Plan p = make_plan(N, K, M, sms);
+  const Plan p = make_plan(type, N, K, M, sms);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.stages_b >= 2 && p.stages_a >= 2, DSQ_ERR_SHAPE,
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.groups_b >= 2 && p.stages_a >= 2 && p.raw_slots >= 1, DSQ_ERR_SHAPE,
               "dsq_gemm_prefill: no pipeline fits");
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -692,9 +771,27 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int32_t *shift = reinterpret_cast<int32_t *>(ws + p.shift_off);
   float *part = reinterpret_cast<float *>(ws + p.part_off);
 
+  // raw weight units: the packed rows viewed as uint32 [N][row_bytes/4], one
+  // 256-element unit (68 or 36 words) x 128 rows per box; rows past N read as
+  // zero (a zero block dequantizes to zero)
+  auto enc = encode_fn();
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
+  CUtensorMap map_w;
+  {
+    const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+    const cuuint32_t unit_words = type == DSQ_Q8_0 ? 68u : 36u;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kBM)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box,
+                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: weight tensor map (%d)", (int)cr);
+  }
   cudaStream_t st = as_stream(stream);
   cudaError_t e = launch_pdl(x_to_f16_kernel<true>, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K,
-                             static_cast<int64_t>(p.m_pad), x16, shift);
+                             static_cast<int64_t>(p.tn), x16, shift);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: x_to_f16: %s", cudaGetErrorString(e));
   rc = after_launch("dsq_gemm_prefill: x_to_f16");
   if (rc != DSQ_OK) return rc;
@@ -706,19 +803,19 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   args.K = K;
   args.M = M;
   args.x16 = x16;
-  args.m_pad = p.m_pad;
   args.shift = shift;
   args.y = p.splits > 1 ? part : y;
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
-  args.stages_b = p.stages_b;
+  args.groups_b = p.groups_b;
+  args.raw_slots = p.raw_slots;
   args.stages_a = p.stages_a;
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
   args.wait = ctl;
-  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(args, p, st) : launch_gemm<DSQ_Q4_K>(args, p, st);
+  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(map_w, args, p, st) : launch_gemm<DSQ_Q4_K>(map_w, args, p, st);
   if (rc != DSQ_OK) return rc;
   if (p.splits > 1) {
     const int64_t total = M * N;
