@@ -15,21 +15,25 @@
 // mantissa bits) keeps the operand rounding at ~3e-4 relative L2 on this
 // workload; bfloat16 operands would give ~2.3e-3, above the 2e-3 bar.
 //
-// Kernel (one CTA per 128 weight rows x TN tokens x K-split):
-//  * the weight tile is the MMA's A operand (M = 128 rows of W), the
-//    activation tile its B operand (N = TN tokens) -- "swap AB", so small
-//    token counts still use a full 128-row MMA and the weight stream stays
-//    HBM-efficient down to one token;
-//  * warp 0: TMA producer of the activation tiles (fp16, 128-byte swizzle);
-//  * warp 1: allocates TMEM and issues tcgen05.mma (kind::f16, fp32
-//    accumulate in TMEM), releasing smem stages with tcgen05.commit;
-//  * warps 2-5: each thread owns one weight row: it streams the row's raw
-//    blocks from global memory (one 256-element unit ahead), dequantizes 64
-//    elements per stage into the 128-byte-swizzled K-major layout the MMA
-//    reads, then runs the epilogue (tcgen05.ld -> scale by 2^-s_m -> global,
-//    coalesced across the 32 rows of a warp);
-//  * every wait is bounded; an expired wait records a timeout, stops every
-//    role, drains copies and MMAs in flight, frees TMEM and returns.
+// GEMM kernel: persistent clusters of two CTAs (one per SM) sharing one
+// tcgen05 MMA of M = 256 weight rows (cta_group::2).  A pair tile is 256
+// weight rows x tn tokens x one K split; CTA r of the pair owns weight rows
+// 128r..128r+127 and holds tokens r*tn/2 .. r*tn/2 + tn/2 - 1 of the tile:
+//  * the dequantized weights are the MMA's A operand and live in TMEM (each
+//    CTA's 128 lanes = its 128 rows), the activations are the B operand in
+//    shared memory (each CTA holds half of the N = tn columns);  "swap AB"
+//    keeps small token counts on full 128-lane MMAs;
+//  * per CTA: warp 0 streams activation stages (bulk copies of a tile-major
+//    fp16 layout, 64 K x tn/2 tokens each); warp 14 streams raw weight units
+//    (TMA, 128 rows x 256 K); warps 2-9 dequantize (two threads per weight
+//    row, alternate 64-K stages) into the TMEM A ring; warps 10-13 drain the
+//    fp32 accumulators (tcgen05.ld -> scale by 2^-s_m -> global);
+//  * warp 1 of the even CTA issues the pair MMAs; warp 1 of the odd CTA
+//    forwards "activation stage landed" to it.  MMA completion releases
+//    stages in both CTAs through multicast tcgen05.commit;
+//  * every wait is bounded; an expired wait records a timeout, raises the
+//    abort flag of both CTAs, drains copies and MMAs in flight, and the pair
+//    meets at a final cluster barrier before TMEM is freed.
 #include <cudaTypedefs.h>
 #include <mutex>
 
@@ -39,62 +43,46 @@
 namespace dsq {
 namespace {
 
-constexpr int kBM = 128;          // weight rows per MMA (the MMA's M)
-constexpr int kHalves = 2;        // a CTA tile holds 2 x 128 weight rows sharing each activation stage
-constexpr int kTileN = kBM * kHalves;   // weight rows per CTA tile
-constexpr int kBK = 64;           // K elements per pipeline stage
-constexpr int kAColsHalf = kBK / 2;     // TMEM columns of one half's A stage (2 fp16 per column)
-constexpr int kAColsStage = kHalves * kAColsHalf;   // 64
-constexpr int kTmemCols = 512;    // the CTA owns all of TMEM (1 CTA per SM)
+constexpr int kRows = 128;          // weight rows per CTA (TMEM lanes)
+constexpr int kTileN = 2 * kRows;   // weight rows per pair tile (the MMA's M)
+constexpr int kBK = 64;             // K elements per pipeline stage
+constexpr int kAColsStage = kBK / 2;   // TMEM columns of one A stage (2 fp16 per column)
+constexpr int kTmemCols = 512;      // the CTA owns all of TMEM (1 CTA per SM)
+constexpr int kMaxStagesA = 8;
 // warp roles
 constexpr int kWarpX = 0;         // bulk-copy producer: fp16 activation stages
-constexpr int kWarpMma = 1;       // TMEM owner, tcgen05.mma issuer
-constexpr int kWarpConv0 = 2;     // warps 2..9: one weight row per thread, dequantize into TMEM
+constexpr int kWarpMma = 1;       // TMEM owner; MMA issuer (even CTA) / activation relay (odd CTA)
+constexpr int kWarpConv0 = 2;     // warps 2..9: dequantize into TMEM
 constexpr int kConvWarps = 8;
 constexpr int kWarpEpi0 = kWarpConv0 + kConvWarps;   // warps 10..13: TMEM -> global epilogue
 constexpr int kWarpW = kWarpEpi0 + 4;                 // warp 14: TMA producer of raw weight units
 constexpr int kThreads = (kWarpW + 1) * 32;
 
 struct PrefillArgs {
-  const uint8_t *w;       // packed weight rows
-  int64_t row_bytes;
   int64_t N, K, M;
   const __half *x16;      // fp16 activations, tile-major and swizzled (see x_to_f16_kernel)
   const int32_t *shift;   // [M] activation row shifts
   float *y;               // [M][N], or [splits][M][N] partials
   int units_per_split;    // 256-element units of K per split
   int splits;
-  int tn;                 // tokens per tile (MMA N): 32..256, multiple of 32
-  int groups_b;           // activation slots in shared memory (one 256-element unit of K each)
-  int raw_slots;          // raw weight unit slots in shared memory (256 rows x unit bytes each)
-  int stages_a;           // dequantized weight stages in TMEM
+  int tn;                 // tokens per pair tile (MMA N): 32..256, multiple of 32
+  int slots_b;            // activation slots in shared memory (stages_per_slot x 64 K x tn/2 tokens each)
+  int stages_per_slot;    // 1, 2 or 4 stages of one K unit per activation copy
+  int slots_raw;          // raw weight unit slots in shared memory (128 rows x 256 K each)
+  int stages_a;           // dequantized weight stages in TMEM (even)
   int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
 };
 
 // ---------------------------------------------------------------- dequant --
-// 256-element unit of one weight row in registers: Q8_0 = 8 blocks (272 B),
-// Q4_K = one super-block (144 B).
-template <int TYPE> struct RawUnit;
-template <> struct RawUnit<DSQ_Q8_0> { static constexpr int kVecs = 17; uint4 v[17]; };
-template <> struct RawUnit<DSQ_Q4_K> { static constexpr int kVecs = 9; uint4 v[9]; };
 template <int TYPE> __host__ __device__ constexpr int unit_bytes() { return TYPE == DSQ_Q8_0 ? 272 : 144; }
-
-template <int TYPE>
-__device__ __forceinline__ void load_unit(RawUnit<TYPE> &u, const uint8_t *p) {
-  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
-#pragma unroll
-  for (int i = 0; i < RawUnit<TYPE>::kVecs; ++i) u.v[i] = __ldg(p4 + i);
-}
-
-template <int TYPE>
-__device__ __forceinline__ uint32_t word_of(const RawUnit<TYPE> &u, int i) {
-  const uint4 &v = u.v[i >> 2];
-  return (i & 3) == 0 ? v.x : (i & 3) == 1 ? v.y : (i & 3) == 2 ? v.z : v.w;
-}
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t b) { return *reinterpret_cast<__half2 *>(&b); }
+
+__device__ __forceinline__ uint32_t word4(const uint4 &v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
 
 // 4 int8 codes (one word) times an fp16 scale -> 4 binary16 values (2 words).
 // A biased byte u = q + 128 placed under exponent byte 0x64 is the half
@@ -110,42 +98,40 @@ __device__ __forceinline__ void q8x4_to_h(uint32_t qw, __half2 d2, uint32_t &o0,
   o1 = h2_bits(__hmul2_rn(hi, d2));
 }
 
-// Q8_0: piece p (64 elements = blocks 2p, 2p+1) as 8 chunks of 8 halves.
-__device__ __forceinline__ void piece_q8_0(const RawUnit<DSQ_Q8_0> &u, int p, uint32_t (&out)[32]) {
+// Q8_0: one 64-element piece = two blocks = 68 bytes = 17 words starting
+// word-aligned (a piece starts at byte 68p of its 256-element unit).
+// word(i), i = 0..16, returns the piece's i-th word.  Block 0: fp16 d in the
+// low half of word 0, codes in bytes 2..33; block 1: d in the high half of
+// word 8, codes in words 9..16.  Output: 8 chunks of 8 halves.
+template <class Word>
+__device__ __forceinline__ void piece_q8_0(Word word, uint32_t (&out)[32]) {
+  {
+    const __half2 d2 = __half2half2(__ushort_as_half(static_cast<unsigned short>(word(0) & 0xffffu)));
 #pragma unroll
-  for (int half_ = 0; half_ < 2; ++half_) {
-    const int b = 2 * p + half_;
-    // block b starts at byte 34b; see gemv.cu for the word alignment rule
-    uint32_t qwd[8];
-    __half dh;
-    if ((b & 1) == 0) {
-      const int a = 17 * b / 2;
-      dh = __ushort_as_half(static_cast<unsigned short>(word_of(u, a) & 0xffffu));
+    for (int i = 0; i < 8; ++i)
+      q8x4_to_h(__funnelshift_r(word(i), word(i + 1), 16), d2, out[2 * i], out[2 * i + 1]);
+  }
+  {
+    const __half2 d2 = __half2half2(__ushort_as_half(static_cast<unsigned short>(word(8) >> 16)));
 #pragma unroll
-      for (int i = 0; i < 8; ++i) qwd[i] = __funnelshift_r(word_of(u, a + i), word_of(u, a + i + 1), 16);
-    } else {
-      const int a = (17 * b - 1) / 2;
-      dh = __ushort_as_half(static_cast<unsigned short>(word_of(u, a) >> 16));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qwd[i] = word_of(u, a + 1 + i);
-    }
-    const __half2 d2 = __half2half2(dh);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q8x4_to_h(qwd[i], d2, out[16 * half_ + 2 * i], out[16 * half_ + 2 * i + 1]);
+    for (int i = 0; i < 8; ++i) q8x4_to_h(word(9 + i), d2, out[16 + 2 * i], out[16 + 2 * i + 1]);
   }
 }
 
-// Q4_K: piece p (64 elements = sub-blocks 2p (low nibbles) and 2p+1 (high
-// nibbles) of bytes qs[32p .. 32p+31]).  Each value is fp32 (d*sc)*q - dmin*m
-// (one rounding: (d*sc)*q and dmin*m are exact), then binary16 RNE.
-__device__ __forceinline__ void piece_q4_k(const RawUnit<DSQ_Q4_K> &u, int p, uint32_t (&out)[32]) {
-  const uint32_t w0 = word_of(u, 0);
-  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(w0 & 0xffffu)));
-  const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(w0 >> 16)));
-  const uint32_t s0 = word_of(u, 1), s1 = word_of(u, 2), s2 = word_of(u, 3);
+// Q4_K: piece P (64 elements = sub-blocks 2P (low nibbles) and 2P+1 (high
+// nibbles) of bytes qs[32P .. 32P+31]).  hdr = the super-block's first 16
+// bytes (fp16 d, fp16 dmin, 12 bytes of packed 6-bit scales and mins);
+// nib(i), i = 0..7, returns word i of qs[32P ..].  Each value is fp32
+// (d*sc)*q - dmin*m (one rounding: (d*sc)*q and dmin*m are exact), then
+// binary16 RNE.
+template <int P, class Nib>
+__device__ __forceinline__ void piece_q4_k(const uint4 &hdr, Nib nib, uint32_t (&out)[32]) {
+  const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(hdr.x & 0xffffu)));
+  const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(hdr.x >> 16)));
+  const uint32_t s0 = hdr.y, s1 = hdr.z, s2 = hdr.w;
 #pragma unroll
   for (int half_ = 0; half_ < 2; ++half_) {
-    const int j = 2 * p + half_;
+    const int j = 2 * P + half_;
     uint32_t scw, mw;
     if (j < 4) {
       scw = s0 & 0x3f3f3f3fu;
@@ -159,13 +145,13 @@ __device__ __forceinline__ void piece_q4_k(const RawUnit<DSQ_Q4_K> &u, int p, ui
     const float nb = -__fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu));
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t byte4 = word_of(u, 4 + 8 * p + i);
-      const uint32_t nib = half_ ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
+      const uint32_t byte4 = nib(i);
+      const uint32_t q4 = half_ ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
       float v[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         // 0x4B000000 | q is the float 2^23 + q; subtracting 2^23 is exact
-        const float f = __uint_as_float(__byte_perm(nib, 0x4B000000u, 0x7540 + e));
+        const float f = __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7540 + e));
         v[e] = __fmaf_rn(__fsub_rn(f, 8388608.0f), a, nb);
       }
       out[16 * half_ + 2 * i] = h2_bits(__floats2half2_rn(v[0], v[1]));
@@ -174,116 +160,211 @@ __device__ __forceinline__ void piece_q4_k(const RawUnit<DSQ_Q4_K> &u, int p, ui
   }
 }
 
-template <int TYPE>
-__device__ __forceinline__ void dequant_piece(const RawUnit<TYPE> &u, int p, uint32_t (&out)[32]) {
-  if constexpr (TYPE == DSQ_Q8_0) piece_q8_0(u, p, out);
-  else piece_q4_k(u, p, out);
+// The registers a converter thread loads for piece P of a unit (uint4
+// granules of the row's 256-element unit), and the dequantization from them.
+// Q8_0: granules 4P .. 4P+4 (80 bytes covering the piece's 68, which start
+// at word P of them).  Q4_K: granule 0 (header) and 1+2P, 2+2P (the 32
+// nibble bytes).
+template <int TYPE> struct PieceRegs;
+template <> struct PieceRegs<DSQ_Q8_0> { uint4 v[5]; };
+template <> struct PieceRegs<DSQ_Q4_K> { uint4 hdr, v[2]; };
+
+template <int TYPE, int P>
+__device__ __forceinline__ void load_piece(PieceRegs<TYPE> &r, const uint4 *unit) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+#pragma unroll
+    for (int i = 0; i < 5; ++i) r.v[i] = unit[4 * P + i];
+  } else {
+    r.hdr = unit[0];
+    r.v[0] = unit[1 + 2 * P];
+    r.v[1] = unit[2 + 2 * P];
+  }
 }
 
+template <int TYPE, int P>
+__device__ __forceinline__ void dequant_piece(const PieceRegs<TYPE> &r, uint32_t (&out)[32]) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+    piece_q8_0([&](int i) { return word4(r.v[(P + i) >> 2], (P + i) & 3); }, out);
+  } else {
+    piece_q4_k<P>(r.hdr, [&](int i) { return word4(r.v[i >> 2], i & 3); }, out);
+  }
+}
 
 // ------------------------------------------------------------------ GEMM ---
-// TMEM map (512 columns x 128 lanes): [0, 2*tn) the fp32 accumulators of the
-// two halves (half h at h*tn); then stages_a dequantized-weight stages of
-// 64 columns each (half h at +32h), lane = row of the half, each column two
-// consecutive fp16 K elements.  The MMA reads A from TMEM and B (the
-// activation tile) from shared memory, so shared memory carries only the
-// activation stream.
+// TMEM map of each CTA (512 columns x 128 lanes): [0, tn) the fp32
+// accumulators (lane = weight row of this CTA, column = token of the pair
+// tile); then stages_a dequantized-weight stages of 32 columns each (lane =
+// weight row, each column two consecutive fp16 K elements).
 struct Smem {
-  uint8_t *b;          // groups_b x 4 x tn*128: activation tiles of one K unit each (MMA B)
-  uint64_t *bfull;     // activation unit landed (1 + tx)
-  uint64_t *bempty;    // MMA finished reading an activation unit (commit)
-  uint64_t *afull;     // converters stored a TMEM weight stage (count 8 warps)
-  uint64_t *aempty;    // MMA finished reading a TMEM weight stage (commit)
-  uint8_t *raw;        // raw_slots x 256 rows x unit bytes: raw weight units (TMA)
+  uint8_t *b;          // slots_b x stages_per_slot x (tn/2 rows x 128 B): activation stages (MMA B, this CTA's half)
+  uint8_t *raw;        // slots_raw x 128 rows x unit bytes: raw weight units (TMA)
+  uint64_t *bfull;     // activation slot landed (1 + tx)
+  uint64_t *bpeer;     // even CTA: the odd CTA's activation slot landed (1, forwarded)
+  uint64_t *bempty;    // pair MMAs finished reading an activation slot (multicast commit)
+  uint64_t *afull;     // even CTA: a TMEM weight stage is stored in both CTAs (8 warp arrivals)
+  uint64_t *aempty;    // pair MMAs finished reading a TMEM weight stage (multicast commit)
   uint64_t *rfull;     // raw unit landed (1 + tx)
-  uint64_t *rempty;    // converters copied a raw unit into registers (count 8 warps)
-  uint64_t *accfull;   // accumulators complete (commit)
-  uint64_t *accempty;  // epilogue drained the accumulators (count 4)
-  uint64_t *drain;     // MMA drain after an abort
+  uint64_t *rempty;    // converters copied a raw unit into registers (8 warps)
+  uint64_t *accfull;   // accumulators complete (multicast commit)
+  uint64_t *accempty;  // even CTA: both epilogues drained the accumulators (8 warp arrivals)
+  uint64_t *drain;     // even CTA: MMA drain after an abort
   uint32_t *tmem;      // TMEM base address
-  volatile int *abort;
+  volatile uint32_t *abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int groups_b, int stages_a, int tn, int raw_slots, int raw_bytes) {
+__device__ __forceinline__ Smem carve(uint8_t *base, int slots_b, uint32_t slot_b_bytes, int slots_raw,
+                                      uint32_t raw_bytes, int stages_a) {
   Smem s;
   s.b = base;
-  s.raw = s.b + static_cast<size_t>(groups_b) * 4 * tn * 128;
-  uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(raw_slots) * raw_bytes);
+  s.raw = s.b + static_cast<size_t>(slots_b) * slot_b_bytes;
+  uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(slots_raw) * raw_bytes);
   s.bfull = p;
-  s.bempty = s.bfull + groups_b;
-  s.afull = s.bempty + groups_b;
+  s.bpeer = s.bfull + slots_b;
+  s.bempty = s.bpeer + slots_b;
+  s.afull = s.bempty + slots_b;
   s.aempty = s.afull + stages_a;
   s.rfull = s.aempty + stages_a;
-  s.rempty = s.rfull + raw_slots;
-  s.accfull = s.rempty + raw_slots;
+  s.rempty = s.rfull + slots_raw;
+  s.accfull = s.rempty + slots_raw;
   s.accempty = s.accfull + 1;
   s.drain = s.accempty + 1;
   s.tmem = reinterpret_cast<uint32_t *>(s.drain + 1);
-  s.abort = reinterpret_cast<volatile int *>(s.tmem + 1);
+  s.abort = reinterpret_cast<volatile uint32_t *>(s.tmem + 1);
   return s;
+}
+__host__ __device__ constexpr size_t barrier_bytes(int slots_b, int slots_raw, int stages_a) {
+  return (3 * static_cast<size_t>(slots_b) + 2 * stages_a + 2 * slots_raw + 3) * sizeof(uint64_t) + 16;
 }
 
 __device__ __forceinline__ bool aborted(const Smem &s) { return *s.abort != 0; }
+// Raise the abort flag of both CTAs of the pair.
 __device__ __forceinline__ void set_abort(const Smem &s, const WaitCtl &w) {
-  *s.abort = 1;
+  *s.abort = 1u;
+  st_shared_remote_u32(mapa_shared(smem_u32(const_cast<uint32_t *>(s.abort)), cluster_ctarank() ^ 1u), 1u);
   record_timeout(w);
 }
 
 // One thread's bounded wait; on expiry (or an abort raised elsewhere) it
-// raises the CTA abort flag and returns false.  sleep_ns: poll back-off for
-// waiters off the critical path.
+// raises the pair's abort flag and returns false.
+// sleep_ns: poll back-off for waiters off the critical path.
 __device__ __forceinline__ bool wait_or_abort(const Smem &s, uint64_t *bar, uint32_t parity, const WaitCtl &w,
                                               uint32_t sleep_ns = 0) {
+  if (mbar_try_wait(bar, parity)) return true;   // fast path: already complete
   if (aborted(s)) return false;
   if (mbar_wait_for(bar, parity, w.limit_ns, sleep_ns)) return true;
   set_abort(s, w);
   return false;
 }
 
-// Tile t -> (first token, first weight row, K split); consecutive tiles
-// share a weight tile, so CTAs running side by side reuse it from L2.
+// Pair tile t -> (token tile, first weight row, K split); consecutive tiles
+// share a weight tile, so pairs running side by side reuse it from L2.  The
+// tile walks its K units [u0, u1) cyclically from u0 + rot: pairs that run
+// at the same time on the same activation tile (other weight rows) or the
+// same weight tile (other tokens) then read different units instead of the
+// same lines at the same moment.
 struct Tile {
-  int64_t m0, n0;
-  int u0, u1;
+  int64_t mt, n0;
+  int u0, u1, rot;
   int split;
 };
 __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   Tile tl;
-  const int64_t m = t % a.tiles_m;
+  tl.mt = t % a.tiles_m;
   const int64_t rest = t / a.tiles_m;
   tl.split = static_cast<int>(rest % a.splits);
-  tl.m0 = m * a.tn;
   tl.n0 = (rest / a.splits) * kTileN;
   tl.u0 = tl.split * a.units_per_split;
   tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
+  tl.rot = static_cast<int>((rest / a.splits + 7 * tl.mt) % (tl.u1 - tl.u0));
   return tl;
 }
 
-// Persistent CTA over tiles of 256 weight rows x tn tokens x one K split:
-// tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Each 64-K stage holds the
-// activation tile once (shared memory) and the two 128-row weight halves
-// (TMEM); the MMA warp issues both halves against the same activation tile.
+// Converter warp of stage parity J (J = 0: stages 0 and 2 of every unit,
+// J = 1: stages 1 and 3): thread = weight row rr of this CTA.  Per unit it
+// copies the granules of its two pieces out of the raw slot, releases the
+// slot, and for each piece waits for a free TMEM stage, dequantizes 64
+// elements and stores them into its lane with one tcgen05.st; one lane per
+// warp then arrives on the even CTA's afull.
+template <int TYPE, int J>
+__device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a, uint32_t tmem_stage0, int rr,
+                                             uint32_t afull_even) {
+  constexpr uint32_t RAW_BYTES = kRows * unit_bytes<TYPE>();
+  const int lane = threadIdx.x & 31;
+  const int SA = a.stages_a, SR = a.slots_raw;
+  const int64_t npairs = gridDim.x / 2;
+  int sa = J;            // TMEM stage slot of this warp's next stage (this warp takes every other one)
+  uint32_t rnd = 0;      // its ring round; round r >= 1 waits for the MMA release of round r - 1
+  int rs = 0;            // raw unit slot and its phase parity
+  uint32_t rpar = 0;
+  for (int64_t t = blockIdx.x / 2; t < a.total_tiles; t += npairs) {
+    const Tile tl = tile_of(a, t);
+    for (int u = tl.u0; u < tl.u1; ++u) {
+      const bool got = wait_or_abort(s, &s.rfull[rs], rpar, a.wait);
+      if (__any_sync(0xffffffffu, !got)) return;
+      const uint4 *unit = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES +
+                                                          static_cast<size_t>(rr) * unit_bytes<TYPE>());
+      PieceRegs<TYPE> r0, r1;
+      load_piece<TYPE, J>(r0, unit);
+      load_piece<TYPE, J + 2>(r1, unit);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.rempty[rs]);
+      if (++rs == SR) {
+        rs = 0;
+        rpar ^= 1u;
+      }
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        if (rnd > 0) {
+          const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
+          if (__any_sync(0xffffffffu, !free_)) return;
+        }
+        uint32_t v[32];
+        if (pp == 0) dequant_piece<TYPE, J>(r0, v);
+        else dequant_piece<TYPE, J + 2>(r1, v);
+        tc_fence_after_sync();
+        tmem_st_32cols(tmem_stage0 + static_cast<uint32_t>(sa * kAColsStage), v);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(afull_even + static_cast<uint32_t>(sa) * 8u);
+        sa += 2;
+        if (sa >= SA) {
+          sa -= SA;
+          ++rnd;
+        }
+      }
+    }
+  }
+}
+
+// Persistent CTA pair over pair tiles (pair index blockIdx.x / 2, stepping
+// by the number of pairs); rank r = this CTA's rank in the cluster.
 template <int TYPE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ PrefillArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
-  constexpr int RAW_BYTES = kTileN * UB;   // one unit of the tile's 256 rows
+  constexpr uint32_t RAW_BYTES = kRows * UB;   // one unit of this CTA's 128 rows
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Smem s = carve(base, a.groups_b, a.stages_a, a.tn, a.raw_slots, RAW_BYTES);
+  const int tnc = a.tn / 2;                                        // tokens of this CTA
+  const uint32_t stage_b_bytes = static_cast<uint32_t>(tnc) * 128u;   // one 64-K activation stage
+  const int S2 = a.stages_per_slot;
+  const uint32_t slot_b_bytes = stage_b_bytes * static_cast<uint32_t>(S2);   // one activation copy
+  const Smem s = carve(base, a.slots_b, slot_b_bytes, a.slots_raw, RAW_BYTES, a.stages_a);
+  const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int SB = a.groups_b, SA = a.stages_a, SR = a.raw_slots;
-  const uint32_t stage_b_bytes = static_cast<uint32_t>(a.tn) * 128u;   // one 64-K activation tile
-  const uint32_t group_b_bytes = 4u * stage_b_bytes;                    // one 256-K unit
+  const int SB = a.slots_b, SA = a.stages_a, SR = a.slots_raw;
+  const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
   const int units = static_cast<int>(a.K / 256);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SB; ++i) {
       mbar_init(&s.bfull[i], 1);
+      mbar_init(&s.bpeer[i], 1);
       mbar_init(&s.bempty[i], 1);
     }
     for (int i = 0; i < SA; ++i) {
-      mbar_init(&s.afull[i], kConvWarps);
+      mbar_init(&s.afull[i], 2 * 4);   // 4 converter warps per stage in each CTA
       mbar_init(&s.aempty[i], 1);
     }
     for (int i = 0; i < SR; ++i) {
@@ -291,122 +372,144 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.rempty[i], kConvWarps);
     }
     mbar_init(s.accfull, 1);
-    mbar_init(s.accempty, 4);
+    mbar_init(s.accempty, 2 * 4);      // 4 epilogue warps in each CTA
     mbar_init(s.drain, 1);
-    *s.abort = 0;
+    *s.abort = 0u;
     fence_barrier_init();
     prefetch_tensormap(&tmap_w);
   }
-  const int conv = (warp >= kWarpConv0 && warp < kWarpEpi0) ? warp - kWarpConv0 : -1;
-  // converter warp c: half c / 4, TMEM lane quadrant warp % 4 (a warp may only
-  // touch its own quadrant), so its row within the half is 32 * (warp % 4) + lane
-  const int conv_half = conv / 4, conv_rr = 32 * (warp & 3) + lane;
-  if (warp == kWarpW && lane == 0 && blockIdx.x < a.total_tiles) {
-    // weights are read-only: start the first units toward L2 while the
-    // activation-rounding kernel before us finishes
-    const Tile tl = tile_of(a, blockIdx.x);
-    for (int u = tl.u0; u < tl.u1 && u < tl.u0 + 2; ++u)
-      for (int h = 0; h < kHalves; ++h)
-        prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0 + h * kBM));
+  if (warp == kWarpW && lane == 0 && pair < a.total_tiles) {
+    // weights are read-only: start this CTA's first units toward L2 while
+    // the activation-rounding kernel before us finishes
+    const Tile tl = tile_of(a, pair);
+    for (int k = 0; k < 2 && k < tl.u1 - tl.u0; ++k) {
+      const int u = tl.u0 + (tl.rot + k) % (tl.u1 - tl.u0);
+      prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0 + kRows * rank));
+    }
   }
   if (warp == kWarpMma) {
-    tmem_alloc(s.tmem, static_cast<uint32_t>(kTmemCols));
-    tmem_relinquish();
+    tmem_alloc_pair(s.tmem, static_cast<uint32_t>(kTmemCols));
+    tmem_relinquish_pair();
   }
+  __syncwarp();
   tc_fence_before_sync();
-  __syncthreads();
+  cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after_sync();
   pdl_trigger();
   pdl_wait();
   const uint32_t tmem_base = *s.tmem;
-  const uint32_t a_col0 = static_cast<uint32_t>(kHalves * a.tn);   // first weight-stage column
+  const uint32_t a_col0 = static_cast<uint32_t>(a.tn);   // first weight-stage column
 
   if (warp == kWarpX) {
     // ---------------------------------------- activation stages (bulk copy)
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();   // every weight tile re-reads these
-      // One bulk copy per 256-element K unit: the activation tile of the
-      // unit is contiguous in the tile-major layout.  Ring position kept
-      // incrementally (no integer division on this path): slot sb of round
-      // rnd; round r >= 1 first waits for the MMA's release from round r - 1.
+      // One copy per slot: stages_per_slot consecutive stages of one K
+      // unit, contiguous in the tile-major layout (the copy engine's cost is
+      // mostly per copy, so copies are made as large as shared memory
+      // allows).  Ring position kept incrementally; round r >= 1 first
+      // waits for the MMA release of round r - 1.
       int64_t gs = 0;
       int sb = 0;
       uint32_t rnd = 0;
-      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
+      bool ok = true;
+      for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
         const Tile tl = tile_of(a, t);
-        const int64_t mt = tl.m0 / a.tn;
-        for (int u = tl.u0; u < tl.u1; ++u, ++gs) {
-          if (rnd > 0 && !wait_or_abort(s, &s.bempty[sb], (rnd - 1) & 1u, a.wait, 64)) break;
-          mbar_arrive_expect_tx(&s.bfull[sb], group_b_bytes);
-          bulk_g2s(s.b + static_cast<size_t>(sb) * group_b_bytes,
-                   reinterpret_cast<const uint8_t *>(a.x16) + (mt * units + u) * static_cast<int64_t>(group_b_bytes),
-                   group_b_bytes, &s.bfull[sb], keep);
-          if (++sb == SB) {
-            sb = 0;
-            ++rnd;
+        const int64_t xt = 2 * tl.mt + rank;   // this CTA's token tile
+        int u = tl.u0 + tl.rot;
+        for (int k = tl.u0; k < tl.u1 && ok; ++k, u = (u + 1 == tl.u1 ? tl.u0 : u + 1)) {
+          for (int kb4 = 0; kb4 < 4; kb4 += S2, ++gs) {
+            if (rnd > 0 && !wait_or_abort(s, &s.bempty[sb], (rnd - 1) & 1u, a.wait, 64)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&s.bfull[sb], slot_b_bytes);
+            bulk_g2s(s.b + static_cast<size_t>(sb) * slot_b_bytes,
+                     reinterpret_cast<const uint8_t *>(a.x16) +
+                         ((xt * units + u) * 4 + kb4) * static_cast<int64_t>(stage_b_bytes),
+                     slot_b_bytes, &s.bfull[sb], keep);
+            if (++sb == SB) {
+              sb = 0;
+              ++rnd;
+            }
           }
         }
       }
-      if (aborted(s))
+      if (!ok)
         for (int64_t g = (gs > SB ? gs - SB : 0); g < gs; ++g)
           mbar_wait_for(&s.bfull[g % SB], static_cast<uint32_t>((g / SB) & 1), kDrainLimitNs);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------ MMA issuer
+  } else if (warp == kWarpMma && rank == 1) {
+    // ------------------------------- odd CTA: forward activation arrivals
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f16(kBM, static_cast<uint32_t>(a.tn), 0);
+      const uint32_t bpeer_even = mapa_shared(smem_u32(s.bpeer), 0);
+      int sb = 0;
+      uint32_t par = 0;
+      bool ok = true;
+      for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
+        const Tile tl = tile_of(a, t);
+        for (int g = 0; g < (4 / S2) * (tl.u1 - tl.u0); ++g) {
+          if (!wait_or_abort(s, &s.bfull[sb], par, a.wait)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_remote(bpeer_even + static_cast<uint32_t>(sb) * 8u);
+          if (++sb == SB) {
+            sb = 0;
+            par ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------- even CTA: MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(kTileN, static_cast<uint32_t>(a.tn), 0);
       const uint32_t b_base = smem_u32(s.b);
       int64_t i = 0;
-      int sb = 0, sa = 0;
-      uint32_t pb = 0, pa = 0;   // phase parity of the current round of each ring
+      int sb = 0, sa = 0, gin = 0;   // gin: stage within the activation slot
+      uint32_t pb = 0, pa = 0;       // phase parity of the current round of each ring
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x, ++i) {
+      for (int64_t t = pair; t < a.total_tiles && ok; t += npairs, ++i) {
         const Tile tl = tile_of(a, t);
         if (i >= 1 && !wait_or_abort(s, s.accempty, static_cast<uint32_t>((i - 1) & 1), a.wait)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        for (int u = tl.u0; u < tl.u1 && ok; ++u) {
-          if (!wait_or_abort(s, &s.bfull[sb], pb, a.wait)) {
+        for (int g = 0; g < 4 * (tl.u1 - tl.u0); ++g) {
+          if ((gin == 0 && (!wait_or_abort(s, &s.bfull[sb], pb, a.wait) ||
+                            !wait_or_abort(s, &s.bpeer[sb], pb, a.wait))) ||
+              !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
             ok = false;
             break;
           }
-          for (int kb4 = 0; kb4 < 4; ++kb4) {
-            if (!wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after_sync();
-            const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * group_b_bytes + static_cast<uint32_t>(kb4) * stage_b_bytes;
-            const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
-            const bool first = (u == tl.u0 && kb4 == 0);
+          tc_fence_after_sync();
+          const uint32_t b_addr =
+              b_base + static_cast<uint32_t>(sb) * slot_b_bytes + static_cast<uint32_t>(gin) * stage_b_bytes;
+          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t bdesc = umma_desc_sw128(b_addr + 32 * k);
-#pragma unroll
-              for (int h = 0; h < kHalves; ++h)
-                umma_f16_ts(tmem_base + static_cast<uint32_t>(h * a.tn),
-                            a_tmem + static_cast<uint32_t>(h * kAColsHalf + 8 * k), bdesc, idesc,
-                            (!first || k > 0) ? 1u : 0u);
-            }
-            umma_commit(&s.aempty[sa]);
-            if (++sa == SA) {
-              sa = 0;
-              pa ^= 1u;
-            }
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_f16_ts_pair(tmem_base, a_tmem + static_cast<uint32_t>(8 * k), umma_desc_sw128(b_addr + 32 * k),
+                             idesc, (g > 0 || k > 0) ? 1u : 0u);
+          umma_commit_pair_mc(&s.aempty[sa], 0x3);
+          if (++sa == SA) {
+            sa = 0;
+            pa ^= 1u;
           }
-          if (!ok) break;
-          umma_commit(&s.bempty[sb]);
-          if (++sb == SB) {
-            sb = 0;
-            pb ^= 1u;
+          if (++gin == S2) {
+            gin = 0;
+            umma_commit_pair_mc(&s.bempty[sb], 0x3);
+            if (++sb == SB) {
+              sb = 0;
+              pb ^= 1u;
+            }
           }
         }
-        if (ok) umma_commit(s.accfull);
+        if (ok) umma_commit_pair_mc(s.accfull, 0x3);
       }
       if (!ok) {
-        umma_commit(s.drain);
+        umma_commit_pair(s.drain);
         mbar_wait_for(s.drain, 0, kDrainLimitNs);
       }
     }
@@ -416,122 +519,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t gu = 0;
       int rs = 0;
       uint32_t rnd = 0;
-      for (int64_t t = blockIdx.x; t < a.total_tiles && !aborted(s); t += gridDim.x) {
+      bool ok = true;
+      for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
         const Tile tl = tile_of(a, t);
-        for (int u = tl.u0; u < tl.u1; ++u, ++gu) {
-          if (rnd > 0 && !wait_or_abort(s, &s.rempty[rs], (rnd - 1) & 1u, a.wait, 64)) break;
-          mbar_arrive_expect_tx(&s.rfull[rs], static_cast<uint32_t>(RAW_BYTES));
-          for (int h = 0; h < kHalves; ++h)
-            tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES + static_cast<size_t>(h) * kBM * UB, &tmap_w,
-                        u * (UB / 4), static_cast<int32_t>(tl.n0 + h * kBM), &s.rfull[rs]);
+        const int32_t row0 = static_cast<int32_t>(tl.n0 + kRows * rank);
+        int u = tl.u0 + tl.rot;
+        for (int k = tl.u0; k < tl.u1; ++k, ++gu, u = (u + 1 == tl.u1 ? tl.u0 : u + 1)) {
+          if (rnd > 0 && !wait_or_abort(s, &s.rempty[rs], (rnd - 1) & 1u, a.wait, 64)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&s.rfull[rs], RAW_BYTES);
+          tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &tmap_w, u * (UB / 4), row0, &s.rfull[rs]);
           if (++rs == SR) {
             rs = 0;
             ++rnd;
           }
         }
       }
-      if (aborted(s))
+      if (!ok)
         for (int64_t g = (gu > SR ? gu - SR : 0); g < gu; ++g)
           mbar_wait_for(&s.rfull[g % SR], static_cast<uint32_t>((g / SR) & 1), kDrainLimitNs);
     }
-  } else if (conv >= 0) {
+  } else if (warp < kWarpEpi0) {
     // ------------------------------------------ converters (dequantize)
-    // Thread (half h, row rr) owns weight row 128h + rr of the tile.  It
-    // reads the row's raw 256-element units from global memory (the next
-    // unit is prefetched into L2 while this one is converted) and writes 64
-    // dequantized fp16 per stage into its TMEM lane with one store.
-    const int h = conv_half, rr = conv_rr;
-    const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    int sa = 0;
-    uint32_t rnd = 0;   // ring round; round r >= 1 waits for the release from round r - 1
-    int rs = 0;         // raw unit slot and its phase parity
-    uint32_t rpar = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < a.total_tiles && ok; t += gridDim.x) {
-      const Tile tl = tile_of(a, t);
-      for (int u = tl.u0; u < tl.u1 && ok; ++u) {
-        const bool got = wait_or_abort(s, &s.rfull[rs], rpar, a.wait);
-        if (__any_sync(0xffffffffu, !got)) {
-          ok = false;
-          break;
-        }
-        RawUnit<TYPE> ru;
-        const uint4 *src = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES +
-                                                           static_cast<size_t>(h * kBM + rr) * UB);
-#pragma unroll
-        for (int v = 0; v < RawUnit<TYPE>::kVecs; ++v) ru.v[v] = src[v];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.rempty[rs]);
-        if (++rs == SR) {
-          rs = 0;
-          rpar ^= 1u;
-        }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          if (rnd > 0) {
-            const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
-            if (__any_sync(0xffffffffu, !free_)) {
-              ok = false;
-              break;
-            }
-          }
-          uint32_t v[32];
-          dequant_piece<TYPE>(ru, p, v);   // rows past N arrive as zero blocks: zeros
-          tc_fence_after_sync();
-          tmem_st_32cols(tmem_base + lane_addr + a_col0 + static_cast<uint32_t>(sa * kAColsStage + h * kAColsHalf), v);
-          tmem_st_wait();
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s.afull[sa]);
-          if (++sa == SA) {
-            sa = 0;
-            ++rnd;
-          }
-        }
-      }
-    }
-  } else if (warp >= kWarpEpi0) {
+    const int q = warp & 3;   // TMEM lane quadrant this warp may access
+    const uint32_t stage0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a_col0;
+    const uint32_t afull_even = mapa_shared(smem_u32(s.afull), 0);
+    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, stage0, 32 * q + lane, afull_even);
+    else convert_role<TYPE, 1>(s, a, stage0, 32 * q + lane, afull_even);
+  } else {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
-    const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = 32 * q + lane;            // row within each 128-row half
+    const int q = warp & 3;
+    const int64_t r = kRows * rank + 32 * q + lane;   // weight row within the pair tile
+    const uint32_t accempty_even = mapa_shared(smem_u32(s.accempty), 0);
+    const int nchunks = a.tn / 32;
     int64_t i = 0;
-    for (int64_t t = blockIdx.x; t < a.total_tiles; t += gridDim.x, ++i) {
+    for (int64_t t = pair; t < a.total_tiles; t += npairs, ++i) {
       const Tile tl = tile_of(a, t);
+      const int64_t n = tl.n0 + r;
+      const bool n_ok = n < a.N;
+      const int64_t m0 = tl.mt * a.tn;
+      // before the wait: lane j holds 2^-s of token m0 + 32c + j for every
+      // chunk c (0 for padding tokens), so the drain below has no loads
+      float my_scale[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int64_t m = m0 + 32 * c + lane;
+        const int sft = (c < nchunks && m < a.M) ? __ldg(a.shift + m) : 0;
+        my_scale[c] = __int_as_float((127 - sft) << 23);   // s in [-64, 64]
+      }
       const bool got = wait_or_abort(s, s.accfull, static_cast<uint32_t>(i & 1), a.wait, 256);
       if (__any_sync(0xffffffffu, !got)) break;
       tc_fence_after_sync();
-      float *y = a.y + static_cast<int64_t>(tl.split) * a.M * a.N;
-      for (int hh = 0; hh < kHalves; ++hh) {
-        const int64_t n = tl.n0 + hh * kBM + r;
-        for (int c = 0; c < a.tn / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(hh * a.tn + 32 * c),
-                         v);
-          tmem_ld_wait();
-          if (hh == kHalves - 1 && c == a.tn / 32 - 1) {
-            // every accumulator column is in registers: let the next tile start
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s.accempty);
-          }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t m = tl.m0 + 32 * c + j;
-            if (m < a.M && n < a.N) {
-              const int sft = __ldg(a.shift + m);
-              const float scale = __int_as_float((127 - sft) << 23);   // 2^-s, s in [-64, 64]
-              y[m * a.N + n] = __fmul_rn(__uint_as_float(v[j]), scale);
-            }
-          }
+      for (int c = 0; c < 8; ++c) {
+        if (c >= nchunks) break;
+        uint32_t v[32];
+        tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), v);
+        tmem_ld_wait();
+        if (c == nchunks - 1) {
+          // every accumulator column is in registers: let the next tile start
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(accempty_even);
+        }
+        // scale branch-free (the shuffles pipeline), then store
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xffffffffu, my_scale[c], j)));
+        const int64_t mc = m0 + 32 * c;
+        float *yp = a.y + (static_cast<int64_t>(tl.split) * a.M + mc) * a.N + n;
+        if (n_ok && mc + 32 <= a.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) yp[static_cast<int64_t>(j) * a.N] = __uint_as_float(v[j]);
+        } else if (n_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (mc + j < a.M) yp[static_cast<int64_t>(j) * a.N] = __uint_as_float(v[j]);
         }
       }
     }
   }
+  __syncwarp();
   tc_fence_before_sync();
-  __syncthreads();
+  cluster_sync();   // no CTA leaves while its pair may still touch its memory
   if (warp == kWarpMma) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, static_cast<uint32_t>(kTmemCols));
+    tmem_dealloc_pair(tmem_base, static_cast<uint32_t>(kTmemCols));
   }
 }
 
@@ -627,7 +702,19 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
 }
 
 // Test hook: the whole dequantized weight matrix in binary16, produced by the
-// same device functions as the GEMM's converter warps.
+// same device functions as the GEMM's converter warps (one thread per
+// 256-element unit of a row).
+template <int TYPE, int P>
+__device__ __forceinline__ void unit_piece_to_f16(const uint4 *unit, uint16_t *dst) {
+  PieceRegs<TYPE> r;
+  load_piece<TYPE, P>(r, unit);
+  uint32_t v[32];
+  dequant_piece<TYPE, P>(r, v);
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst + P * 64);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) d4[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
 template <int TYPE>
 __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict__ w, int64_t N, int64_t K,
                                                        int64_t row_bytes, uint16_t *__restrict__ w16) {
@@ -635,23 +722,19 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= N * units) return;
   const int64_t n = idx / units, u = idx % units;
-  RawUnit<TYPE> ru;
-  load_unit<TYPE>(ru, w + n * row_bytes + u * (TYPE == DSQ_Q8_0 ? 272 : 144));
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    uint32_t v[32];
-    dequant_piece<TYPE>(ru, p, v);
-    uint4 *dst = reinterpret_cast<uint4 *>(w16 + n * K + u * 256 + p * 64);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-  }
+  const uint4 *unit = reinterpret_cast<const uint4 *>(w + n * row_bytes + u * unit_bytes<TYPE>());
+  uint16_t *dst = w16 + n * K + u * 256;
+  unit_piece_to_f16<TYPE, 0>(unit, dst);
+  unit_piece_to_f16<TYPE, 1>(unit, dst);
+  unit_piece_to_f16<TYPE, 2>(unit, dst);
+  unit_piece_to_f16<TYPE, 3>(unit, dst);
 }
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, groups_b, stages_a, raw_slots, splits, units_per_split;
+  int tn, slots_b, stages_per_slot, slots_raw, stages_a, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
-  unsigned grid;
+  unsigned grid;   // CTAs (2 per pair)
   size_t smem, x16_bytes, shift_off, part_off, total;
 };
 
@@ -659,38 +742,106 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int num_sms) {
+template <int TYPE>
+cudaError_t launch_pair(const CUtensorMap &map_w, const PrefillArgs &args, unsigned grid, size_t smem,
+                        cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<TYPE>, map_w, args);
+}
+
+// How many CTA pairs of the GEMM kernel can be resident at once (clusters
+// of 2 need two SMs of one GPC); cached per device, type and smem size.
+int resident_pairs(int type, size_t smem, int sms) {
+  static std::mutex mu;
+  static int cache[64][2][4] = {};
+  static size_t cache_smem[64][2][4] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
+  const int ti = type == DSQ_Q8_0 ? 0 : 1;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < 4; ++i)
+    if (cache[dev][ti][i] > 0 && cache_smem[dev][ti][i] == smem) return cache[dev][ti][i];
+  const void *kern = type == DSQ_Q8_0 ? reinterpret_cast<const void *>(prefill_kernel<DSQ_Q8_0>)
+                                      : reinterpret_cast<const void *>(prefill_kernel<DSQ_Q4_K>);
+  if (set_smem_once(kern, static_cast<int>(smem), "prefill") != DSQ_OK) return sms / 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = sms / 2;
+  }
+  if (n > sms / 2) n = sms / 2;
+  for (int i = 0; i < 4; ++i)
+    if (cache[dev][ti][i] == 0) {
+      cache[dev][ti][i] = n;
+      cache_smem[dev][ti][i] = smem;
+      break;
+    }
+  return n;
+}
+
+// pairs < 0: ask the device (needs a current device), else use that count
+Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   Plan p{};
-  const int64_t tiles_n = (N + kTileN - 1) / kTileN;
-  // tokens per tile: the smallest multiple of 32 that covers M, at most 128
-  // (TMEM holds 2 x tn accumulator columns plus the weight stages, so tn <= 128)
-  p.tn = M <= 128 ? static_cast<int>((M + 31) / 32 * 32) : 128;
+  // tokens per pair tile: the smallest multiple of 32 that covers M, at most
+  // 256 (the MMA's N; each CTA holds tn/2 of them)
+  p.tn = M <= 256 ? static_cast<int>((M + 31) / 32 * 32) : 256;
   p.tiles_m = (M + p.tn - 1) / p.tn;
-  p.tiles_n = tiles_n;
+  p.tiles_n = (N + kTileN - 1) / kTileN;
   const int units = static_cast<int>(K / 256);
+  // TMEM: tn accumulator columns, then up to 8 (an even number of) 32-column
+  // weight stages
+  p.stages_a = (kTmemCols - p.tn) / kAColsStage;
+  if (p.stages_a > kMaxStagesA) p.stages_a = kMaxStagesA;
+  p.stages_a &= ~1;
+  // shared memory.  The SM's copy engine costs a few hundred cycles per
+  // copy whatever its size, so activation copies take up to 32 KB (2 or 4
+  // stages of one K unit); up to 4 (at most 8) activation slots next to 2
+  // raw weight units, then the rest to more raw units (at most 4).
+  const size_t stage_b = static_cast<size_t>(p.tn / 2) * 128;
+  p.stages_per_slot = 1;
+  while (p.stages_per_slot < 4 && p.stages_per_slot * stage_b < 32 * 1024) p.stages_per_slot *= 2;
+  const size_t slot_b = p.stages_per_slot * stage_b;
+  const size_t raw_bytes = static_cast<size_t>(kRows) * (type == DSQ_Q8_0 ? 272 : 144);
+  const size_t fixed = 1024 + barrier_bytes(8, 4, p.stages_a);
+  p.slots_b = static_cast<int>((kSmemLimit - fixed - 2 * raw_bytes) / slot_b);
+  if (p.slots_b > 8) p.slots_b = 8;
+  if (p.slots_b > 4 && slot_b >= 16 * 1024) p.slots_b = 4;
+  p.slots_raw = static_cast<int>((kSmemLimit - fixed - p.slots_b * slot_b) / raw_bytes);
+  if (p.slots_raw > 4) p.slots_raw = 4;
+  p.smem = 1024 + p.slots_b * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots_b, p.slots_raw, p.stages_a);
+  if (pairs < 0) pairs = resident_pairs(type, p.smem, sms);
   const int64_t tiles = p.tiles_m * p.tiles_n;
-  // split K only when the tiles leave more than half the SMs idle
+  // split K only when the tiles leave more than half the pairs idle
   p.splits = 1;
-  while (tiles * p.splits * 2 <= num_sms && p.splits * 2 <= 16 && p.splits * 2 <= units) p.splits *= 2;
+  while (tiles * p.splits * 2 <= pairs && p.splits * 2 <= 16 && p.splits * 2 <= units) p.splits *= 2;
   p.units_per_split = (units + p.splits - 1) / p.splits;
   p.splits = (units + p.units_per_split - 1) / p.units_per_split;
   p.total_tiles = tiles * p.splits;
-  p.grid = static_cast<unsigned>(p.total_tiles < num_sms ? p.total_tiles : num_sms);
-  // TMEM: the accumulators (2 halves x tn fp32 columns), then as many
-  // 64-column weight stages as fit (at most 6)
-  p.stages_a = (kTmemCols - kHalves * p.tn) / kAColsStage;
-  if (p.stages_a > 6) p.stages_a = 6;
-  // shared memory: raw weight slots (one 256-element unit of the tile's 256
-  // rows each; two when they fit, else one) and activation slots (one unit
-  // of K each; two or more)
-  const int group_bytes = 4 * p.tn * 128;
-  const int raw_bytes = kTileN * (type == DSQ_Q8_0 ? 272 : 144);
-  const size_t fixed = 1024 + 512;
-  p.raw_slots = (fixed + 2 * static_cast<size_t>(raw_bytes) + 2 * group_bytes <= kSmemLimit) ? 2 : 1;
-  p.groups_b = static_cast<int>((kSmemLimit - fixed - static_cast<size_t>(p.raw_slots) * raw_bytes) / group_bytes);
-  if (p.groups_b > 6) p.groups_b = 6;
-  p.smem = 1024 + static_cast<size_t>(p.groups_b) * group_bytes + static_cast<size_t>(p.raw_slots) * raw_bytes +
-           (2 * p.groups_b + 2 * p.stages_a + 2 * p.raw_slots + 3) * sizeof(uint64_t) + 16;
+  p.grid = static_cast<unsigned>(2 * (p.total_tiles < pairs ? p.total_tiles : pairs));
   // the fp16 activation buffer is padded with zero rows to whole token tiles
   p.m_pad = p.tiles_m * p.tn;
   p.x16_bytes = align_up(static_cast<size_t>(p.m_pad) * K * 2, 1024);
@@ -726,13 +877,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int TYPE>
 int launch_gemm(const CUtensorMap &map_w, const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
-  auto kern = prefill_kernel<TYPE>;
-  const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(p.smem), "prefill");
+  const void *kern = reinterpret_cast<const void *>(prefill_kernel<TYPE>);
+  const int rc = set_smem_once(kern, static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  // ask for no more shared-memory carveout than the kernel uses: the rest is L1
-  const int carve = static_cast<int>((p.smem * 100 + 228 * 1024 - 1) / (228 * 1024));
-  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, carve);
-  const cudaError_t e = launch_pdl(kern, dim3(p.grid), dim3(kThreads), p.smem, stream, map_w, args);
+  const cudaError_t e = launch_pair<TYPE>(map_w, args, p.grid, p.smem, stream);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
@@ -745,7 +893,7 @@ extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, in
   if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
-  return make_plan(type, N, K, M, sms).total;
+  return make_plan(type, N, K, M, sms, -1).total;
 }
 
 extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
@@ -759,11 +907,11 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   int sms = 0;
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
-  const Plan p = make_plan(type, N, K, M, sms);
+  const Plan p = make_plan(type, N, K, M, sms, -1);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.groups_b >= 2 && p.stages_a >= 2 && p.raw_slots >= 1, DSQ_ERR_SHAPE,
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots_b >= 2 && p.stages_a >= 2 && p.slots_raw >= 2, DSQ_ERR_SHAPE,
               "dsq_gemm_prefill: no pipeline fits");
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -773,7 +921,8 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
 
   // raw weight units: the packed rows viewed as uint32 [N][row_bytes/4], one
   // 256-element unit (68 or 36 words) x 128 rows per box; rows past N read as
-  // zero (a zero block dequantizes to zero)
+  // zero (a zero block dequantizes to zero).  The kernel reads the weights
+  // only through this map.
   auto enc = encode_fn();
   DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
   CUtensorMap map_w;
@@ -782,7 +931,7 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
     const cuuint32_t unit_words = type == DSQ_Q8_0 ? 68u : 36u;
     const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
     const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
-    const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kBM)};
+    const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estride[2] = {1u, 1u};
     const CUresult cr = enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box,
                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -791,14 +940,12 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   }
   cudaStream_t st = as_stream(stream);
   cudaError_t e = launch_pdl(x_to_f16_kernel<true>, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K,
-                             static_cast<int64_t>(p.tn), x16, shift);
+                             static_cast<int64_t>(p.tn / 2), x16, shift);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: x_to_f16: %s", cudaGetErrorString(e));
   rc = after_launch("dsq_gemm_prefill: x_to_f16");
   if (rc != DSQ_OK) return rc;
 
   PrefillArgs args{};
-  args.w = static_cast<const uint8_t *>(w);
-  args.row_bytes = static_cast<int64_t>(dsq_row_bytes(type, K));
   args.N = N;
   args.K = K;
   args.M = M;
@@ -808,8 +955,9 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
-  args.groups_b = p.groups_b;
-  args.raw_slots = p.raw_slots;
+  args.slots_b = p.slots_b;
+  args.stages_per_slot = p.stages_per_slot;
+  args.slots_raw = p.slots_raw;
   args.stages_a = p.stages_a;
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
