@@ -47,8 +47,9 @@ constexpr int kRows = 128;          // weight rows per CTA (TMEM lanes)
 constexpr int kTileN = 2 * kRows;   // weight rows per pair tile (the MMA's M)
 constexpr int kBK = 64;             // K elements per pipeline stage
 constexpr int kAColsStage = kBK / 2;   // TMEM columns of one A stage (2 fp16 per column)
+constexpr int kAColsSlot = 2 * kAColsStage;   // an A slot holds 2 consecutive stages
 constexpr int kTmemCols = 512;      // the CTA owns all of TMEM (1 CTA per SM)
-constexpr int kMaxStagesA = 8;
+constexpr int kMaxSlotsA = 4;
 // warp roles
 constexpr int kWarpX = 0;         // bulk-copy producer: fp16 activation stages
 constexpr int kWarpMma = 1;       // TMEM owner; MMA issuer (even CTA) / activation relay (odd CTA)
@@ -69,7 +70,7 @@ struct PrefillArgs {
   int slots_b;            // activation slots in shared memory (stages_per_slot x 64 K x tn/2 tokens each)
   int stages_per_slot;    // 1, 2 or 4 stages of one K unit per activation copy
   int slots_raw;          // raw weight unit slots in shared memory (128 rows x 256 K each)
-  int stages_a;           // dequantized weight stages in TMEM (even)
+  int slots_a;            // dequantized weight slots in TMEM (2 stages each; even)
   int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
 };
@@ -160,49 +161,51 @@ __device__ __forceinline__ void piece_q4_k(const uint4 &hdr, Nib nib, uint32_t (
   }
 }
 
-// The registers a converter thread loads for piece P of a unit (uint4
-// granules of the row's 256-element unit), and the dequantization from them.
-// Q8_0: granules 4P .. 4P+4 (80 bytes covering the piece's 68, which start
-// at word P of them).  Q4_K: granule 0 (header) and 1+2P, 2+2P (the 32
-// nibble bytes).
-template <int TYPE> struct PieceRegs;
-template <> struct PieceRegs<DSQ_Q8_0> { uint4 v[5]; };
-template <> struct PieceRegs<DSQ_Q4_K> { uint4 hdr, v[2]; };
+// The registers a converter thread loads for stage pair J of a unit
+// (stages 2J and 2J+1 = pieces 2J, 2J+1; uint4 granules of the row's
+// 256-element unit) and the dequantization of piece 2J + i from them.
+// Q8_0: granules 8J .. 8J+8 (144 bytes covering the pair's 136, piece P
+// starting at word 17P - 32J of them).  Q4_K: granule 0 (header) and
+// 1+4J .. 4+4J (the pair's 64 nibble bytes).
+template <int TYPE> struct PairRegs;
+template <> struct PairRegs<DSQ_Q8_0> { uint4 v[9]; };
+template <> struct PairRegs<DSQ_Q4_K> { uint4 hdr, v[4]; };
 
-template <int TYPE, int P>
-__device__ __forceinline__ void load_piece(PieceRegs<TYPE> &r, const uint4 *unit) {
+template <int TYPE, int J>
+__device__ __forceinline__ void load_pair(PairRegs<TYPE> &r, const uint4 *unit) {
   if constexpr (TYPE == DSQ_Q8_0) {
 #pragma unroll
-    for (int i = 0; i < 5; ++i) r.v[i] = unit[4 * P + i];
+    for (int i = 0; i < 9; ++i) r.v[i] = unit[8 * J + i];
   } else {
     r.hdr = unit[0];
-    r.v[0] = unit[1 + 2 * P];
-    r.v[1] = unit[2 + 2 * P];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r.v[i] = unit[1 + 4 * J + i];
   }
 }
 
-template <int TYPE, int P>
-__device__ __forceinline__ void dequant_piece(const PieceRegs<TYPE> &r, uint32_t (&out)[32]) {
+template <int TYPE, int J, int I>
+__device__ __forceinline__ void dequant_pair_piece(const PairRegs<TYPE> &r, uint32_t (&out)[32]) {
+  constexpr int P = 2 * J + I;
   if constexpr (TYPE == DSQ_Q8_0) {
-    piece_q8_0([&](int i) { return word4(r.v[(P + i) >> 2], (P + i) & 3); }, out);
+    constexpr int o = 17 * P - 32 * J;
+    piece_q8_0([&](int i) { return word4(r.v[(o + i) >> 2], (o + i) & 3); }, out);
   } else {
-    piece_q4_k<P>(r.hdr, [&](int i) { return word4(r.v[i >> 2], i & 3); }, out);
+    piece_q4_k<P>(r.hdr, [&](int i) { return word4(r.v[2 * I + (i >> 2)], i & 3); }, out);
   }
 }
 
 // ------------------------------------------------------------------ GEMM ---
 // TMEM map of each CTA (512 columns x 128 lanes): [0, tn) the fp32
 // accumulators (lane = weight row of this CTA, column = token of the pair
-// tile); then stages_a dequantized-weight stages of 32 columns each (lane =
+// tile); then slots_a dequantized-weight slots of 2 stages = 64 columns each (lane =
 // weight row, each column two consecutive fp16 K elements).
 struct Smem {
   uint8_t *b;          // slots_b x stages_per_slot x (tn/2 rows x 128 B): activation stages (MMA B, this CTA's half)
   uint8_t *raw;        // slots_raw x 128 rows x unit bytes: raw weight units (TMA)
-  uint64_t *bfull;     // activation slot landed (1 + tx)
-  uint64_t *bpeer;     // even CTA: the odd CTA's activation slot landed (1, forwarded)
+  uint64_t *bfull;     // activation slot landed: odd CTA 1 + tx; even CTA 1 + tx + the odd CTA's forwarded arrival
   uint64_t *bempty;    // pair MMAs finished reading an activation slot (multicast commit)
-  uint64_t *afull;     // even CTA: a TMEM weight stage is stored in both CTAs (8 warp arrivals)
-  uint64_t *aempty;    // pair MMAs finished reading a TMEM weight stage (multicast commit)
+  uint64_t *afull;     // even CTA: a TMEM weight slot is stored in both CTAs (8 warp arrivals)
+  uint64_t *aempty;    // pair MMAs finished reading a TMEM weight slot (multicast commit)
   uint64_t *rfull;     // raw unit landed (1 + tx)
   uint64_t *rempty;    // converters copied a raw unit into registers (8 warps)
   uint64_t *accfull;   // accumulators complete (multicast commit)
@@ -213,17 +216,16 @@ struct Smem {
 };
 
 __device__ __forceinline__ Smem carve(uint8_t *base, int slots_b, uint32_t slot_b_bytes, int slots_raw,
-                                      uint32_t raw_bytes, int stages_a) {
+                                      uint32_t raw_bytes, int slots_a) {
   Smem s;
   s.b = base;
   s.raw = s.b + static_cast<size_t>(slots_b) * slot_b_bytes;
   uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(slots_raw) * raw_bytes);
   s.bfull = p;
-  s.bpeer = s.bfull + slots_b;
-  s.bempty = s.bpeer + slots_b;
+  s.bempty = s.bfull + slots_b;
   s.afull = s.bempty + slots_b;
-  s.aempty = s.afull + stages_a;
-  s.rfull = s.aempty + stages_a;
+  s.aempty = s.afull + slots_a;
+  s.rfull = s.aempty + slots_a;
   s.rempty = s.rfull + slots_raw;
   s.accfull = s.rempty + slots_raw;
   s.accempty = s.accfull + 1;
@@ -232,8 +234,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, int slots_b, uint32_t slot_
   s.abort = reinterpret_cast<volatile uint32_t *>(s.tmem + 1);
   return s;
 }
-__host__ __device__ constexpr size_t barrier_bytes(int slots_b, int slots_raw, int stages_a) {
-  return (3 * static_cast<size_t>(slots_b) + 2 * stages_a + 2 * slots_raw + 3) * sizeof(uint64_t) + 16;
+__host__ __device__ constexpr size_t barrier_bytes(int slots_b, int slots_raw, int slots_a) {
+  return (2 * static_cast<size_t>(slots_b) + 2 * slots_a + 2 * slots_raw + 3) * sizeof(uint64_t) + 16;
 }
 
 __device__ __forceinline__ bool aborted(const Smem &s) { return *s.abort != 0; }
@@ -279,20 +281,21 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   return tl;
 }
 
-// Converter warp of stage parity J (J = 0: stages 0 and 2 of every unit,
-// J = 1: stages 1 and 3): thread = weight row rr of this CTA.  Per unit it
-// copies the granules of its two pieces out of the raw slot, releases the
-// slot, and for each piece waits for a free TMEM stage, dequantizes 64
-// elements and stores them into its lane with one tcgen05.st; one lane per
-// warp then arrives on the even CTA's afull.
+// Converter warp of stage pair J (J = 0: stages 0 and 1 of every unit, J =
+// 1: stages 2 and 3): thread = weight row rr of this CTA.  Per unit it copies
+// the granules of its two pieces out of the raw slot, releases the slot,
+// waits for a free TMEM slot, dequantizes both stages (64 elements each) into
+// its lane with two tcgen05.st, and one lane per warp arrives on the even
+// CTA's afull once for the pair.  The warps of J = 0 fill slots 0, 2, 4, ...
+// of the ring, those of J = 1 slots 1, 3, 5, ...
 template <int TYPE, int J>
-__device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a, uint32_t tmem_stage0, int rr,
+__device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a, uint32_t tmem_slot0, int rr,
                                              uint32_t afull_even) {
   constexpr uint32_t RAW_BYTES = kRows * unit_bytes<TYPE>();
   const int lane = threadIdx.x & 31;
-  const int SA = a.stages_a, SR = a.slots_raw;
+  const int SA = a.slots_a, SR = a.slots_raw;
   const int64_t npairs = gridDim.x / 2;
-  int sa = J;            // TMEM stage slot of this warp's next stage (this warp takes every other one)
+  int sa = J;            // TMEM slot of this warp's next pair (every other slot)
   uint32_t rnd = 0;      // its ring round; round r >= 1 waits for the MMA release of round r - 1
   int rs = 0;            // raw unit slot and its phase parity
   uint32_t rpar = 0;
@@ -303,35 +306,37 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
       if (__any_sync(0xffffffffu, !got)) return;
       const uint4 *unit = reinterpret_cast<const uint4 *>(s.raw + static_cast<size_t>(rs) * RAW_BYTES +
                                                           static_cast<size_t>(rr) * unit_bytes<TYPE>());
-      PieceRegs<TYPE> r0, r1;
-      load_piece<TYPE, J>(r0, unit);
-      load_piece<TYPE, J + 2>(r1, unit);
+      PairRegs<TYPE> r;
+      load_pair<TYPE, J>(r, unit);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.rempty[rs]);
       if (++rs == SR) {
         rs = 0;
         rpar ^= 1u;
       }
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        if (rnd > 0) {
-          const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
-          if (__any_sync(0xffffffffu, !free_)) return;
-        }
+      if (rnd > 0) {
+        const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
+        if (__any_sync(0xffffffffu, !free_)) return;
+      }
+      tc_fence_after_sync();
+      {
         uint32_t v[32];
-        if (pp == 0) dequant_piece<TYPE, J>(r0, v);
-        else dequant_piece<TYPE, J + 2>(r1, v);
-        tc_fence_after_sync();
-        tmem_st_32cols(tmem_stage0 + static_cast<uint32_t>(sa * kAColsStage), v);
-        tmem_st_wait();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(afull_even + static_cast<uint32_t>(sa) * 8u);
-        sa += 2;
-        if (sa >= SA) {
-          sa -= SA;
-          ++rnd;
-        }
+        dequant_pair_piece<TYPE, J, 0>(r, v);
+        tmem_st_32cols(tmem_slot0 + static_cast<uint32_t>(sa * kAColsSlot), v);
+      }
+      {
+        uint32_t v[32];
+        dequant_pair_piece<TYPE, J, 1>(r, v);
+        tmem_st_32cols(tmem_slot0 + static_cast<uint32_t>(sa * kAColsSlot + kAColsStage), v);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(afull_even + static_cast<uint32_t>(sa) * 8u);
+      sa += 2;
+      if (sa >= SA) {
+        sa -= SA;
+        ++rnd;
       }
     }
   }
@@ -350,21 +355,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t stage_b_bytes = static_cast<uint32_t>(tnc) * 128u;   // one 64-K activation stage
   const int S2 = a.stages_per_slot;
   const uint32_t slot_b_bytes = stage_b_bytes * static_cast<uint32_t>(S2);   // one activation copy
-  const Smem s = carve(base, a.slots_b, slot_b_bytes, a.slots_raw, RAW_BYTES, a.stages_a);
+  const Smem s = carve(base, a.slots_b, slot_b_bytes, a.slots_raw, RAW_BYTES, a.slots_a);
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int SB = a.slots_b, SA = a.stages_a, SR = a.slots_raw;
+  const int SB = a.slots_b, SA = a.slots_a, SR = a.slots_raw;
   const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
   const int units = static_cast<int>(a.K / 256);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SB; ++i) {
-      mbar_init(&s.bfull[i], 1);
-      mbar_init(&s.bpeer[i], 1);
+      // the even CTA's also counts the odd CTA's forwarded arrival, so one
+      // wait covers both halves of the activation tile
+      mbar_init(&s.bfull[i], rank == 0 ? 2 : 1);
       mbar_init(&s.bempty[i], 1);
     }
     for (int i = 0; i < SA; ++i) {
-      mbar_init(&s.afull[i], 2 * 4);   // 4 converter warps per stage in each CTA
+      mbar_init(&s.afull[i], 2 * 4);   // 4 converter warps per slot in each CTA
       mbar_init(&s.aempty[i], 1);
     }
     for (int i = 0; i < SR; ++i) {
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma && rank == 1) {
     // ------------------------------- odd CTA: forward activation arrivals
     if (lane == 0) {
-      const uint32_t bpeer_even = mapa_shared(smem_u32(s.bpeer), 0);
+      const uint32_t bfull_even = mapa_shared(smem_u32(s.bfull), 0);
       int sb = 0;
       uint32_t par = 0;
       bool ok = true;
@@ -453,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_remote(bpeer_even + static_cast<uint32_t>(sb) * 8u);
+          mbar_arrive_remote(bfull_even + static_cast<uint32_t>(sb) * 8u);
           if (++sb == SB) {
             sb = 0;
             par ^= 1u;
@@ -467,7 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = umma_idesc_f16(kTileN, static_cast<uint32_t>(a.tn), 0);
       const uint32_t b_base = smem_u32(s.b);
       int64_t i = 0;
-      int sb = 0, sa = 0, gin = 0;   // gin: stage within the activation slot
+      const int P2 = S2 / 2;         // stage pairs per activation slot
+      int sb = 0, sa = 0, qin = 0;   // qin: stage pair within the activation slot
       uint32_t pb = 0, pa = 0;       // phase parity of the current round of each ring
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs, ++i) {
@@ -477,28 +484,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        for (int g = 0; g < 4 * (tl.u1 - tl.u0); ++g) {
-          if ((gin == 0 && (!wait_or_abort(s, &s.bfull[sb], pb, a.wait) ||
-                            !wait_or_abort(s, &s.bpeer[sb], pb, a.wait))) ||
-              !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
+        // one set of waits per 8 MMAs: the MMA issue queue is shallow, so the
+        // waits and commits between issues must stay short
+        for (int q = 0; q < 2 * (tl.u1 - tl.u0); ++q) {
+          if ((qin == 0 && !wait_or_abort(s, &s.bfull[sb], pb, a.wait)) || !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t b_addr =
-              b_base + static_cast<uint32_t>(sb) * slot_b_bytes + static_cast<uint32_t>(gin) * stage_b_bytes;
-          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsStage);
+          const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * slot_b_bytes +
+                                  static_cast<uint32_t>(2 * qin) * stage_b_bytes;
+          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsSlot);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_f16_ts_pair(tmem_base, a_tmem + static_cast<uint32_t>(8 * k), umma_desc_sw128(b_addr + 32 * k),
-                             idesc, (g > 0 || k > 0) ? 1u : 0u);
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_f16_ts_pair(tmem_base, a_tmem + static_cast<uint32_t>(h * kAColsStage + 8 * k),
+                               umma_desc_sw128(b_addr + static_cast<uint32_t>(h) * stage_b_bytes + 32 * k), idesc,
+                               (q > 0 || h > 0 || k > 0) ? 1u : 0u);
           umma_commit_pair_mc(&s.aempty[sa], 0x3);
           if (++sa == SA) {
             sa = 0;
             pa ^= 1u;
           }
-          if (++gin == S2) {
-            gin = 0;
+          if (++qin == P2) {
+            qin = 0;
             umma_commit_pair_mc(&s.bempty[sb], 0x3);
             if (++sb == SB) {
               sb = 0;
@@ -544,10 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kWarpEpi0) {
     // ------------------------------------------ converters (dequantize)
     const int q = warp & 3;   // TMEM lane quadrant this warp may access
-    const uint32_t stage0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a_col0;
+    const uint32_t slot0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a_col0;
     const uint32_t afull_even = mapa_shared(smem_u32(s.afull), 0);
-    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, stage0, 32 * q + lane, afull_even);
-    else convert_role<TYPE, 1>(s, a, stage0, 32 * q + lane, afull_even);
+    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, slot0, 32 * q + lane, afull_even);
+    else convert_role<TYPE, 1>(s, a, slot0, 32 * q + lane, afull_even);
   } else {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
     const int q = warp & 3;
@@ -703,16 +713,20 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
 
 // Test hook: the whole dequantized weight matrix in binary16, produced by the
 // same device functions as the GEMM's converter warps (one thread per
-// 256-element unit of a row).
-template <int TYPE, int P>
-__device__ __forceinline__ void unit_piece_to_f16(const uint4 *unit, uint16_t *dst) {
-  PieceRegs<TYPE> r;
-  load_piece<TYPE, P>(r, unit);
-  uint32_t v[32];
-  dequant_piece<TYPE, P>(r, v);
-  uint4 *d4 = reinterpret_cast<uint4 *>(dst + P * 64);
+// 256-element unit of a row, both stage pairs).
+template <int TYPE, int J>
+__device__ __forceinline__ void pair_to_f16(const uint4 *unit, uint16_t *dst) {
+  PairRegs<TYPE> r;
+  load_pair<TYPE, J>(r, unit);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) d4[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  for (int i = 0; i < 2; ++i) {
+    uint32_t v[32];
+    if (i == 0) dequant_pair_piece<TYPE, J, 0>(r, v);
+    else dequant_pair_piece<TYPE, J, 1>(r, v);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst + (2 * J + i) * 64);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) d4[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
 }
 
 template <int TYPE>
@@ -724,15 +738,13 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
   const int64_t n = idx / units, u = idx % units;
   const uint4 *unit = reinterpret_cast<const uint4 *>(w + n * row_bytes + u * unit_bytes<TYPE>());
   uint16_t *dst = w16 + n * K + u * 256;
-  unit_piece_to_f16<TYPE, 0>(unit, dst);
-  unit_piece_to_f16<TYPE, 1>(unit, dst);
-  unit_piece_to_f16<TYPE, 2>(unit, dst);
-  unit_piece_to_f16<TYPE, 3>(unit, dst);
+  pair_to_f16<TYPE, 0>(unit, dst);
+  pair_to_f16<TYPE, 1>(unit, dst);
 }
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, slots_b, stages_per_slot, slots_raw, stages_a, splits, units_per_split;
+  int tn, slots_b, stages_per_slot, slots_raw, slots_a, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
   unsigned grid;   // CTAs (2 per pair)
   size_t smem, x16_bytes, shift_off, part_off, total;
@@ -814,9 +826,9 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   const int units = static_cast<int>(K / 256);
   // TMEM: tn accumulator columns, then up to 8 (an even number of) 32-column
   // weight stages
-  p.stages_a = (kTmemCols - p.tn) / kAColsStage;
-  if (p.stages_a > kMaxStagesA) p.stages_a = kMaxStagesA;
-  p.stages_a &= ~1;
+  p.slots_a = (kTmemCols - p.tn) / kAColsSlot;
+  if (p.slots_a > kMaxSlotsA) p.slots_a = kMaxSlotsA;
+  p.slots_a &= ~1;   // the two converter groups alternate slots
   // shared memory.  The SM's copy engine costs a few hundred cycles per
   // copy whatever its size, so activation copies take up to 32 KB (2 or 4
   // stages of one K unit); up to 4 (at most 8) activation slots next to 2
@@ -826,13 +838,13 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   while (p.stages_per_slot < 4 && p.stages_per_slot * stage_b < 32 * 1024) p.stages_per_slot *= 2;
   const size_t slot_b = p.stages_per_slot * stage_b;
   const size_t raw_bytes = static_cast<size_t>(kRows) * (type == DSQ_Q8_0 ? 272 : 144);
-  const size_t fixed = 1024 + barrier_bytes(8, 4, p.stages_a);
+  const size_t fixed = 1024 + barrier_bytes(8, 4, p.slots_a);
   p.slots_b = static_cast<int>((kSmemLimit - fixed - 2 * raw_bytes) / slot_b);
   if (p.slots_b > 8) p.slots_b = 8;
   if (p.slots_b > 4 && slot_b >= 16 * 1024) p.slots_b = 4;
   p.slots_raw = static_cast<int>((kSmemLimit - fixed - p.slots_b * slot_b) / raw_bytes);
   if (p.slots_raw > 4) p.slots_raw = 4;
-  p.smem = 1024 + p.slots_b * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots_b, p.slots_raw, p.stages_a);
+  p.smem = 1024 + p.slots_b * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots_b, p.slots_raw, p.slots_a);
   if (pairs < 0) pairs = resident_pairs(type, p.smem, sms);
   const int64_t tiles = p.tiles_m * p.tiles_n;
   // split K only when the tiles leave more than half the pairs idle
@@ -911,7 +923,9 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots_b >= 2 && p.stages_a >= 2 && p.slots_raw >= 2, DSQ_ERR_SHAPE,
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots_b >= 2 && p.slots_a >= 2 && p.slots_raw >= 2 &&
+                  p.stages_per_slot % 2 == 0,
+              DSQ_ERR_SHAPE,
               "dsq_gemm_prefill: no pipeline fits");
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -958,7 +972,7 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   args.slots_b = p.slots_b;
   args.stages_per_slot = p.stages_per_slot;
   args.slots_raw = p.slots_raw;
-  args.stages_a = p.stages_a;
+  args.slots_a = p.slots_a;
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
