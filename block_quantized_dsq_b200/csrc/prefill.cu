@@ -49,7 +49,7 @@ constexpr int kBK = 64;             // K elements per pipeline stage
 constexpr int kAColsStage = kBK / 2;   // TMEM columns of one A stage (2 fp16 per column)
 constexpr int kAColsSlot = 2 * kAColsStage;   // an A slot holds 2 consecutive stages
 constexpr int kTmemCols = 512;      // the CTA owns all of TMEM (1 CTA per SM)
-constexpr int kMaxSlotsA = 4;
+constexpr int kMaxSlots = 6;
 // warp roles
 constexpr int kWarpX = 0;         // bulk-copy producer: fp16 activation stages
 constexpr int kWarpMma = 1;       // TMEM owner; MMA issuer (even CTA) / activation relay (odd CTA)
@@ -67,10 +67,9 @@ struct PrefillArgs {
   int units_per_split;    // 256-element units of K per split
   int splits;
   int tn;                 // tokens per pair tile (MMA N): 32..256, multiple of 32
-  int slots_b;            // activation slots in shared memory (stages_per_slot x 64 K x tn/2 tokens each)
-  int stages_per_slot;    // 1, 2 or 4 stages of one K unit per activation copy
+  int slots;              // pipeline slots: one stage pair each, activations in shared memory
+                          // (2 x 64 K x tn/2 tokens) and dequantized weights in TMEM (64 columns); even
   int slots_raw;          // raw weight unit slots in shared memory (128 rows x 256 K each)
-  int slots_a;            // dequantized weight slots in TMEM (2 stages each; even)
   int64_t tiles_m, tiles_n, total_tiles;
   WaitCtl wait;
 };
@@ -197,15 +196,15 @@ __device__ __forceinline__ void dequant_pair_piece(const PairRegs<TYPE> &r, uint
 // ------------------------------------------------------------------ GEMM ---
 // TMEM map of each CTA (512 columns x 128 lanes): [0, tn) the fp32
 // accumulators (lane = weight row of this CTA, column = token of the pair
-// tile); then slots_a dequantized-weight slots of 2 stages = 64 columns each (lane =
+// tile); then the dequantized-weight halves of the pipeline slots, 2 stages = 64 columns each (lane =
 // weight row, each column two consecutive fp16 K elements).
 struct Smem {
-  uint8_t *b;          // slots_b x stages_per_slot x (tn/2 rows x 128 B): activation stages (MMA B, this CTA's half)
+  uint8_t *b;          // slots x 2 stages x (tn/2 rows x 128 B): activation stages (MMA B, this CTA's half)
   uint8_t *raw;        // slots_raw x 128 rows x unit bytes: raw weight units (TMA)
-  uint64_t *bfull;     // activation slot landed: odd CTA 1 + tx; even CTA 1 + tx + the odd CTA's forwarded arrival
-  uint64_t *bempty;    // pair MMAs finished reading an activation slot (multicast commit)
-  uint64_t *afull;     // even CTA: a TMEM weight slot is stored in both CTAs (8 warp arrivals)
-  uint64_t *aempty;    // pair MMAs finished reading a TMEM weight slot (multicast commit)
+  uint64_t *ready;     // slot filled.  Even CTA: its activation copy (1 + tx), the odd CTA's forwarded
+                       // copy arrival (1) and the 4 converter warps of the slot in each CTA (8).
+                       // Odd CTA: its activation copy only (1 + tx), forwarded by its warp 1.
+  uint64_t *consumed;  // pair MMAs finished reading a slot (multicast commit to both CTAs)
   uint64_t *rfull;     // raw unit landed (1 + tx)
   uint64_t *rempty;    // converters copied a raw unit into registers (8 warps)
   uint64_t *accfull;   // accumulators complete (multicast commit)
@@ -215,17 +214,15 @@ struct Smem {
   volatile uint32_t *abort;
 };
 
-__device__ __forceinline__ Smem carve(uint8_t *base, int slots_b, uint32_t slot_b_bytes, int slots_raw,
-                                      uint32_t raw_bytes, int slots_a) {
+__device__ __forceinline__ Smem carve(uint8_t *base, int slots, uint32_t slot_b_bytes, int slots_raw,
+                                      uint32_t raw_bytes) {
   Smem s;
   s.b = base;
-  s.raw = s.b + static_cast<size_t>(slots_b) * slot_b_bytes;
+  s.raw = s.b + static_cast<size_t>(slots) * slot_b_bytes;
   uint64_t *p = reinterpret_cast<uint64_t *>(s.raw + static_cast<size_t>(slots_raw) * raw_bytes);
-  s.bfull = p;
-  s.bempty = s.bfull + slots_b;
-  s.afull = s.bempty + slots_b;
-  s.aempty = s.afull + slots_a;
-  s.rfull = s.aempty + slots_a;
+  s.ready = p;
+  s.consumed = s.ready + slots;
+  s.rfull = s.consumed + slots;
   s.rempty = s.rfull + slots_raw;
   s.accfull = s.rempty + slots_raw;
   s.accempty = s.accfull + 1;
@@ -234,8 +231,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, int slots_b, uint32_t slot_
   s.abort = reinterpret_cast<volatile uint32_t *>(s.tmem + 1);
   return s;
 }
-__host__ __device__ constexpr size_t barrier_bytes(int slots_b, int slots_raw, int slots_a) {
-  return (2 * static_cast<size_t>(slots_b) + 2 * slots_a + 2 * slots_raw + 3) * sizeof(uint64_t) + 16;
+__host__ __device__ constexpr size_t barrier_bytes(int slots, int slots_raw) {
+  return (2 * static_cast<size_t>(slots) + 2 * slots_raw + 3) * sizeof(uint64_t) + 16;
 }
 
 __device__ __forceinline__ bool aborted(const Smem &s) { return *s.abort != 0; }
@@ -286,14 +283,14 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
 // the granules of its two pieces out of the raw slot, releases the slot,
 // waits for a free TMEM slot, dequantizes both stages (64 elements each) into
 // its lane with two tcgen05.st, and one lane per warp arrives on the even
-// CTA's afull once for the pair.  The warps of J = 0 fill slots 0, 2, 4, ...
+// CTA's ready barrier of the slot.  The warps of J = 0 fill slots 0, 2, 4, ...
 // of the ring, those of J = 1 slots 1, 3, 5, ...
 template <int TYPE, int J>
 __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a, uint32_t tmem_slot0, int rr,
-                                             uint32_t afull_even) {
+                                             uint32_t ready_even) {
   constexpr uint32_t RAW_BYTES = kRows * unit_bytes<TYPE>();
   const int lane = threadIdx.x & 31;
-  const int SA = a.slots_a, SR = a.slots_raw;
+  const int SA = a.slots, SR = a.slots_raw;
   const int64_t npairs = gridDim.x / 2;
   int sa = J;            // TMEM slot of this warp's next pair (every other slot)
   uint32_t rnd = 0;      // its ring round; round r >= 1 waits for the MMA release of round r - 1
@@ -315,7 +312,7 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
         rpar ^= 1u;
       }
       if (rnd > 0) {
-        const bool free_ = wait_or_abort(s, &s.aempty[sa], (rnd - 1) & 1u, a.wait, 32);
+        const bool free_ = wait_or_abort(s, &s.consumed[sa], (rnd - 1) & 1u, a.wait, 32);
         if (__any_sync(0xffffffffu, !free_)) return;
       }
       tc_fence_after_sync();
@@ -332,7 +329,7 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(afull_even + static_cast<uint32_t>(sa) * 8u);
+      if (lane == 0) mbar_arrive_remote(ready_even + static_cast<uint32_t>(sa) * 8u);
       sa += 2;
       if (sa >= SA) {
         sa -= SA;
@@ -353,25 +350,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tnc = a.tn / 2;                                        // tokens of this CTA
   const uint32_t stage_b_bytes = static_cast<uint32_t>(tnc) * 128u;   // one 64-K activation stage
-  const int S2 = a.stages_per_slot;
-  const uint32_t slot_b_bytes = stage_b_bytes * static_cast<uint32_t>(S2);   // one activation copy
-  const Smem s = carve(base, a.slots_b, slot_b_bytes, a.slots_raw, RAW_BYTES, a.slots_a);
+  const uint32_t slot_b_bytes = 2u * stage_b_bytes;                    // one activation copy: a stage pair
+  const Smem s = carve(base, a.slots, slot_b_bytes, a.slots_raw, RAW_BYTES);
   const uint32_t rank = cluster_ctarank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int SB = a.slots_b, SA = a.slots_a, SR = a.slots_raw;
+  const int SQ = a.slots, SR = a.slots_raw;
   const int64_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
   const int units = static_cast<int>(a.K / 256);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < SB; ++i) {
-      // the even CTA's also counts the odd CTA's forwarded arrival, so one
-      // wait covers both halves of the activation tile
-      mbar_init(&s.bfull[i], rank == 0 ? 2 : 1);
-      mbar_init(&s.bempty[i], 1);
-    }
-    for (int i = 0; i < SA; ++i) {
-      mbar_init(&s.afull[i], 2 * 4);   // 4 converter warps per slot in each CTA
-      mbar_init(&s.aempty[i], 1);
+    for (int i = 0; i < SQ; ++i) {
+      // even CTA: its copy, the forwarded odd copy, 4 converter warps of each
+      // CTA -- one wait per slot covers all inputs of 8 MMAs
+      mbar_init(&s.ready[i], rank == 0 ? 2 + 2 * 4 : 1);
+      mbar_init(&s.consumed[i], 1);
     }
     for (int i = 0; i < SR; ++i) {
       mbar_init(&s.rfull[i], 1);
@@ -410,13 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------- activation stages (bulk copy)
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();   // every weight tile re-reads these
-      // One copy per slot: stages_per_slot consecutive stages of one K
-      // unit, contiguous in the tile-major layout (the copy engine's cost is
-      // mostly per copy, so copies are made as large as shared memory
-      // allows).  Ring position kept incrementally; round r >= 1 first
-      // waits for the MMA release of round r - 1.
+      // One copy per slot: the stage pair of one K unit, contiguous in the
+      // tile-major layout (32 KB for 128 tokens: the copy engine's cost is
+      // mostly per copy).  Ring position kept incrementally; round r >= 1
+      // first waits for the MMA release of round r - 1.
       int64_t gs = 0;
-      int sb = 0;
+      int sq = 0;
       uint32_t rnd = 0;
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
@@ -424,44 +415,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t xt = 2 * tl.mt + rank;   // this CTA's token tile
         int u = tl.u0 + tl.rot;
         for (int k = tl.u0; k < tl.u1 && ok; ++k, u = (u + 1 == tl.u1 ? tl.u0 : u + 1)) {
-          for (int kb4 = 0; kb4 < 4; kb4 += S2, ++gs) {
-            if (rnd > 0 && !wait_or_abort(s, &s.bempty[sb], (rnd - 1) & 1u, a.wait, 64)) {
+          for (int kb4 = 0; kb4 < 4; kb4 += 2, ++gs) {
+            if (rnd > 0 && !wait_or_abort(s, &s.consumed[sq], (rnd - 1) & 1u, a.wait, 64)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&s.bfull[sb], slot_b_bytes);
-            bulk_g2s(s.b + static_cast<size_t>(sb) * slot_b_bytes,
+            mbar_arrive_expect_tx(&s.ready[sq], slot_b_bytes);
+            bulk_g2s(s.b + static_cast<size_t>(sq) * slot_b_bytes,
                      reinterpret_cast<const uint8_t *>(a.x16) +
                          ((xt * units + u) * 4 + kb4) * static_cast<int64_t>(stage_b_bytes),
-                     slot_b_bytes, &s.bfull[sb], keep);
-            if (++sb == SB) {
-              sb = 0;
+                     slot_b_bytes, &s.ready[sq], keep);
+            if (++sq == SQ) {
+              sq = 0;
               ++rnd;
             }
           }
         }
       }
       if (!ok)
-        for (int64_t g = (gs > SB ? gs - SB : 0); g < gs; ++g)
-          mbar_wait_for(&s.bfull[g % SB], static_cast<uint32_t>((g / SB) & 1), kDrainLimitNs);
+        for (int64_t g = (gs > SQ ? gs - SQ : 0); g < gs; ++g)
+          mbar_wait_for(&s.ready[g % SQ], static_cast<uint32_t>((g / SQ) & 1), kDrainLimitNs);
     }
   } else if (warp == kWarpMma && rank == 1) {
     // ------------------------------- odd CTA: forward activation arrivals
     if (lane == 0) {
-      const uint32_t bfull_even = mapa_shared(smem_u32(s.bfull), 0);
-      int sb = 0;
+      const uint32_t ready_even = mapa_shared(smem_u32(s.ready), 0);
+      int sq = 0;
       uint32_t par = 0;
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
         const Tile tl = tile_of(a, t);
-        for (int g = 0; g < (4 / S2) * (tl.u1 - tl.u0); ++g) {
-          if (!wait_or_abort(s, &s.bfull[sb], par, a.wait)) {
+        for (int g = 0; g < 2 * (tl.u1 - tl.u0); ++g) {
+          if (!wait_or_abort(s, &s.ready[sq], par, a.wait)) {
             ok = false;
             break;
           }
-          mbar_arrive_remote(bfull_even + static_cast<uint32_t>(sb) * 8u);
-          if (++sb == SB) {
-            sb = 0;
+          mbar_arrive_remote(ready_even + static_cast<uint32_t>(sq) * 8u);
+          if (++sq == SQ) {
+            sq = 0;
             par ^= 1u;
           }
         }
@@ -473,9 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = umma_idesc_f16(kTileN, static_cast<uint32_t>(a.tn), 0);
       const uint32_t b_base = smem_u32(s.b);
       int64_t i = 0;
-      const int P2 = S2 / 2;         // stage pairs per activation slot
-      int sb = 0, sa = 0, qin = 0;   // qin: stage pair within the activation slot
-      uint32_t pb = 0, pa = 0;       // phase parity of the current round of each ring
+      int sq = 0;
+      uint32_t pq = 0;   // phase parity of the current round of the slot ring
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs, ++i) {
         const Tile tl = tile_of(a, t);
@@ -484,17 +474,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        // one set of waits per 8 MMAs: the MMA issue queue is shallow, so the
-        // waits and commits between issues must stay short
+        // One wait and one commit per 8 MMAs: the MMA issue queue is shallow,
+        // so what this thread does between issues must stay short.
         for (int q = 0; q < 2 * (tl.u1 - tl.u0); ++q) {
-          if ((qin == 0 && !wait_or_abort(s, &s.bfull[sb], pb, a.wait)) || !wait_or_abort(s, &s.afull[sa], pa, a.wait)) {
+          if (!wait_or_abort(s, &s.ready[sq], pq, a.wait)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t b_addr = b_base + static_cast<uint32_t>(sb) * slot_b_bytes +
-                                  static_cast<uint32_t>(2 * qin) * stage_b_bytes;
-          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAColsSlot);
+          const uint32_t b_addr = b_base + static_cast<uint32_t>(sq) * slot_b_bytes;
+          const uint32_t a_tmem = tmem_base + a_col0 + static_cast<uint32_t>(sq * kAColsSlot);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -502,18 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               umma_f16_ts_pair(tmem_base, a_tmem + static_cast<uint32_t>(h * kAColsStage + 8 * k),
                                umma_desc_sw128(b_addr + static_cast<uint32_t>(h) * stage_b_bytes + 32 * k), idesc,
                                (q > 0 || h > 0 || k > 0) ? 1u : 0u);
-          umma_commit_pair_mc(&s.aempty[sa], 0x3);
-          if (++sa == SA) {
-            sa = 0;
-            pa ^= 1u;
-          }
-          if (++qin == P2) {
-            qin = 0;
-            umma_commit_pair_mc(&s.bempty[sb], 0x3);
-            if (++sb == SB) {
-              sb = 0;
-              pb ^= 1u;
-            }
+          umma_commit_pair_mc(&s.consumed[sq], 0x3);
+          if (++sq == SQ) {
+            sq = 0;
+            pq ^= 1u;
           }
         }
         if (ok) umma_commit_pair_mc(s.accfull, 0x3);
@@ -555,9 +536,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------ converters (dequantize)
     const int q = warp & 3;   // TMEM lane quadrant this warp may access
     const uint32_t slot0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a_col0;
-    const uint32_t afull_even = mapa_shared(smem_u32(s.afull), 0);
-    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, slot0, 32 * q + lane, afull_even);
-    else convert_role<TYPE, 1>(s, a, slot0, 32 * q + lane, afull_even);
+    const uint32_t ready_even = mapa_shared(smem_u32(s.ready), 0);
+    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, slot0, 32 * q + lane, ready_even);
+    else convert_role<TYPE, 1>(s, a, slot0, 32 * q + lane, ready_even);
   } else {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
     const int q = warp & 3;
@@ -744,7 +725,7 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 
 // ------------------------------------------------------------------- host --
 struct Plan {
-  int tn, slots_b, stages_per_slot, slots_raw, slots_a, splits, units_per_split;
+  int tn, slots, slots_raw, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
   unsigned grid;   // CTAs (2 per pair)
   size_t smem, x16_bytes, shift_off, part_off, total;
@@ -826,25 +807,21 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   const int units = static_cast<int>(K / 256);
   // TMEM: tn accumulator columns, then up to 8 (an even number of) 32-column
   // weight stages
-  p.slots_a = (kTmemCols - p.tn) / kAColsSlot;
-  if (p.slots_a > kMaxSlotsA) p.slots_a = kMaxSlotsA;
-  p.slots_a &= ~1;   // the two converter groups alternate slots
-  // shared memory.  The SM's copy engine costs a few hundred cycles per
-  // copy whatever its size, so activation copies take up to 32 KB (2 or 4
-  // stages of one K unit); up to 4 (at most 8) activation slots next to 2
-  // raw weight units, then the rest to more raw units (at most 4).
-  const size_t stage_b = static_cast<size_t>(p.tn / 2) * 128;
-  p.stages_per_slot = 1;
-  while (p.stages_per_slot < 4 && p.stages_per_slot * stage_b < 32 * 1024) p.stages_per_slot *= 2;
-  const size_t slot_b = p.stages_per_slot * stage_b;
+  // pipeline slots (a stage pair each): as many as TMEM holds next to the
+  // accumulators (at most 6, even, so the two converter groups alternate)
+  p.slots = (kTmemCols - p.tn) / kAColsSlot;
+  if (p.slots > kMaxSlots) p.slots = kMaxSlots;
+  p.slots &= ~1;
+  // shared memory: the slots' activation pairs (32 KB each for 128 tokens:
+  // the copy engine's cost is mostly per copy), the rest to raw weight
+  // units (at least 2, at most 4)
+  const size_t slot_b = 2 * static_cast<size_t>(p.tn / 2) * 128;
   const size_t raw_bytes = static_cast<size_t>(kRows) * (type == DSQ_Q8_0 ? 272 : 144);
-  const size_t fixed = 1024 + barrier_bytes(8, 4, p.slots_a);
-  p.slots_b = static_cast<int>((kSmemLimit - fixed - 2 * raw_bytes) / slot_b);
-  if (p.slots_b > 8) p.slots_b = 8;
-  if (p.slots_b > 4 && slot_b >= 16 * 1024) p.slots_b = 4;
-  p.slots_raw = static_cast<int>((kSmemLimit - fixed - p.slots_b * slot_b) / raw_bytes);
+  const size_t fixed = 1024 + barrier_bytes(kMaxSlots, 4);
+  while (p.slots > 2 && fixed + p.slots * slot_b + 2 * raw_bytes > kSmemLimit) p.slots -= 2;
+  p.slots_raw = static_cast<int>((kSmemLimit - fixed - p.slots * slot_b) / raw_bytes);
   if (p.slots_raw > 4) p.slots_raw = 4;
-  p.smem = 1024 + p.slots_b * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots_b, p.slots_raw, p.slots_a);
+  p.smem = 1024 + p.slots * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots, p.slots_raw);
   if (pairs < 0) pairs = resident_pairs(type, p.smem, sms);
   const int64_t tiles = p.tiles_m * p.tiles_n;
   // split K only when the tiles leave more than half the pairs idle
@@ -923,9 +900,7 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots_b >= 2 && p.slots_a >= 2 && p.slots_raw >= 2 &&
-                  p.stages_per_slot % 2 == 0,
-              DSQ_ERR_SHAPE,
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots >= 2 && p.slots_raw >= 2, DSQ_ERR_SHAPE,
               "dsq_gemm_prefill: no pipeline fits");
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -969,10 +944,8 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
-  args.slots_b = p.slots_b;
-  args.stages_per_slot = p.stages_per_slot;
+  args.slots = p.slots;
   args.slots_raw = p.slots_raw;
-  args.slots_a = p.slots_a;
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
