@@ -23,14 +23,16 @@
 //    CTA's 128 lanes = its 128 rows), the activations are the B operand in
 //    shared memory (each CTA holds half of the N = tn columns);  "swap AB"
 //    keeps small token counts on full 128-lane MMAs;
-//  * per CTA: warp 0 streams activation stages (bulk copies of a tile-major
-//    fp16 layout, 64 K x tn/2 tokens each); warp 14 streams raw weight units
-//    (TMA, 128 rows x 256 K); warps 2-9 dequantize (two threads per weight
-//    row, alternate 64-K stages) into the TMEM A ring; warps 10-13 drain the
-//    fp32 accumulators (tcgen05.ld -> scale by 2^-s_m -> global);
-//  * warp 1 of the even CTA issues the pair MMAs; warp 1 of the odd CTA
-//    forwards "activation stage landed" to it.  MMA completion releases
-//    stages in both CTAs through multicast tcgen05.commit;
+//  * the pipeline runs in slots of one stage pair (2 x 64 K): per CTA, warp 0
+//    copies the slot's activations (one bulk copy of a tile-major fp16
+//    layout), warp 14 streams raw weight units (TMA, 128 rows x 256 K), warps
+//    2-9 dequantize (thread = weight row; warps 2-5 the first stage pair of
+//    each unit, 6-9 the second) into the slot's TMEM columns, warps 10-13
+//    drain the fp32 accumulators (tcgen05.ld -> scale by 2^-s_m -> global);
+//  * warp 1 of the even CTA issues the pair MMAs: one wait on the slot's
+//    ready barrier and one multicast tcgen05.commit to both CTAs' consumed
+//    barrier per 8 MMAs (the tcgen05 issue queue is shallow); warp 1 of the
+//    odd CTA forwards "activation slot landed" to the even CTA;
 //  * every wait is bounded; an expired wait records a timeout, raises the
 //    abort flag of both CTAs, drains copies and MMAs in flight, and the pair
 //    meets at a final cluster barrier before TMEM is freed.
