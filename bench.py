@@ -431,7 +431,9 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
         rows["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 3),
                                           "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 2)}
 
-    def gemv_row(name, qtype, N, K, seed, xseed, G=1):
+    def gemv_row(name, qtype, N, K, seed, xseed, G=1, fused=False):
+        """fused: the *_f32 entry point (fp32 activation quantized in the
+        kernel) instead of the two-call path's GEMV alone."""
         if not want(name):
             return
         w = quantized_weights(dsq, qtype, seed, G * N, K)
@@ -442,14 +444,22 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
         x, xq, xd, xs = act(xseed, G, K)
         y = torch.empty((G, N), dtype=torch.float32, device="cuda")
         pq, pd, ps, py = xq.data_ptr(), xd.data_ptr(), xs.data_ptr(), y.data_ptr()
-        if G > 1:
+        px = x.data_ptr()
+        if fused and G > 1:
+            fn = lambda i, st: L.dsq_gemv_grouped_f32(qtype, ptrs[i % R], G, N, K, px, py, st)  # noqa: E731
+        elif fused:
+            fn = lambda i, st: L.dsq_gemv_f32(qtype, ptrs[i % R], N, K, px, py, st)  # noqa: E731
+        elif G > 1:
             fn = lambda i, st: L.dsq_gemv_grouped(qtype, ptrs[i % R], G, N, K, pq, pd, ps, py, st)  # noqa: E731
         elif qtype == dsq.DSQ_Q8_0:
             fn = lambda i, st: L.dsq_gemv_q8_0(ptrs[i % R], N, K, pq, pd, py, st)  # noqa: E731
         else:
             fn = lambda i, st: L.dsq_gemv_q4_k(ptrs[i % R], N, K, pq, pd, ps, py, st)  # noqa: E731
         t = time_graph(fn, R * max(1, 200 // R))
-        alg = nbytes + G * (K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1)) + G * N * 4
+        if fused:
+            alg = nbytes + G * K * 4 + G * N * 4
+        else:
+            alg = nbytes + G * (K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1)) + G * N * 4
         gbs = alg / t / 1e9
         rows[name] = {"us_per_call": round(t * 1e6, 3), "GB/s": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
                       "algorithmic_bytes": alg, "weight_copies": R}
@@ -462,6 +472,39 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
              seeds["gemv_q4_k_4096"]["x"])
     gemv_row("grouped_q8_0_8x1024x4096", dsq.DSQ_Q8_0, 1024, 4096, seeds["grouped_q8_0_8x1024x4096"]["w_base"],
              seeds["grouped_q8_0_8x1024x4096"]["x_base"], G=8)
+    # the same decode GEMVs through the fused entry points (activation fp32
+    # in, quantized inside the GEMV: one launch per call)
+    gemv_row("f32_gemv_q8_0_1024x1024", dsq.DSQ_Q8_0, 1024, 1024, seeds["gemv_q8_0_1024"]["w"],
+             seeds["gemv_q8_0_1024"]["x"], fused=True)
+    gemv_row("f32_gemv_q4_k_4096x4096", dsq.DSQ_Q4_K, 4096, 4096, seeds["gemv_q4_k_4096"]["w"],
+             seeds["gemv_q4_k_4096"]["x"], fused=True)
+    gemv_row("f32_grouped_q8_0_8x1024x4096", dsq.DSQ_Q8_0, 1024, 4096,
+             seeds["grouped_q8_0_8x1024x4096"]["w_base"], seeds["grouped_q8_0_8x1024x4096"]["x_base"], G=8,
+             fused=True)
+    if want("f32_paired_q8_0_2x8192x4096"):
+        sp = seeds["paired_q8_0_2x8192x4096"]
+        W0 = quantized_weights(dsq, dsq.DSQ_Q8_0, sp["w0"], N_PAIR, K_PAIR)
+        W1 = quantized_weights(dsq, dsq.DSQ_Q8_0, sp["w1"], N_PAIR, K_PAIR)
+        nb2 = W0.numel() + W1.numel()
+        R = copies_for(nb2)
+        pw = [(W0.data_ptr(), W1.data_ptr())]
+        keep = []
+        for _ in range(R - 1):
+            c0, c1 = W0.clone(), W1.clone()
+            keep += [c0, c1]
+            pw.append((c0.data_ptr(), c1.data_ptr()))
+        xs_ = torch.from_numpy(synth.activations(sp["x_base"], 1, K_PAIR)).cuda()
+        y2 = torch.empty((2, N_PAIR), dtype=torch.float32, device="cuda")
+        px, py0, py1 = xs_.data_ptr(), y2[0].data_ptr(), y2[1].data_ptr()
+        fn = lambda i, st: L.dsq_gemv_paired_f32(dsq.DSQ_Q8_0, pw[i % R][0], N_PAIR, pw[i % R][1], N_PAIR,  # noqa: E731
+                                                 K_PAIR, px, py0, py1, st)
+        t = time_graph(fn, R * max(1, 128 // R))
+        alg = nb2 + K_PAIR * 4 + 2 * N_PAIR * 4
+        gbs = alg / t / 1e9
+        rows["f32_paired_q8_0_2x8192x4096"] = {"us_per_call": round(t * 1e6, 3), "GB/s": round(gbs, 1),
+                                               "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes": alg,
+                                               "weight_copies": R}
+        del keep, W0, W1
 
     # prefill dequant-GEMM sweep
     K = 4096

@@ -15,7 +15,8 @@ import threading
 
 __all__ = [
     "DSQ_Q8_0", "DSQ_Q4_K", "DsqError", "lib", "dsq_row_bytes", "dsq_quantize_act_q8",
-    "dsq_gemv_q8_0", "dsq_gemv_q4_k", "dsq_gemv_paired", "dsq_gemv_grouped", "dsq_gemm_prefill",
+    "dsq_gemv_q8_0", "dsq_gemv_q4_k", "dsq_gemv_paired", "dsq_gemv_grouped", "dsq_gemv_f32",
+    "dsq_gemv_paired_f32", "dsq_gemv_grouped_f32", "dsq_gemm_prefill",
     "dsq_prefill_workspace_bytes", "dsq_gemm_prefill_noalloc", "dsq_quantize_weights", "dsq_device_status", "dsq_last_error",
     "dsq_version", "dsq_launch_count", "dsq_test_block_sums", "dsq_test_set_wait_limit_ns",
     "dsq_test_prefill_operands", "LIB_PATH",
@@ -43,6 +44,9 @@ _SIGS = {
     "dsq_gemv_q4_k": (_INT, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "dsq_gemv_paired": (_INT, [_INT, _P, _I64, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "dsq_gemv_grouped": (_INT, [_INT, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "dsq_gemv_f32": (_INT, [_INT, _P, _I64, _I64, _P, _P, _P]),
+    "dsq_gemv_paired_f32": (_INT, [_INT, _P, _I64, _P, _I64, _I64, _P, _P, _P, _P]),
+    "dsq_gemv_grouped_f32": (_INT, [_INT, _P, _I64, _I64, _I64, _P, _P, _P]),
     "dsq_gemm_prefill": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "dsq_prefill_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64]),
     "dsq_gemm_prefill_noalloc": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P]),
@@ -134,6 +138,22 @@ def dsq_gemv_grouped(qtype, w, G, N, K, xq, xd, xs, y, stream=None):
     _check("dsq_gemv_grouped",
            lib().dsq_gemv_grouped(qtype, _ptr(w), G, N, K, _ptr(xq), _ptr(xd), _ptr(xs), _ptr(y),
                                   _stream(stream)))
+
+
+def dsq_gemv_f32(qtype, w, N, K, x, y, stream=None):
+    """Quantize the fp32 activation and run the GEMV in one launch."""
+    _check("dsq_gemv_f32", lib().dsq_gemv_f32(qtype, _ptr(w), N, K, _ptr(x), _ptr(y), _stream(stream)))
+
+
+def dsq_gemv_paired_f32(qtype, w0, N0, w1, N1, K, x, y0, y1, stream=None):
+    _check("dsq_gemv_paired_f32",
+           lib().dsq_gemv_paired_f32(qtype, _ptr(w0), N0, _ptr(w1), N1, K, _ptr(x), _ptr(y0), _ptr(y1),
+                                     _stream(stream)))
+
+
+def dsq_gemv_grouped_f32(qtype, w, G, N, K, x, y, stream=None):
+    _check("dsq_gemv_grouped_f32",
+           lib().dsq_gemv_grouped_f32(qtype, _ptr(w), G, N, K, _ptr(x), _ptr(y), _stream(stream)))
 
 
 def dsq_gemm_prefill(qtype, w, N, K, x, M, y, workspace, workspace_bytes, stream=None):

@@ -28,7 +28,14 @@
 //    (d_w * xd) * isum in fp32; lanes reduce with xor-shuffles; one store
 //    per row.  Rows whose byte length is not a multiple of 16 (Q8_0 with
 //    K % 256 != 0) take a plain warp-per-row kernel instead.
+//  * The *_f32 entry points take the fp32 activation and quantize it inside
+//    the GEMV: each CTA starts its weight copies, then its 256 threads
+//    quantize every activation row into shared memory (the rule of
+//    act_q8.cuh), and the lanes read their slices from there.  Same codes,
+//    same dot order -- the outputs equal the two-call path bit for bit --
+//    but one launch per call instead of two.
 #include "../../include/dsq_test.h"
+#include "act_q8.cuh"
 #include "dsq_host.h"
 
 // Launch shape (compile-time constants; the defaults are the tuned values).
@@ -70,6 +77,9 @@ struct GemvArgs {
   int slot_bytes;       // rows-per-slot * row_bytes
   WaitCtl wait;
   int32_t *isum;        // test hook: per-block int32 sums (NULL in production)
+  const float *x32;     // fused mode: fp32 activation rows [act_rows][K], quantized in the kernel
+  int64_t act_rows;     // activation rows (1, or the group count)
+  int act_off;          // fused mode: byte offset of the activation area in shared memory
 };
 
 template <int TYPE> struct Unit;
@@ -86,26 +96,64 @@ struct ActSlice {
   int32_t s[8];     // 8 block code sums (Q4_K only)
 };
 
-template <int TYPE>
+// SMEM: the slice lives in this CTA's shared memory (fused mode), else in
+// global memory (read-only path).
+template <int TYPE, bool SMEM>
 __device__ __forceinline__ void load_act(ActSlice &act, const int8_t *xq, const float *xd, const int32_t *xs) {
   const uint4 *q4 = reinterpret_cast<const uint4 *>(xq);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint4 v = __ldg(q4 + i);
+    const uint4 v = SMEM ? q4[i] : __ldg(q4 + i);
     act.q[4 * i + 0] = v.x; act.q[4 * i + 1] = v.y; act.q[4 * i + 2] = v.z; act.q[4 * i + 3] = v.w;
   }
   const float4 *d4 = reinterpret_cast<const float4 *>(xd);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const float4 v = __ldg(d4 + i);
+    const float4 v = SMEM ? d4[i] : __ldg(d4 + i);
     act.d[4 * i + 0] = v.x; act.d[4 * i + 1] = v.y; act.d[4 * i + 2] = v.z; act.d[4 * i + 3] = v.w;
   }
   if (TYPE == DSQ_Q4_K) {
     const int4 *s4 = reinterpret_cast<const int4 *>(xs);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int4 v = __ldg(s4 + i);
+      const int4 v = SMEM ? s4[i] : __ldg(s4 + i);
       act.s[4 * i + 0] = v.x; act.s[4 * i + 1] = v.y; act.s[4 * i + 2] = v.z; act.s[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// Fused mode: the CTA's threads quantize activation rows [g0, g0 + rows)
+// into shared memory (xq [rows][K] int8, then xd and xs [rows][K/32]).  8 lanes
+// per 32-block, 4 elements each.  Each thread issues the loads of 4 float4s
+// before quantizing them (one L2 round trip per batch, not per float4), and
+// the loop runs the same number of iterations in every thread so each warp's
+// shuffles see all 32 lanes.
+__device__ __forceinline__ void quantize_act_to_smem(const GemvArgs &a, int64_t g0, int64_t rows, int8_t *sq,
+                                                     float *sd, int32_t *ss) {
+  constexpr int kBatch = 4;
+  const int64_t tasks = rows * a.K / 4;   // float4s
+  const float4 *x4 = reinterpret_cast<const float4 *>(a.x32 + g0 * a.K);
+  const int64_t step = static_cast<int64_t>(blockDim.x) * kBatch;
+  for (int64_t base = 0; base < tasks; base += step) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t t = base + i * blockDim.x + threadIdx.x;
+      v[i] = t < tasks ? __ldg(x4 + t) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int64_t t = base + i * blockDim.x + threadIdx.x;
+      float d;
+      int sum;
+      const uint32_t packed = q8_block_lanes(v[i], d, sum);
+      if (t < tasks) {
+        reinterpret_cast<uint32_t *>(sq)[t] = packed;
+        if ((t & 7) == 0) {
+          sd[t >> 3] = d;
+          ss[t >> 3] = sum;
+        }
+      }
     }
   }
 }
@@ -209,7 +257,7 @@ __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_
   }
 }
 
-template <int TYPE, int G, bool ISUM>
+template <int TYPE, int G, bool ISUM, bool FUSED>
 __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
   constexpr int RPC = 32 / G;  // rows per slot
   extern __shared__ __align__(128) uint8_t smem[];
@@ -236,12 +284,22 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       }
     }
   }
+  if (FUSED && threadIdx.x == 0) {
+    // the fp32 activation rows this CTA will quantize, toward L2 (a hint:
+    // the predecessor's writes still win, L2 being the point of coherence)
+    int64_t ga = 0, gb = 0;
+    if (r1 > r0 && a.act_rows > 1) {
+      ga = r0 / a.group_rows;
+      gb = (r1 - 1) / a.group_rows;
+    }
+    prefetch_l2(a.x32 + ga * a.K, static_cast<uint32_t>((gb - ga + 1) * a.K * 4));
+  }
   pdl_trigger();
   pdl_wait();
-  if (mine == 0) return;
+  if (!FUSED && mine == 0) return;
 
   const uint64_t policy = l2_policy_evict_first();
-  if (lane == 0) {
+  if (lane == 0 && mine > 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
     for (int64_t k = 0; k < mine && k < S; ++k) {
@@ -249,6 +307,30 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
       issue_rows(a, ra, rb, ring + k * a.slot_bytes, &bars[k], policy);
     }
+  }
+  // activation source: global (two-call path) or quantized here, into shared
+  // memory, while the first weight copies are in flight
+  const int8_t *xq = a.xq;
+  const float *xd = a.xd;
+  const int32_t *xs = a.xs;
+  if (FUSED) {
+    // only the activation groups this CTA's rows read: [g0, g1]
+    int64_t g0 = 0, g1 = 0;
+    if (r1 > r0 && a.act_rows > 1) {
+      g0 = r0 / a.group_rows;
+      g1 = (r1 - 1) / a.group_rows;
+    }
+    const int64_t rows = g1 - g0 + 1;
+    int8_t *sq = reinterpret_cast<int8_t *>(smem + a.act_off);
+    float *sd = reinterpret_cast<float *>(sq + rows * a.K);
+    int32_t *ss = reinterpret_cast<int32_t *>(sd + rows * (a.K / 32));
+    quantize_act_to_smem(a, g0, rows, sq, sd, ss);
+    __syncthreads();
+    if (mine == 0) return;
+    // indexed by absolute group below: shift the bases by g0 rows
+    xq = sq - g0 * a.K;
+    xd = sd - g0 * (a.K / 32);
+    xs = ss - g0 * (a.K / 32);
   }
   __syncwarp();
 
@@ -282,7 +364,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
         const int64_t key = group * a.nunits + u;
         if (key != cached) {
           const int64_t e0 = group * a.K + static_cast<int64_t>(u) * 256;
-          load_act<TYPE>(act, a.xq + e0, a.xd + e0 / 32, TYPE == DSQ_Q4_K ? a.xs + e0 / 32 : nullptr);
+          load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
           cached = key;
         }
         int32_t is[8];
@@ -356,12 +438,21 @@ __global__ void __launch_bounds__(256) gemv_q8_0_rowwise_kernel(const __grid_con
 constexpr int kMaxWarps = DSQ_GEMV_MAX_WARPS;
 constexpr size_t kSmemBudget = DSQ_GEMV_SMEM_KB * 1024;
 
-template <int TYPE, int G, bool ISUM>
+// Shared memory of the activation area in fused mode: int8 codes plus fp32
+// scales and int32 sums per 32-block.
+size_t act_smem_bytes(int64_t rows, int64_t K) { return static_cast<size_t>(rows) * (K + 8 * (K / 32)); }
+
+template <int TYPE, int G, bool ISUM, bool FUSED>
 int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   constexpr int RPC = 32 / G;
-  const size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
-                      static_cast<size_t>(a.warps) * a.stages * sizeof(uint64_t);
-  auto kern = gemv_kernel<TYPE, G, ISUM>;
+  size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
+                static_cast<size_t>(a.warps) * a.stages * sizeof(uint64_t);
+  if (FUSED) {
+    smem = (smem + 15) / 16 * 16;
+    a.act_off = static_cast<int>(smem);
+    smem += act_smem_bytes(a.act_rows, a.K);
+  }
+  auto kern = gemv_kernel<TYPE, G, ISUM, FUSED>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
   if (rc != DSQ_OK) return rc;
   const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
@@ -372,21 +463,28 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   return after_launch("gemv");
 }
 
-template <int TYPE, bool ISUM>
+template <int TYPE, bool ISUM, bool FUSED>
 int dispatch_g(GemvArgs &a, int G, int num_sms, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_fast<TYPE, 1, ISUM>(a, num_sms, stream);
-    case 2: return launch_fast<TYPE, 2, ISUM>(a, num_sms, stream);
-    case 4: return launch_fast<TYPE, 4, ISUM>(a, num_sms, stream);
-    case 8: return launch_fast<TYPE, 8, ISUM>(a, num_sms, stream);
-    case 16: return launch_fast<TYPE, 16, ISUM>(a, num_sms, stream);
-    default: return launch_fast<TYPE, 32, ISUM>(a, num_sms, stream);
+    case 1: return launch_fast<TYPE, 1, ISUM, FUSED>(a, num_sms, stream);
+    case 2: return launch_fast<TYPE, 2, ISUM, FUSED>(a, num_sms, stream);
+    case 4: return launch_fast<TYPE, 4, ISUM, FUSED>(a, num_sms, stream);
+    case 8: return launch_fast<TYPE, 8, ISUM, FUSED>(a, num_sms, stream);
+    case 16: return launch_fast<TYPE, 16, ISUM, FUSED>(a, num_sms, stream);
+    default: return launch_fast<TYPE, 32, ISUM, FUSED>(a, num_sms, stream);
   }
 }
 
-// Validates and launches one GEMV over up to two segments.
+// Largest activation area the fused mode keeps in shared memory (e.g. 8 rows
+// of K = 4096, or one row of K = 49152).
+constexpr size_t kMaxActSmem = 64 * 1024;
+
+// Validates and launches one GEMV over up to two segments.  x32 != NULL
+// selects the fused mode (fp32 activation rows quantized inside the kernel;
+// xq/xd/xs unused).
 int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int64_t groups, int64_t K,
-             const int8_t *xq, const float *xd, const int32_t *xs, int32_t *isum, cudaStream_t stream) {
+             const int8_t *xq, const float *xd, const int32_t *xs, int32_t *isum, cudaStream_t stream,
+             const float *x32 = nullptr) {
   DSQ_REQUIRE(type == DSQ_Q8_0 || type == DSQ_Q4_K, DSQ_ERR_INVALID_ARG, "%s: unsupported type %d", name, type);
   DSQ_REQUIRE(K > 0 && s0.rows >= 0 && s1.rows >= 0, DSQ_ERR_INVALID_ARG, "%s: negative size", name);
   const size_t rb = dsq_row_bytes(type, K);
@@ -396,15 +494,22 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
               "%s: size out of range (K <= 2^20, rows <= 2^31)", name);
   const int64_t total = s0.rows + s1.rows;
   if (total == 0) return DSQ_OK;
-  DSQ_REQUIRE(xq && xd && (type == DSQ_Q8_0 || xs), DSQ_ERR_INVALID_ARG, "%s: null activation pointer", name);
+  if (x32) {
+    DSQ_REQUIRE(aligned(x32, 16), DSQ_ERR_ALIGNMENT, "%s: x must be 16-byte aligned", name);
+    DSQ_REQUIRE(rb % 16 == 0, DSQ_ERR_SHAPE, "%s: K=%lld: the fused form needs K %% 256 == 0", name, (long long)K);
+    DSQ_REQUIRE(act_smem_bytes(groups, K) <= kMaxActSmem, DSQ_ERR_SHAPE,
+                "%s: %lld activation rows of K=%lld exceed the fused form's %zu bytes of shared memory", name,
+                (long long)groups, (long long)K, kMaxActSmem);
+  } else {
+    DSQ_REQUIRE(xq && xd && (type == DSQ_Q8_0 || xs), DSQ_ERR_INVALID_ARG, "%s: null activation pointer", name);
+  }
   DSQ_REQUIRE((s0.rows == 0 || (s0.w && s0.y)) && (s1.rows == 0 || (s1.w && s1.y)), DSQ_ERR_INVALID_ARG,
               "%s: null weight/output pointer", name);
-  DSQ_REQUIRE(aligned(xq, 16) && aligned(xd, 16) && (!xs || aligned(xs, 16)), DSQ_ERR_ALIGNMENT,
+  DSQ_REQUIRE(x32 || (aligned(xq, 16) && aligned(xd, 16) && (!xs || aligned(xs, 16))), DSQ_ERR_ALIGNMENT,
               "%s: xq/xd/xs must be 16-byte aligned", name);
   DSQ_REQUIRE((s0.rows == 0 || (aligned(s0.w, 16) && aligned(s0.y, 4))) &&
                   (s1.rows == 0 || (aligned(s1.w, 16) && aligned(s1.y, 4))),
               DSQ_ERR_ALIGNMENT, "%s: weights must be 16-byte and outputs 4-byte aligned", name);
-  (void)groups;
   WaitCtl ctl;
   int num_sms = 0;
   int rc = wait_ctl(&ctl, &num_sms);
@@ -423,6 +528,8 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   a.row_bytes = static_cast<int64_t>(rb);
   a.wait = ctl;
   a.isum = isum;
+  a.x32 = x32;
+  a.act_rows = groups;
 
   if (rb % 16 != 0) {  // Q8_0 with K % 256 != 0
     const int64_t blocks = (total + 7) / 8;
@@ -436,15 +543,22 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   int G = 1;
   while (G < a.nunits && G < 32) G <<= 1;
   a.slot_bytes = static_cast<int>((32 / G) * rb);
+  // the ring gets the shared memory the fused activation area leaves
+  const size_t budget = kSmemBudget - (x32 ? act_smem_bytes(groups, K) + 16 : 0);
   a.warps = kMaxWarps;
-  while (a.warps > 1 && static_cast<size_t>(a.warps) * 2 * a.slot_bytes > kSmemBudget) a.warps >>= 1;
-  DSQ_REQUIRE(static_cast<size_t>(a.warps) * 2 * a.slot_bytes <= kSmemBudget, DSQ_ERR_SHAPE,
+  while (a.warps > 1 && static_cast<size_t>(a.warps) * 2 * a.slot_bytes > budget) a.warps >>= 1;
+  DSQ_REQUIRE(static_cast<size_t>(a.warps) * 2 * a.slot_bytes <= budget, DSQ_ERR_SHAPE,
               "%s: K=%lld rows do not fit the shared-memory pipeline", name, (long long)K);
-  a.stages = static_cast<int>(kSmemBudget / (static_cast<size_t>(a.warps) * a.slot_bytes));
+  a.stages = static_cast<int>(budget / (static_cast<size_t>(a.warps) * a.slot_bytes));
   if (a.stages > DSQ_GEMV_MAX_STAGES) a.stages = DSQ_GEMV_MAX_STAGES;
+  if (x32)
+    return type == DSQ_Q8_0 ? dispatch_g<DSQ_Q8_0, false, true>(a, G, num_sms, stream)
+                            : dispatch_g<DSQ_Q4_K, false, true>(a, G, num_sms, stream);
   if (type == DSQ_Q8_0)
-    return isum ? dispatch_g<DSQ_Q8_0, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q8_0, false>(a, G, num_sms, stream);
-  return isum ? dispatch_g<DSQ_Q4_K, true>(a, G, num_sms, stream) : dispatch_g<DSQ_Q4_K, false>(a, G, num_sms, stream);
+    return isum ? dispatch_g<DSQ_Q8_0, true, false>(a, G, num_sms, stream)
+                : dispatch_g<DSQ_Q8_0, false, false>(a, G, num_sms, stream);
+  return isum ? dispatch_g<DSQ_Q4_K, true, false>(a, G, num_sms, stream)
+              : dispatch_g<DSQ_Q4_K, false, false>(a, G, num_sms, stream);
 }
 
 constexpr int64_t kOneGroup = int64_t(1) << 62;
@@ -484,6 +598,33 @@ int dsq_gemv_grouped(int type, const void *w, int64_t G, int64_t N, int64_t K, c
                                              1, 0, K, xq, xd, xs, nullptr, as_stream(stream));
   return run_gemv("dsq_gemv_grouped", type, Seg{static_cast<const uint8_t *>(w), y, G * N}, Seg{nullptr, nullptr, 0}, N,
                   G, K, xq, xd, xs, nullptr, as_stream(stream));
+}
+
+int dsq_gemv_f32(int type, const void *w, int64_t N, int64_t K, const float *x, float *y, void *stream) {
+  using namespace dsq;
+  return run_gemv("dsq_gemv_f32", type, Seg{static_cast<const uint8_t *>(w), y, N}, Seg{nullptr, nullptr, 0},
+                  kOneGroup, 1, K, nullptr, nullptr, nullptr, nullptr, as_stream(stream), x);
+}
+
+int dsq_gemv_paired_f32(int type, const void *w0, int64_t N0, const void *w1, int64_t N1, int64_t K, const float *x,
+                        float *y0, float *y1, void *stream) {
+  using namespace dsq;
+  return run_gemv("dsq_gemv_paired_f32", type, Seg{static_cast<const uint8_t *>(w0), y0, N0},
+                  Seg{static_cast<const uint8_t *>(w1), y1, N1}, kOneGroup, 1, K, nullptr, nullptr, nullptr, nullptr,
+                  as_stream(stream), x);
+}
+
+int dsq_gemv_grouped_f32(int type, const void *w, int64_t G, int64_t N, int64_t K, const float *x, float *y,
+                         void *stream) {
+  using namespace dsq;
+  DSQ_REQUIRE(G >= 0 && N >= 0, DSQ_ERR_INVALID_ARG, "dsq_gemv_grouped_f32: G=%lld N=%lld", (long long)G,
+              (long long)N);
+  DSQ_REQUIRE(G <= (int64_t(1) << 20), DSQ_ERR_SHAPE, "dsq_gemv_grouped_f32: G out of range");
+  if (G == 0 || N == 0)
+    return run_gemv("dsq_gemv_grouped_f32", type, Seg{nullptr, nullptr, 0}, Seg{nullptr, nullptr, 0}, 1, 0, K,
+                    nullptr, nullptr, nullptr, nullptr, as_stream(stream), x);
+  return run_gemv("dsq_gemv_grouped_f32", type, Seg{static_cast<const uint8_t *>(w), y, G * N},
+                  Seg{nullptr, nullptr, 0}, N, G, K, nullptr, nullptr, nullptr, nullptr, as_stream(stream), x);
 }
 
 int dsq_test_block_sums(int type, const void *w, int64_t N, int64_t K, const int8_t *xq, const float *xd,

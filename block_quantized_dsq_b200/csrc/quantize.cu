@@ -7,6 +7,7 @@
 // All float steps are single IEEE operations with explicit rounding
 // (__fdiv_rn / __fmul_rn / __fadd_rn / __fsub_rn, no contraction) so the
 // codes and scales are bit-identical to the CPU oracle's.
+#include "act_q8.cuh"
 #include "dsq_host.h"
 
 namespace dsq {
@@ -14,11 +15,6 @@ namespace {
 
 // One 32-element block is handled by 8 consecutive lanes, 4 elements each
 // (one float4 load per lane; a warp covers 4 blocks = 512 contiguous bytes).
-__device__ __forceinline__ float q8_code(float x, float d) {
-  if (d == 0.0f) return 0.0f;
-  float v = roundf(__fdiv_rn(x, d));   // roundf: half away from zero
-  return fminf(fmaxf(v, -127.0f), 127.0f);
-}
 
 __global__ void __launch_bounds__(256) act_q8_kernel(const float4 *__restrict__ x, int64_t nblocks,
                                                      int8_t *__restrict__ xq, float *__restrict__ xd,
@@ -29,22 +25,11 @@ __global__ void __launch_bounds__(256) act_q8_kernel(const float4 *__restrict__ 
   const int64_t blk = tid >> 3;
   const int sub = threadIdx.x & 7;
   const bool live = blk < nblocks;
-  float4 v = live ? __ldg(&x[blk * 8 + sub]) : make_float4(0.f, 0.f, 0.f, 0.f);
-  float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-#pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float d = __fdiv_rn(amax, 127.0f);
-  const int q0 = static_cast<int>(q8_code(v.x, d));
-  const int q1 = static_cast<int>(q8_code(v.y, d));
-  const int q2 = static_cast<int>(q8_code(v.z, d));
-  const int q3 = static_cast<int>(q8_code(v.w, d));
-  int s = q0 + q1 + q2 + q3;
-#pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float4 v = live ? __ldg(&x[blk * 8 + sub]) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float d;
+  int s;
+  const uint32_t packed = q8_block_lanes(v, d, s);
   if (!live) return;
-  const uint32_t packed = (static_cast<uint32_t>(q0) & 0xffu) | ((static_cast<uint32_t>(q1) & 0xffu) << 8) |
-                          ((static_cast<uint32_t>(q2) & 0xffu) << 16) |
-                          ((static_cast<uint32_t>(q3) & 0xffu) << 24);
   reinterpret_cast<uint32_t *>(xq)[blk * 8 + sub] = packed;
   if (sub == 0) {
     xd[blk] = d;

@@ -130,6 +130,30 @@ int dsq_gemv_grouped(int type, const void *w, int64_t G, int64_t N, int64_t K,
                      float *y, void *stream);
 
 /*
+ * The three decode GEMV forms with the activation given in fp32: the same
+ * computation as dsq_quantize_act_q8 followed by dsq_gemv_q8_0 / _q4_k,
+ * dsq_gemv_paired or dsq_gemv_grouped (the activation prequantized to Q8
+ * per 32-block once and shared by every row that reads it [ds4-623 Summary;
+ * strix]), in one launch: each CTA quantizes the activation rows into its
+ * shared memory while its first weight copies are in flight.  The outputs
+ * equal those of the two-call path bit for bit; the quantized activation is
+ * not written out.
+ *   x: fp32 [rows][K], 16-byte aligned, rows = 1 (single, paired) or G
+ *      (grouped, group g's row at x + g*K).
+ * Requires K % 256 == 0 (both types) and rows*(K + 8*K/32) <= 65536 bytes
+ * (e.g. 8 rows of K = 4096, or one row of K <= 52428); otherwise
+ * DSQ_ERR_SHAPE and nothing is launched.  Other arguments, layouts and
+ * errors as in the corresponding two-call entry points.
+ */
+int dsq_gemv_f32(int type, const void *w, int64_t N, int64_t K, const float *x,
+                 float *y, void *stream);
+int dsq_gemv_paired_f32(int type, const void *w0, int64_t N0, const void *w1,
+                        int64_t N1, int64_t K, const float *x, float *y0,
+                        float *y1, void *stream);
+int dsq_gemv_grouped_f32(int type, const void *w, int64_t G, int64_t N,
+                         int64_t K, const float *x, float *y, void *stream);
+
+/*
  * Prefill dequantize-into-dense-GEMM [ds4-621 GB10 report: "dequant + GEMM
  * prefill path"]:  Y[M][N] = X[M][K] * deq(W)^T, X fp32 row-major, Y fp32
  * row-major.  Tensor-core contraction with 16-bit float operands and fp32
