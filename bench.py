@@ -160,11 +160,14 @@ def barrier(world):
 
 
 def max_over_ranks(world, v: float) -> float:
+    """The largest of the ranks' values (device times: the slowest rank sets
+    the job's time).  NCCL reduces a device tensor, gloo a host one."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
