@@ -126,6 +126,25 @@ __device__ __forceinline__ void piece_q8_0(Word word, uint32_t (&out)[32]) {
 // nib(i), i = 0..7, returns word i of qs[32P ..].  Each value is fp32
 // (d*sc)*q - dmin*m (one rounding: (d*sc)*q and dmin*m are exact), then
 // binary16 RNE.
+// Paired fp32 arithmetic (sm_100): two independent IEEE single operations per
+// instruction, lane 0 in the low 32 bits.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float lo_of(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_of(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t sub2_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+constexpr uint64_t kMagic2 = 0x4B0000004B000000ull;   // (2^23, 2^23)
+
 template <int P, class Nib>
 __device__ __forceinline__ void piece_q4_k(const uint4 &hdr, Nib nib, uint32_t (&out)[32]) {
   const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(hdr.x & 0xffffu)));
@@ -145,19 +164,21 @@ __device__ __forceinline__ void piece_q4_k(const uint4 &hdr, Nib nib, uint32_t (
     const int sh = 8 * (j & 3);
     const float a = __fmul_rn(d, static_cast<float>((scw >> sh) & 0xffu));
     const float nb = -__fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu));
+    const uint64_t a2 = pack2(a, a), nb2 = pack2(nb, nb);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t byte4 = nib(i);
       const uint32_t q4 = half_ ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
-      float v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // 0x4B000000 | q is the float 2^23 + q; subtracting 2^23 is exact
-        const float f = __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7540 + e));
-        v[e] = __fmaf_rn(__fsub_rn(f, 8388608.0f), a, nb);
+      for (int e = 0; e < 4; e += 2) {
+        // 0x4B000000 | q is the float 2^23 + q; subtracting 2^23 is exact.
+        // Two elements per paired-fp32 instruction, each rounded as its
+        // own __fsub_rn / __fmaf_rn would be.
+        const uint64_t f2 = pack2(__uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7540 + e)),
+                                  __uint_as_float(__byte_perm(q4, 0x4B000000u, 0x7540 + e + 1)));
+        const uint64_t v2 = fma2_rn(sub2_rn(f2, kMagic2), a2, nb2);
+        out[16 * half_ + 2 * i + e / 2] = h2_bits(__floats2half2_rn(lo_of(v2), hi_of(v2)));
       }
-      out[16 * half_ + 2 * i] = h2_bits(__floats2half2_rn(v[0], v[1]));
-      out[16 * half_ + 2 * i + 1] = h2_bits(__floats2half2_rn(v[2], v[3]));
     }
   }
 }
