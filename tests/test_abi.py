@@ -89,6 +89,15 @@ def test_host_side_validation(dsq):
     assert L.dsq_gemv_q8_0(None, 0, 256, None, None, None, None) == 0
     assert L.dsq_gemv_paired(8, None, 0, None, 0, 256, None, None, None, None, None, None) == 0
     assert L.dsq_quantize_act_q8(None, 0, 32, None, None, None, None) == 0
+    # the fp32-activation (fused) forms
+    assert L.dsq_gemv_f32(7, A16, 8, 256, A16, A16, None) == 1                 # unsupported type
+    assert L.dsq_gemv_f32(8, A16, 8, 96, A16, A16, None) == 3                  # K % 256 != 0: no fused form
+    assert L.dsq_gemv_f32(8, A16, 8, 256, A16 + 4, A16, None) == 2             # misaligned x
+    assert L.dsq_gemv_f32(8, A16, 8, 256, None, A16, None) == 1                # null x
+    assert L.dsq_gemv_grouped_f32(8, A16, 16, 8, 8192, A16, A16, None) == 3    # activations beyond 64 KB
+    assert L.dsq_gemv_grouped_f32(8, A16, -1, 8, 256, A16, A16, None) == 1
+    assert L.dsq_gemv_paired_f32(12, A16, 8, A16, 8, 256, A16 + 8, A16, A16, None) == 2
+    assert L.dsq_gemv_paired_f32(8, None, 0, None, 0, 256, None, None, None, None) == 0   # empty: no-op
     # nothing was launched
     assert dsq.dsq_launch_count() == before
     assert "multiple" in dsq.dsq_last_error() or dsq.dsq_last_error()
