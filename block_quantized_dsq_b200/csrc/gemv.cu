@@ -337,6 +337,20 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   const int sub = lane / G, j = lane % G;
   ActSlice act;
   int64_t cached = -1;  // (group * nunits + unit) currently in registers
+  {
+    // the slice of this lane's first (group, unit), loaded now so its
+    // latency overlaps the first weight slot's instead of following it
+    const int64_t row = r0 + static_cast<int64_t>(warp) * RPC + sub;
+    if (row < min(r0 + static_cast<int64_t>(warp) * RPC + RPC, r1) && j < a.nunits) {
+      int seg;
+      int64_t local;
+      locate(a, row, seg, local);
+      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
+      const int64_t e0 = group * a.K + static_cast<int64_t>(j) * 256;
+      load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
+      cached = group * a.nunits + j;
+    }
+  }
   int slot = 0;         // ring position kept incrementally (no division per chunk)
   uint32_t parity = 0;
   for (int64_t k = 0; k < mine; ++k) {
