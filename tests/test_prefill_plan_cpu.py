@@ -1,0 +1,65 @@
+"""Host logic of the prefill planner, through dsq_prefill_workspace_bytes (no
+GPU: the planner then assumes 148 SMs, i.e. 74 CTA pairs).
+
+The workspace holds the fp16 activations padded to whole token tiles, the
+per-row shifts, and the fp32 partials when K is split; K is split only while
+the pair tiles leave more than half the pairs idle.
+"""
+import pytest
+
+Q8, Q4 = 8, 12
+
+
+@pytest.fixture(scope="module")
+def dsq():
+    """libdsq without a device: the planner's default of 74 pairs.  With a
+    CUDA device present the planner asks the device instead, so skip."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present: the plan follows its SM count")
+    from block_quantized_dsq_b200 import build
+    build.build()
+    import block_quantized_dsq_b200 as dsq
+    return dsq
+
+
+def _align(v, a):
+    return (v + a - 1) // a * a
+
+
+def test_refusals_return_zero(dsq):
+    f = dsq.dsq_prefill_workspace_bytes
+    assert f(7, 256, 256, 4) == 0          # unsupported type
+    assert f(Q8, 256, 96, 4) == 0          # K % 256 != 0
+    assert f(Q4, 0, 256, 4) == 0           # N < 1
+    assert f(Q8, 256, 256, 0) == 0         # M < 1
+
+
+def test_large_problem_has_no_split(dsq):
+    # 8 token tiles (256 tokens each) x 32 weight tiles = 256 pair tiles:
+    # no split, workspace = fp16 activations + shifts
+    M, N, K = 2048, 8192, 4096
+    assert dsq.dsq_prefill_workspace_bytes(Q8, N, K, M) == M * K * 2 + _align(M * 4, 1024)
+
+
+def test_small_problem_splits_k_and_holds_partials(dsq):
+    # one 64-token tile x 2 weight tiles: K is split 16 ways (16 units of 256)
+    M, N, K = 64, 512, 4096
+    x16 = _align(M * K * 2, 1024)
+    got = dsq.dsq_prefill_workspace_bytes(Q8, N, K, M)
+    assert got == x16 + _align(M * 4, 1024) + 16 * M * N * 4
+
+
+def test_padding_to_whole_token_tiles(dsq):
+    # M = 300 -> two tiles of 256 tokens: 512 padded rows of fp16 activations
+    K = 1024
+    got = dsq.dsq_prefill_workspace_bytes(Q4, 8192, K, 300)
+    assert got == 512 * K * 2 + _align(512 * 4, 1024)
+
+
+@pytest.mark.parametrize("qtype", [Q8, Q4])
+def test_workspace_grows_with_tokens_once_unsplit(dsq, qtype):
+    N, K = 8192, 4096
+    sizes = [dsq.dsq_prefill_workspace_bytes(qtype, N, K, M) for M in (512, 1024, 2048, 4096)]
+    assert all(a < b for a, b in zip(sizes, sizes[1:]))
+    assert all(s >= M * K * 2 for s, M in zip(sizes, (512, 1024, 2048, 4096)))
