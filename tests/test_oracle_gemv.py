@@ -7,6 +7,7 @@ float64/int64 matmuls, and closed forms on hand-built blocks.
 import numpy as np
 import pytest
 
+import oracle
 from block_quantized_dsq_b200 import synth
 
 
@@ -159,3 +160,77 @@ def test_paired_and_grouped_are_independent_gemvs(ref):
     xf = (xd.astype(np.float64).repeat(32, axis=1) * xq.astype(np.float64))
     want = np.einsum("gnk,gk->gn", wf, xf).reshape(-1)
     assert np.allclose(flat, want, rtol=1e-12, atol=1e-15)
+
+
+def _q4k_rows_const(N, K, d_f16, dmin_f16, sc, m, code):
+    """Hand-assembled Q4_K rows: one fp16 d / dmin, every (sc_j, m_j) equal,
+    every 4-bit code equal (scale field packed by the pinned setter)."""
+    nsb = K // 256
+    blk = np.zeros(144, np.uint8)
+    blk[0:2] = np.array([d_f16], np.uint16).view(np.uint8)
+    blk[2:4] = np.array([dmin_f16], np.uint16).view(np.uint8)
+    s = np.zeros(12, np.uint8)
+    for j in range(8):
+        oracle.q4k_set_scale_min(s, j, sc, m)
+    blk[4:16] = s
+    blk[16:] = (code | (code << 4)) & 0xFF
+    return np.tile(blk, (N, nsb))
+
+
+def test_absum_closed_forms_q8_0(ref):
+    """absum is the sum of the magnitudes of the block terms d_w * xd_b * isum_b.
+    Unit codes make isum_b = xs_b, so with block signs s_b and scale d:
+    y = d * sum_b s_b xd_b xs_b and absum = |d| * sum_b |xd_b xs_b|."""
+    K = 1024
+    nb = K // 32
+    xq, xd, xs = ref.quantize_act_q8(synth.activations(21, 1, K))
+    base = np.abs(xd[0].astype(np.float64) * xs[0].astype(np.float64))
+    signs = np.where(np.arange(nb) % 2 == 0, 1, -1)
+    rows = [(0x3C00, np.ones(K, int)),                       # d = 1, all +1
+            (0x3C00, np.repeat(signs, 32)),                  # alternating block signs
+            (0x4000, -np.ones(K, int))]                      # d = 2, all -1
+    w = np.concatenate([_q8_0_bytes(d, q[None, :]) for d, q in rows])
+    y, absum = ref.gemv(8, w, K, xq, xd, xs)
+    want_abs = np.array([base.sum(), base.sum(), 2.0 * base.sum()])
+    signed = xd[0].astype(np.float64) * xs[0].astype(np.float64)
+    want_y = np.array([signed.sum(), (signs * signed).sum(), -2.0 * signed.sum()])
+    assert np.allclose(absum, want_abs, rtol=1e-14, atol=0)
+    assert np.allclose(y, want_y, rtol=1e-12, atol=1e-12 * base.sum())
+    # the mixed-sign row cancels: |y| is well below the condition scale
+    assert abs(y[1]) < 0.5 * absum[1]
+
+
+def test_absum_counts_both_q4_k_terms(ref):
+    """Q4_K forms two products per sub-block, (d sc) xd isum and (dmin m) xd xs,
+    and absum adds both magnitudes.  With d = dmin = 1, sc = m = 1 and every
+    code 1 the weights dequantize to exactly 0, so y = 0 while each product
+    is xd_b xs_b: absum = 2 sum_b |xd_b xs_b|.  With codes 0 only the min
+    term is left: absum = m sum_b |xd_b xs_b|."""
+    K = 512
+    xq, xd, xs = ref.quantize_act_q8(synth.activations(22, 1, K))
+    base = float(np.sum(np.abs(xd[0].astype(np.float64) * xs[0].astype(np.float64))))
+    w_cancel = _q4k_rows_const(1, K, 0x3C00, 0x3C00, 1, 1, 1)
+    assert np.all(ref.dequantize(12, w_cancel, K) == 0.0)
+    y, absum = ref.gemv(12, w_cancel, K, xq, xd, xs)
+    assert y[0] == 0.0
+    assert abs(absum[0] - 2.0 * base) <= 1e-14 * base
+    w_min = _q4k_rows_const(1, K, 0x3C00, 0x3C00, 5, 3, 0)
+    y, absum = ref.gemv(12, w_min, K, xq, xd, xs)
+    assert abs(absum[0] - 3.0 * base) <= 1e-14 * base
+    signed = float(np.sum(xd[0].astype(np.float64) * xs[0].astype(np.float64)))
+    assert abs(y[0] + 3.0 * signed) <= 1e-13 * base
+
+
+@pytest.mark.parametrize("qtype", [8, 12])
+def test_absum_bounds_the_result(ref, qtype):
+    """Triangle inequality on seeded data: |y_n| <= absum_n, and absum_n is at
+    least the magnitude of the largest single block contribution."""
+    N, K = 16, 1024
+    w = ref.quantize(qtype, synth.weights(23, N, K))
+    xq, xd, xs = ref.quantize_act_q8(synth.activations(24, 1, K))
+    y, absum = ref.gemv(qtype, w, K, xq, xd, xs)
+    assert np.all(np.abs(y) <= absum * (1 + 1e-14))
+    wf = ref.dequantize(qtype, w, K).astype(np.float64)
+    xf = xd[0].astype(np.float64).repeat(32) * xq[0].astype(np.float64)
+    per_block = np.abs((wf * xf).reshape(N, K // 32, 32).sum(-1)).max(-1)
+    assert np.all(absum >= per_block * (1 - 1e-6))
