@@ -428,8 +428,11 @@ int dsqref_row_shift(const float *row, int64_t K)
     int e;
     frexpf(amax, &e);            /* amax in [2^(e-1), 2^e) */
     int s = 15 - e;              /* amax * 2^s in [2^14, 2^15) */
-    if (s > 64) s = 64;
-    if (s < -64) s = -64;
+    /* 2^s and 2^-s must both be normal fp32 numbers with an exponent field
+     * in [1, 254]: s in [-113, 126].  -113 is reached by rows near FLT_MAX
+     * (e = 128), so every row with amax >= 2^-112 lands in the binade. */
+    if (s > 126) s = 126;
+    if (s < -113) s = -113;
     return s;
 }
 

@@ -100,7 +100,9 @@ void dsqref_prefill_f64(int type, const uint8_t *w, int64_t N, int64_t K,
 
 /* Per-row power-of-two shift used before rounding activations to a 16-bit
  * float: the smallest-magnitude choice that puts the row's largest |x| in
- * [2^14, 2^15); 0 for an all-zero row; clamped to [-64, 64]. */
+ * [2^14, 2^15); 0 for an all-zero row; clamped to [-113, 126], so every
+ * finite row whose largest magnitude is at least 2^-112 lands in that
+ * binade and smaller rows are scaled by 2^126. */
 int dsqref_row_shift(const float *row, int64_t K);
 
 /* Operand-rounded reference: the same sum with x -> r(x * 2^s_m) and

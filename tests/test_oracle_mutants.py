@@ -39,6 +39,12 @@ MUTANTS = {
     "prefill_transposed_output": ("            y[m * N + n] = acc;\n", "            y[n * M + m] = acc;\n"),
     "prefill_shift_not_undone": ("y[m * N + n] = ldexp(acc, -shift[m]);", "y[m * N + n] = acc;"),
     "q4k_quantizer_no_zero_in_range": ("float lo = 0.0f, hi = xs[32 * j];", "float lo = xs[32 * j], hi = xs[32 * j];"),
+    # the condition scale behind the GEMV tolerance's denominator floor
+    "absum_min_term_dropped": ("mag += fabs(t1) + fabs(t2);", "mag += fabs(t1);"),
+    "absum_of_difference": ("mag += fabs(t1) + fabs(t2);", "mag += fabs(t1 - t2);"),
+    "absum_doubled": ("                mag += fabs(t);\n", "                mag += 2.0 * fabs(t);\n"),
+    "absum_is_abs_of_sum": ("if (absum) absum[n] = mag;", "if (absum) absum[n] = fabs(acc);"),
+    "row_shift_narrow_clamp": ("if (s < -113) s = -113;", "if (s < -64) s = -64;"),
 }
 
 

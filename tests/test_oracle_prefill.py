@@ -40,8 +40,24 @@ def test_row_shift_places_row_max_in_binade_14(ref):
         amax = float(np.abs(row).max()) * 2.0 ** s
         assert 2.0 ** 14 <= amax < 2.0 ** 15, (e, s)
     assert ref.row_shift(np.zeros(64, np.float32)) == 0
-    assert ref.row_shift(np.array([1e-38, 0], np.float32)) == 64   # clamped
-    assert ref.row_shift(np.array([3e38, 0], np.float32)) == -64   # clamped
+
+
+def test_row_shift_covers_every_finite_binade(ref):
+    """Every finite row with max |x| >= 2^-112 lands in [2^14, 2^15) -- up to
+    FLT_MAX -- and the shift stays where 2^s and 2^-s are normal fp32."""
+    fmax = float(np.finfo(np.float32).max)
+    for e in range(-111, 129):
+        for frac in (0.5, 0.75, 0.999):
+            v = np.float32(min(frac * 2.0 ** e, fmax))
+            s = ref.row_shift(np.array([v, -v / 3, 0], np.float32))
+            assert 2.0 ** 14 <= float(v) * 2.0 ** s < 2.0 ** 15, (e, frac, s)
+            assert -113 <= s <= 126
+    assert ref.row_shift(np.array([fmax, 1.0], np.float32)) == -113
+    assert ref.row_shift(np.array([-fmax], np.float32)) == -113
+    # below 2^-112 the shift stops at 126 (2^-126 is the smallest normal scale)
+    tiny = np.float32(2.0 ** -120)
+    assert ref.row_shift(np.array([tiny, 0], np.float32)) == 126
+    assert ref.row_shift(np.array([np.float32(1e-45)], np.float32)) == 126   # subnormal
 
 
 @pytest.mark.parametrize("op16", ["f16", "bf16"])
