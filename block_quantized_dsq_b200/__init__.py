@@ -27,7 +27,7 @@ DSQ_Q4_K = 12
 
 STATUS = {0: "DSQ_OK", 1: "DSQ_ERR_INVALID_ARG", 2: "DSQ_ERR_ALIGNMENT", 3: "DSQ_ERR_SHAPE",
           4: "DSQ_ERR_UNSUPPORTED_DEVICE", 5: "DSQ_ERR_WORKSPACE", 6: "DSQ_ERR_LAUNCH",
-          7: "DSQ_ERR_TIMEOUT", 8: "DSQ_ERR_CUDA"}
+          7: "DSQ_ERR_TIMEOUT", 8: "DSQ_ERR_CUDA", 9: "DSQ_ERR_RANGE"}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsq.so")
 

@@ -5,6 +5,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/dsq_test.h"
 #include "dsq_host.h"
 
@@ -19,16 +21,56 @@ thread_local char t_error[512] = "no error";
 std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_limit_ns{1000ull * 1000ull * 1000ull};
 
-constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
 struct DevState {
-  bool checked = false;
+  uint64_t ctx = 0;   // context the entries below belong to (0: none yet)
   int ok = DSQ_ERR_UNSUPPORTED_DEVICE;
   uint32_t *status = nullptr;
   int sms = 0;
 };
 DevState g_dev[kMaxDevices];
+
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_ctx_fns_once;
+
+void load_ctx_fns() {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  p = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+}
 }  // namespace
+
+int current_context(int *device, uint64_t *ctx_id) {
+  cudaError_t e = cudaGetDevice(device);
+  if (e != cudaSuccess) return fail(DSQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (*device < 0 || *device >= kMaxDevices) return fail(DSQ_ERR_UNSUPPORTED_DEVICE, "device %d", *device);
+  std::call_once(g_ctx_fns_once, load_ctx_fns);
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr)
+    return fail(DSQ_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId are not available from the driver");
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    CUcontext c = nullptr;
+    if (g_ctx_current(&c) != CUDA_SUCCESS) return fail(DSQ_ERR_CUDA, "cuCtxGetCurrent failed");
+    if (c != nullptr) {
+      unsigned long long id = 0;
+      if (g_ctx_id(c, &id) != CUDA_SUCCESS) return fail(DSQ_ERR_CUDA, "cuCtxGetId failed");
+      *ctx_id = static_cast<uint64_t>(id) + 1;   // never 0
+      return DSQ_OK;
+    }
+    // No context is current on this thread yet: the runtime binds the
+    // device's primary context on its first call that needs one.
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return fail(DSQ_ERR_CUDA, "cudaGetSymbolAddress(status): %s", cudaGetErrorString(e));
+  }
+  return fail(DSQ_ERR_CUDA, "no CUDA context is current");
+}
 
 int fail(int code, const char *fmt, ...) {
   va_list ap;
@@ -40,30 +82,34 @@ int fail(int code, const char *fmt, ...) {
 
 int device_ready(uint32_t **status_word, int *num_sms) {
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(DSQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return fail(DSQ_ERR_UNSUPPORTED_DEVICE, "device %d", dev);
+  uint64_t ctx = 0;
+  int rc = current_context(&dev, &ctx);
+  if (rc != DSQ_OK) return rc;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DevState &s = g_dev[dev];
-  if (!s.checked) {
-    s.checked = true;
+  if (s.ctx != ctx) {
+    // First call in this context (a new process, a cudaDeviceReset, or a
+    // context the caller made current): device addresses from another
+    // context are not valid here, so look everything up again.
     int major = 0, minor = 0, sms = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    s.status = nullptr;
     if (major != 10 || minor != 0) {
       s.ok = DSQ_ERR_UNSUPPORTED_DEVICE;
     } else {
       void *p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_status_word);
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
       if (e != cudaSuccess) {
-        s.checked = false;
+        s.ctx = 0;
         return fail(DSQ_ERR_CUDA, "cudaGetSymbolAddress(status): %s", cudaGetErrorString(e));
       }
       s.status = static_cast<uint32_t *>(p);
       s.sms = sms;
       s.ok = DSQ_OK;
     }
+    s.ctx = ctx;
   }
   if (s.ok != DSQ_OK)
     return fail(s.ok, "device %d is not a compute capability 10.0 (B200) device", dev);
@@ -84,25 +130,27 @@ int wait_ctl(WaitCtl *ctl, int *num_sms) {
 int set_smem_once(const void *kernel, int bytes, const char *what) {
   struct Entry {
     const void *k;
-    int dev;
+    uint64_t ctx;   // the attribute belongs to the context it was set in
     int bytes;
   };
   static std::mutex mu;
   static Entry done[256];
   static int n_done = 0;
   int dev = 0;
-  cudaGetDevice(&dev);
+  uint64_t ctx = 0;
+  const int rc = current_context(&dev, &ctx);
+  if (rc != DSQ_OK) return rc;
   std::lock_guard<std::mutex> lk(mu);
   for (int i = 0; i < n_done; ++i)
-    if (done[i].k == kernel && done[i].dev == dev && done[i].bytes >= bytes) return DSQ_OK;
+    if (done[i].k == kernel && done[i].ctx == ctx && done[i].bytes >= bytes) return DSQ_OK;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: shared-memory attribute: %s", what, cudaGetErrorString(e));
   for (int i = 0; i < n_done; ++i)
-    if (done[i].k == kernel && done[i].dev == dev) {
+    if (done[i].k == kernel && done[i].ctx == ctx) {
       done[i].bytes = bytes;
       return DSQ_OK;
     }
-  if (n_done < 256) done[n_done++] = Entry{kernel, dev, bytes};
+  if (n_done < 256) done[n_done++] = Entry{kernel, ctx, bytes};
   return DSQ_OK;
 }
 
@@ -137,6 +185,11 @@ int dsq_device_status(void *stream) {
   if (e != cudaSuccess) return dsq::fail(DSQ_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
   if (v & dsq::kStatusTimeout)
     return dsq::fail(DSQ_ERR_TIMEOUT, "a bounded device wait expired (status word 0x%x)", v);
+  if (v & dsq::kStatusRange)
+    return dsq::fail(DSQ_ERR_RANGE,
+                     "a prefill weight block admits dequantized values outside the binary16 range "
+                     "(status word 0x%x); the outputs that read it are inf or NaN",
+                     v);
   return DSQ_OK;
 }
 

@@ -12,7 +12,10 @@
 namespace dsq {
 
 // Bits of the device status word.
-enum : uint32_t { kStatusTimeout = 1u };
+enum : uint32_t {
+  kStatusTimeout = 1u,   // a bounded wait expired
+  kStatusRange = 2u      // a prefill weight block admits values outside binary16
+};
 
 // Arguments every pipelined kernel receives for its bounded waits.
 struct WaitCtl {

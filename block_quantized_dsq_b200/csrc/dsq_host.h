@@ -16,8 +16,16 @@ namespace dsq {
 // Records a message for dsq_last_error() and returns `code`.
 int fail(int code, const char *fmt, ...);
 
-// Checks the current device once (compute capability 10.0) and returns its
-// status-word pointer and SM count through the out-parameters.
+constexpr int kMaxDevices = 64;
+
+// The current device and a process-unique id of the CUDA context current on
+// this thread (never reused, never 0).  Caches of device addresses or
+// per-context settings are keyed by this id, so none outlives its context
+// (cudaDeviceReset, or a driver context the caller made current).
+int current_context(int *device, uint64_t *ctx_id);
+
+// Checks the current device once per context (compute capability 10.0) and
+// returns its status-word pointer and SM count through the out-parameters.
 int device_ready(uint32_t **status_word, int *num_sms);
 
 // Wait control for kernels launched now (status word + current limit).
@@ -26,8 +34,8 @@ int wait_ctl(WaitCtl *ctl, int *num_sms);
 // After a launch: maps a launch error to DSQ_ERR_LAUNCH and counts launches.
 int after_launch(const char *what, int n_kernels = 1);
 
-// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
-// the first call on a device configures it; later calls (for example inside
+// Raises a kernel's dynamic shared-memory limit once per (kernel, context):
+// the first call in a context configures it; later calls (for example inside
 // a CUDA graph capture) only launch.
 int set_smem_once(const void *kernel, int bytes, const char *what);
 

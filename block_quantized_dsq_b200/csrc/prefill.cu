@@ -216,6 +216,56 @@ __device__ __forceinline__ void dequant_pair_piece(const PairRegs<TYPE> &r, uint
   }
 }
 
+// Range guard of the binary16 weight operand: false when a block this thread
+// dequantizes for stage pair J admits a value of magnitude >= 65520, which
+// rounds to +-inf in binary16.  Q8_0 (blocks 4J .. 4J+3 of the unit): |d| *
+// 127 >= 65520, i.e. |d| >= 516 (binary16 bits 0x6008), or a non-finite d.
+// Q4_K (sub-blocks 4J .. 4J+3): the dequantized value is a line in the code
+// q, so its extremes are the codes 0 and 15: -dmin*m and 15*(d*sc) - dmin*m,
+// formed in fp32 exactly as the converter forms them.  A cheap bound on the
+// whole super-block (|d|*63*15 + |dmin|*63 < 65520) settles almost every
+// block before the per-sub-block test.
+template <int TYPE, int J>
+__device__ __forceinline__ bool pair_in_range(const PairRegs<TYPE> &r) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+    uint32_t worst = 0;
+#pragma unroll
+    for (int I = 0; I < 2; ++I) {
+      const int o = 17 * (2 * J + I) - 32 * J;   // first word of piece 2J + I
+      const uint32_t d0 = word4(r.v[o >> 2], o & 3) & 0x7fffu;
+      const uint32_t d1 = (word4(r.v[(o + 8) >> 2], (o + 8) & 3) >> 16) & 0x7fffu;
+      worst = max(worst, max(d0, d1));
+    }
+    return worst < 0x6008u;
+  } else {
+    const float d = fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x & 0xffffu))));
+    const float dmin = fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x >> 16))));
+    if (__fadd_rn(__fmul_rn(d, 945.0f), __fmul_rn(dmin, 63.0f)) < 65520.0f) return true;
+    const float ds = __half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x & 0xffffu)));
+    const float dm = __half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x >> 16)));
+    bool ok = true;
+#pragma unroll
+    for (int j = 4 * J; j < 4 * J + 4; ++j) {
+      uint32_t scw, mw;
+      if (j < 4) {
+        scw = r.hdr.y & 0x3f3f3f3fu;
+        mw = r.hdr.z & 0x3f3f3f3fu;
+      } else {
+        scw = (r.hdr.w & 0x0f0f0f0fu) | ((r.hdr.y >> 2) & 0x30303030u);
+        mw = ((r.hdr.w >> 4) & 0x0f0f0f0fu) | ((r.hdr.z >> 2) & 0x30303030u);
+      }
+      const int sh = 8 * (j & 3);
+      const float a = __fmul_rn(ds, static_cast<float>((scw >> sh) & 0xffu));
+      const float b = __fmul_rn(dm, static_cast<float>((mw >> sh) & 0xffu));
+      const float v15 = __fmaf_rn(15.0f, a, -b);
+      ok = ok && fabsf(b) < 65520.0f && fabsf(v15) < 65520.0f;
+    }
+    return ok;
+  }
+}
+
+__device__ __forceinline__ void record_range(uint32_t *status) { atomicOr(status, kStatusRange); }
+
 // ------------------------------------------------------------------ GEMM ---
 // TMEM map of each CTA (512 columns x 128 lanes): [0, tn) the fp32
 // accumulators (lane = weight row of this CTA, column = token of the pair
@@ -330,6 +380,7 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
       load_pair<TYPE, J>(r, unit);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.rempty[rs]);
+      if (!pair_in_range<TYPE, J>(r)) record_range(a.wait.status);
       if (++rs == SR) {
         rs = 0;
         rpar ^= 1u;
@@ -581,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 8; ++c) {
         const int64_t m = m0 + 32 * c + lane;
         const int sft = (c < nchunks && m < a.M) ? __ldg(a.shift + m) : 0;
-        my_scale[c] = __int_as_float((127 - sft) << 23);   // s in [-64, 64]
+        my_scale[c] = __int_as_float((127 - sft) << 23);   // s in [-113, 126]: a normal 2^-s
       }
       const bool got = wait_or_abort(s, s.accfull, static_cast<uint32_t>(i & 1), a.wait, 256);
       if (__any_sync(0xffffffffu, !got)) break;
@@ -626,8 +677,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // --------------------------------------------------- activation rounding --
 // One CTA per activation row: row max -> shift s (max |x| * 2^s in
-// [2^14, 2^15), 0 for a zero row, clamped to [-64, 64]) -> binary16 RNE of
-// x * 2^s (an exact scaling unless the product is an fp32 subnormal).
+// [2^14, 2^15), 0 for a zero row, clamped to [-113, 126] so that 2^s and
+// 2^-s are both normal fp32: every finite row with max |x| >= 2^-112 lands in
+// the binade, up to FLT_MAX) -> binary16 RNE of x * 2^s (an exact scaling
+// unless the product is an fp32 subnormal, far below binary16's range).
 // BLOCKED = true writes the tile-major layout the MMA reads, so the
 // activations of one token tile for one 256-element unit of K are a single
 // contiguous block (one bulk copy): for token tile mt = m / tn, unit ub and
@@ -677,7 +730,7 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__
   if (amax > 0.0f && !isinf(amax)) {
     int e;
     frexpf(amax, &e);
-    s = min(64, max(-64, 15 - e));
+    s = min(126, max(-113, 15 - e));
   }
   const float scale = __int_as_float((127 + s) << 23);
   if (threadIdx.x == 0) shift[m] = s;
@@ -719,9 +772,10 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
 // same device functions as the GEMM's converter warps (one thread per
 // 256-element unit of a row, both stage pairs).
 template <int TYPE, int J>
-__device__ __forceinline__ void pair_to_f16(const uint4 *unit, uint16_t *dst) {
+__device__ __forceinline__ void pair_to_f16(const uint4 *unit, uint16_t *dst, uint32_t *status) {
   PairRegs<TYPE> r;
   load_pair<TYPE, J>(r, unit);
+  if (!pair_in_range<TYPE, J>(r)) record_range(status);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     uint32_t v[32];
@@ -735,15 +789,16 @@ __device__ __forceinline__ void pair_to_f16(const uint4 *unit, uint16_t *dst) {
 
 template <int TYPE>
 __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict__ w, int64_t N, int64_t K,
-                                                       int64_t row_bytes, uint16_t *__restrict__ w16) {
+                                                       int64_t row_bytes, uint16_t *__restrict__ w16,
+                                                       uint32_t *status) {
   const int64_t units = K / 256;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= N * units) return;
   const int64_t n = idx / units, u = idx % units;
   const uint4 *unit = reinterpret_cast<const uint4 *>(w + n * row_bytes + u * unit_bytes<TYPE>());
   uint16_t *dst = w16 + n * K + u * 256;
-  pair_to_f16<TYPE, 0>(unit, dst);
-  pair_to_f16<TYPE, 1>(unit, dst);
+  pair_to_f16<TYPE, 0>(unit, dst, status);
+  pair_to_f16<TYPE, 1>(unit, dst, status);
 }
 
 // ------------------------------------------------------------------- host --
@@ -779,17 +834,19 @@ cudaError_t launch_pair(const CUtensorMap &map_w, const PrefillArgs &args, unsig
 }
 
 // How many CTA pairs of the GEMM kernel can be resident at once (clusters
-// of 2 need two SMs of one GPC); cached per device, type and smem size.
-int resident_pairs(int type, size_t smem, int sms) {
+// of 2 need two SMs of one GPC).  The shared-memory size is a function of
+// (type, tn), so the answer is cached per device, type and tn (tn = 32 ..
+// 256 in steps of 32): after the first call of each shape no call asks the
+// runtime again.
+int resident_pairs(int type, int tn, size_t smem, int sms) {
   static std::mutex mu;
-  static int cache[64][2][4] = {};
-  static size_t cache_smem[64][2][4] = {};
+  static int cache[kMaxDevices][2][8] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return sms / 2;
   const int ti = type == DSQ_Q8_0 ? 0 : 1;
+  const int ni = tn / 32 - 1;   // 0..7
   std::lock_guard<std::mutex> lk(mu);
-  for (int i = 0; i < 4; ++i)
-    if (cache[dev][ti][i] > 0 && cache_smem[dev][ti][i] == smem) return cache[dev][ti][i];
+  if (cache[dev][ti][ni] > 0) return cache[dev][ti][ni];
   const void *kern = type == DSQ_Q8_0 ? reinterpret_cast<const void *>(prefill_kernel<DSQ_Q8_0>)
                                       : reinterpret_cast<const void *>(prefill_kernel<DSQ_Q4_K>);
   if (set_smem_once(kern, static_cast<int>(smem), "prefill") != DSQ_OK) return sms / 2;
@@ -810,12 +867,7 @@ int resident_pairs(int type, size_t smem, int sms) {
     n = sms / 2;
   }
   if (n > sms / 2) n = sms / 2;
-  for (int i = 0; i < 4; ++i)
-    if (cache[dev][ti][i] == 0) {
-      cache[dev][ti][i] = n;
-      cache_smem[dev][ti][i] = smem;
-      break;
-    }
+  cache[dev][ti][ni] = n;
   return n;
 }
 
@@ -845,7 +897,7 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   p.slots_raw = static_cast<int>((kSmemLimit - fixed - p.slots * slot_b) / raw_bytes);
   if (p.slots_raw > 4) p.slots_raw = 4;
   p.smem = 1024 + p.slots * slot_b + p.slots_raw * raw_bytes + barrier_bytes(p.slots, p.slots_raw);
-  if (pairs < 0) pairs = resident_pairs(type, p.smem, sms);
+  if (pairs < 0) pairs = resident_pairs(type, p.tn, p.smem, sms);
   const int64_t tiles = p.tiles_m * p.tiles_n;
   // split K only when the tiles leave more than half the pairs idle
   p.splits = 1;
@@ -995,7 +1047,8 @@ extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int
   DSQ_REQUIRE(x16 && shift && w16, DSQ_ERR_INVALID_ARG, "dsq_test_prefill_operands: null output");
   DSQ_REQUIRE(aligned(x16, 16) && aligned(w16, 16) && aligned(shift, 4), DSQ_ERR_ALIGNMENT,
               "dsq_test_prefill_operands: output alignment");
-  rc = device_ready(nullptr, nullptr);
+  uint32_t *status = nullptr;
+  rc = device_ready(&status, nullptr);
   if (rc != DSQ_OK) return rc;
   cudaStream_t st = as_stream(stream);
   x_to_f16_kernel<false><<<static_cast<unsigned>(M), 256, 0, st>>>(x, M, K, M, reinterpret_cast<__half *>(x16), shift);
@@ -1005,9 +1058,9 @@ extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int
   const unsigned grid = static_cast<unsigned>((work + 127) / 128);
   const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
   if (type == DSQ_Q8_0)
-    w_to_f16_kernel<DSQ_Q8_0><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16);
+    w_to_f16_kernel<DSQ_Q8_0><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16, status);
   else
-    w_to_f16_kernel<DSQ_Q4_K><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16);
+    w_to_f16_kernel<DSQ_Q4_K><<<grid, 128, 0, st>>>(static_cast<const uint8_t *>(w), N, K, rb, w16, status);
   return after_launch("dsq_test_prefill_operands: w");
 }
 
@@ -1022,37 +1075,52 @@ static __device__ __align__(256) uint8_t g_prefill_scratch[DSQ_PREFILL_NOALLOC_S
 namespace dsq {
 namespace {
 std::mutex g_scratch_mu;
-void *g_scratch_addr[64] = {};   // device address of g_prefill_scratch, per device
+// Device address of g_prefill_scratch, per device, with the id of the CUDA
+// context it was looked up in: a new context (cudaDeviceReset, or a driver
+// context the caller made current) maps the array elsewhere, so the address
+// is looked up again once in it.
+struct ScratchAddr {
+  uint64_t ctx = 0;
+  void *addr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 }  // namespace
 }  // namespace dsq
 
 extern "C" int dsq_gemm_prefill_noalloc(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M,
                                         float *y, void *stream) {
   using namespace dsq;
+  // the argument checks of dsq_gemm_prefill come first, so a bad argument is
+  // named as such even when the problem would also be too large
+  int rc = validate("dsq_gemm_prefill_noalloc", type, w, N, K, x, M);
+  if (rc != DSQ_OK) return rc;
+  DSQ_REQUIRE(y != nullptr, DSQ_ERR_INVALID_ARG, "dsq_gemm_prefill_noalloc: null output");
+  DSQ_REQUIRE(aligned(y, 16), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill_noalloc: y must be 16-byte aligned");
   const size_t need = dsq_prefill_workspace_bytes(type, N, K, M);
-  if (need == 0)  // invalid type or shape: let the regular entry point name it
-    return dsq_gemm_prefill(type, w, N, K, x, M, y, nullptr, 0, stream);
   DSQ_REQUIRE(need <= DSQ_PREFILL_NOALLOC_SCRATCH_BYTES, DSQ_ERR_WORKSPACE,
               "dsq_gemm_prefill_noalloc: this problem needs %zu bytes of scratch but the built-in scratch holds "
               "%llu bytes (M x K x 2 bytes of fp16 activations plus split-K partials must fit); use "
               "dsq_gemm_prefill with a caller-provided workspace",
               need, (unsigned long long)DSQ_PREFILL_NOALLOC_SCRATCH_BYTES);
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  DSQ_REQUIRE(e == cudaSuccess && dev >= 0 && dev < 64, DSQ_ERR_CUDA, "dsq_gemm_prefill_noalloc: no current device");
+  uint64_t ctx = 0;
+  rc = current_context(&dev, &ctx);
+  if (rc != DSQ_OK) return rc;
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-      // One-time set-up on this device (the device is current): the host
+    ScratchAddr &sa = g_scratch_addr[dev];
+    if (sa.ctx != ctx) {
+      // One-time set-up in this context (its device is current): the host
       // name of the array is only a stand-in, so fetch its device address.
       void *p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_prefill_scratch);
       DSQ_REQUIRE(e == cudaSuccess && p != nullptr, DSQ_ERR_CUDA,
                   "dsq_gemm_prefill_noalloc: cudaGetSymbolAddress of the scratch failed: %s", cudaGetErrorString(e));
-      g_scratch_addr[dev] = p;
+      sa.addr = p;
+      sa.ctx = ctx;
     }
-    scratch = g_scratch_addr[dev];
+    scratch = sa.addr;
   }
   return dsq_gemm_prefill(type, w, N, K, x, M, y, scratch, static_cast<size_t>(DSQ_PREFILL_NOALLOC_SCRATCH_BYTES),
                           stream);

@@ -64,7 +64,10 @@ typedef enum dsq_status {
     DSQ_ERR_WORKSPACE = 5,          /* workspace NULL or smaller than needed */
     DSQ_ERR_LAUNCH = 6,             /* the CUDA launch itself failed         */
     DSQ_ERR_TIMEOUT = 7,            /* a bounded device wait expired         */
-    DSQ_ERR_CUDA = 8                /* another CUDA runtime error            */
+    DSQ_ERR_CUDA = 8,               /* another CUDA runtime error            */
+    DSQ_ERR_RANGE = 9               /* reported by dsq_device_status: a
+                                       prefill weight block admits values
+                                       outside the binary16 range            */
 } dsq_status;
 
 typedef enum dsq_type { DSQ_Q8_0 = 8, DSQ_Q4_K = 12 } dsq_type;
@@ -160,13 +163,21 @@ int dsq_gemv_grouped_f32(int type, const void *w, int64_t G, int64_t N,
  * accumulation:
  *   - each X row m is scaled by an exact power of two 2^s_m chosen so its
  *     largest magnitude lies in [2^14, 2^15) (s_m = 0 for a zero row,
- *     clamped to [-64, 64]) and rounded to IEEE binary16 (RNE);
+ *     clamped to [-113, 126]: every finite row with max |x| >= 2^-112 lands
+ *     in that binade, up to FLT_MAX) and rounded to IEEE binary16 (RNE);
  *   - each weight element is dequantized in fp32 (Q8_0: d*q; Q4_K:
  *     (d*sc)*q - dmin*m) and rounded to binary16 (RNE);
  *   - the fp32 sum over K is scaled back by 2^-s_m.
  * Error vs the fp64 dequantized reference: relative L2 ~3e-4 on N(0,1)
- * activations and N(0, 0.02^2) weights (gate 2e-3).  Dequantized weights
- * must lie inside the binary16 range (|w| < 65504).
+ * activations and N(0, 0.02^2) weights (gate 2e-3).
+ * Weight range: dequantized weights must lie inside the binary16 range.  A
+ * block whose scales admit a value of magnitude >= 65520 -- a Q8_0 block
+ * with |d|*127 >= 65520, or a Q4_K sub-block whose code-0 or code-15 value
+ * (-dmin*m or 15*d*sc - dmin*m, in fp32) reaches 65520 -- makes the kernel
+ * record DSQ_ERR_RANGE in the device status word (read it with
+ * dsq_device_status); the outputs that read such a block are inf or NaN.
+ * Weights below 2^-14 in magnitude become binary16 subnormals (absolute
+ * spacing 2^-24) and keep less relative precision.
  * workspace: device scratch of at least dsq_prefill_workspace_bytes(...)
  * bytes, 256-byte aligned, used only for the duration of the call's kernels
  * on `stream`.  Requires K % 256 == 0 for both types, 1 <= M, N >= 1.
@@ -194,8 +205,10 @@ size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M);
  * those of dsq_gemm_prefill.  No call allocates or frees device memory.
  *
  * The first call on a device performs a one-time set-up (it looks up the
- * device address of the scratch array); make that first call before any
- * stream capture.  All calls on a device share the one scratch array, so
+ * device address of the scratch array in the current CUDA context; a new
+ * context -- after cudaDeviceReset, or a driver context the caller made
+ * current -- repeats it once); make that first call before any stream
+ * capture.  All calls on a device share the one scratch array, so
  * calls that may overlap on the GPU (different streams without ordering,
  * or concurrent host threads) race and must be serialized by the caller.
  * Nothing in the array needs to be cleared between calls: each call writes
@@ -218,8 +231,9 @@ int dsq_quantize_weights(int type, const float *x, int64_t N, int64_t K,
                          void *w, void *stream);
 
 /* Synchronizes `stream`, then returns and clears the device status word of
- * the current device: DSQ_OK, or DSQ_ERR_TIMEOUT if a bounded device wait
- * expired since the last read. */
+ * the current device: DSQ_OK; DSQ_ERR_TIMEOUT if a bounded device wait
+ * expired since the last read; else DSQ_ERR_RANGE if a prefill kernel met a
+ * weight block outside the binary16 range (see dsq_gemm_prefill). */
 int dsq_device_status(void *stream);
 
 /* Human-readable description of the last error on this host thread. */

@@ -98,6 +98,14 @@ def test_host_side_validation(dsq):
     assert L.dsq_gemv_grouped_f32(8, A16, -1, 8, 256, A16, A16, None) == 1
     assert L.dsq_gemv_paired_f32(12, A16, 8, A16, 8, 256, A16 + 8, A16, A16, None) == 2
     assert L.dsq_gemv_paired_f32(8, None, 0, None, 0, 256, None, None, None, None) == 0   # empty: no-op
+    # the allocation-free prefill names a bad argument before it looks at the
+    # scratch size, even for a problem too large for its scratch
+    big_m = 8192                                    # 8192 x 8192 x 2 B of fp16 activations > 32 MiB
+    assert L.dsq_gemm_prefill_noalloc(8, None, 256, 8192, A16, big_m, A16, None) == 1
+    assert L.dsq_gemm_prefill_noalloc(8, A16, 256, 8192, A16 + 4, big_m, A16, None) == 2
+    assert L.dsq_gemm_prefill_noalloc(8, A16, 256, 8192, A16, big_m, None, None) == 1
+    assert L.dsq_gemm_prefill_noalloc(8, A16, 256, 96, A16, 4, A16, None) == 3
+    assert L.dsq_gemm_prefill_noalloc(7, A16, 256, 256, A16, 4, A16, None) == 1
     # nothing was launched
     assert dsq.dsq_launch_count() == before
     assert "multiple" in dsq.dsq_last_error() or dsq.dsq_last_error()

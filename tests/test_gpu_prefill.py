@@ -100,3 +100,117 @@ def test_prefill_workspace_is_checked(dsq, ref):
     with pytest.raises(DsqError) as ei:
         dsq.dsq_gemm_prefill(8, to_dev(w), 128, 256, to_dev(x), 4, y, None, need)
     assert ei.value.status == 5
+
+
+def _operands_and_status(dsq, ref, qtype, w, K, x):
+    """The kernels' rounded operands and the device status they leave, with
+    the oracle's operands for the same inputs."""
+    N, M = w.shape[0], x.shape[0]
+    x16 = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    sh = torch.empty(M, dtype=torch.int32, device="cuda")
+    w16 = torch.empty((N, K), dtype=torch.int16, device="cuda")
+    assert dsq.dsq_device_status() == 0
+    dsq.dsq_test_prefill_operands(qtype, to_dev(w), N, K, to_dev(x), M, x16, sh, w16)
+    status = dsq.dsq_device_status()
+    got = (x16.cpu().numpy().view(np.uint16), sh.cpu().numpy(), w16.cpu().numpy().view(np.uint16))
+    x16_r, sh_r, w16_r = ref.prefill_operands(qtype, w, K, x, "f16")
+    return got, (x16_r, sh_r, w16_r), status
+
+
+@pytest.mark.parametrize("qtype", [8, 12])
+@pytest.mark.parametrize("sigma_scale", [5e-5, 1e-3])
+def test_prefill_operands_tiny_weights_and_extreme_rows(dsq, ref, qtype, sigma_scale):
+    """Weights of sigma 1e-6 and 2e-5 (binary16 subnormals, and values around
+    the smallest normal 2^-14) and activation rows at the ends of the shift
+    range: max |x| near FLT_MAX (shift -113), 2^-118 (shift clamped at 126),
+    fp32 subnormals.  The operand bits must still equal the oracle's."""
+    N, K, M = 96, 512, 6
+    w = ref.quantize(qtype, synth.weights(330, N, K) * np.float32(sigma_scale))
+    x = synth.activations(331, M, K)
+    x[0] *= np.float32(3.0e38 / np.abs(x[0]).max())
+    x[1] *= np.float32(2.0 ** -118 / np.abs(x[1]).max())
+    x[2] = (x[2] * np.float32(1e-40)).astype(np.float32)          # fp32 subnormals
+    x[3, ::2] = 0.0
+    x[4] = 0.0
+    got, want, status = _operands_and_status(dsq, ref, qtype, w, K, x)
+    assert status == 0
+    assert want[1][0] == -113 and want[1][1] == 126 and want[1][4] == 0
+    for g, r in zip(got, want):
+        assert np.array_equal(g, r)
+    # at least some weights landed in the binary16 subnormal range
+    if sigma_scale == 5e-5:
+        mag = want[2] & 0x7FFF
+        assert np.any((mag > 0) & (mag < 0x0400))
+
+
+def test_prefill_extreme_rows_parity(dsq, ref):
+    """Rows near FLT_MAX and near 2^-118 go through the whole GEMM: each row
+    within the rounded-reference tolerance of its own norm."""
+    qtype, N, K, M = 8, 256, 256, 40
+    w = ref.quantize(qtype, synth.weights(332, N, K))
+    x = synth.activations(333, M, K)
+    x[0] *= np.float32(1.0e37 / np.abs(x[0]).max())
+    x[1] *= np.float32(2.0 ** -118 / np.abs(x[1]).max())
+    x[2] *= np.float32(2.0 ** 100)
+    y = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    assert np.isfinite(y).all()
+    y_rounded = ref.prefill_rounded(qtype, w, K, x, "f16")
+    y64 = ref.prefill_f64(qtype, w, K, x)
+    for m in range(M):
+        assert rel_l2(y[m], y_rounded[m]) <= PREFILL_ROUNDED_TOL, m
+        assert rel_l2(y[m], y64[m]) <= PREFILL_TOL, m
+
+
+def _q8_0_row_with_block(ref, N, K, d_bits, code):
+    """Seeded Q8_0 rows; row 5's first block gets scale bits d_bits and
+    codes alternating +code / -code."""
+    w = ref.quantize(8, synth.weights(334, N, K))
+    blk = w[5, 0:34]
+    blk[0:2] = np.array([d_bits], np.uint16).view(np.uint8)
+    blk[2:] = np.array([code, -code] * 16, np.int8).view(np.uint8)
+    return w
+
+
+def _q4_k_row_with_subblock(ref, N, K, d_bits, dmin_bits, sc, m, codes):
+    """Seeded Q4_K rows; row 5's first super-block gets d / dmin bits, sub-block
+    0 the scale pair (sc, m) and the given codes, the others (0, 0)."""
+    w = ref.quantize(12, synth.weights(335, N, K))
+    blk = w[5, 0:144]
+    blk[0:2] = np.array([d_bits], np.uint16).view(np.uint8)
+    blk[2:4] = np.array([dmin_bits], np.uint16).view(np.uint8)
+    sc12 = np.zeros(12, np.uint8)
+    ref.q4k_set_scale_min(sc12, 0, sc, m)
+    blk[4:16] = sc12
+    blk[16:48] = (np.array(codes, np.uint8) & 0x0F) | (blk[16:48] & 0xF0)
+    return w
+
+
+RANGE_CASES = [
+    # (type, builder args, out of range?)
+    (8, (0x6007, 127), False),          # |d| = 515.5: 515.5 * 127 = 65468.5 -> 65472, finite
+    (8, (0x6008, 127), True),           # |d| = 516:   516 * 127 = 65532 -> inf
+    (8, (0xE008, 127), True),           # d = -516
+    (12, (0x5450, 0x0000, 63, 0, [15, 0] * 16), False),   # 15 * 69 * 63 = 65205 -> 65216, finite
+    (12, (0x5460, 0x0000, 63, 0, [15, 0] * 16), True),    # 15 * 70 * 63 = 66150 -> inf
+    (12, (0x0000, 0x6410, 0, 63, [0, 1] * 16), True),     # -dmin * m = -65520 -> -inf
+]
+
+
+@pytest.mark.parametrize("qtype,args,bad", RANGE_CASES)
+def test_prefill_weight_range_fails_closed(dsq, ref, qtype, args, bad):
+    """A weight block whose dequantized values leave the binary16 range makes
+    the kernels record DSQ_ERR_RANGE; a block just inside the bound does not.
+    Either way the operand bits equal the oracle's (inf where it overflows)."""
+    N, K, M = 128, 256, 8
+    w = _q8_0_row_with_block(ref, N, K, *args) if qtype == 8 else _q4_k_row_with_subblock(ref, N, K, *args)
+    x = synth.activations(336, M, K)
+    got, want, status = _operands_and_status(dsq, ref, qtype, w, K, x)
+    assert np.array_equal(got[2], want[2])
+    w16 = want[2]
+    has_inf = bool(np.any((w16 & 0x7FFF) == 0x7C00))
+    assert has_inf == bad
+    assert status == (9 if bad else 0)
+    y = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    assert dsq.dsq_device_status() == (9 if bad else 0)
+    assert np.isfinite(np.delete(y, 5, axis=1)).all()
+    assert np.isfinite(y[:, 5]).all() != bad
