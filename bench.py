@@ -189,6 +189,24 @@ def copies_for(nbytes: int, lo: int = 2) -> int:
     return max(lo, -(-3 * L2_BYTES // max(nbytes, 1)) + 1)
 
 
+def paired_copies() -> int:
+    """Weight copies the headline rotates over: past 3x L2, and the last call
+    of a step and the first of the next never read the same copy."""
+    R = copies_for(paired_bytes_per_call()["gemv"])
+    while (CALLS - 1) % R == 0:
+        R += 1
+    return R
+
+
+def bench_config(world: int) -> dict:
+    """The workload description both arms print."""
+    R = paired_copies()
+    return {"workload": WORKLOAD, "weights": "N(0,0.02^2) fp32 quantized to Q8_0, seeds 1/2",
+            "activations": "N(0,1) fp32, seeds 1000..1063, quantized to Q8 per call",
+            "l2": f"weights rotated over {R} copies ({R * paired_bytes_per_call()['gemv'] / 1e6:.0f} MB > 3x L2)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 PROFILE = False   # --profile: run each selected workload a few times, untimed
 
 
@@ -220,10 +238,13 @@ def time_calls(fn, n_calls: int, warmup: int = 5):
     return e0.elapsed_time(e1) / 1e3 / n_calls
 
 
-def time_graph(fn, calls_per_graph: int, replays: int = 5):
+def time_graph(fn, calls_per_graph: int, replays: int = 21):
     """Device time per call with the calls captured in a CUDA graph, so host
-    launch cost cannot hide in the figure (CUDA events around the replays)."""
+    launch cost cannot hide in the figure.  Each replay is bracketed by its
+    own CUDA events on the replay stream; returns the median per-call time
+    and sets LAST_STATS to {median, min, max, replays} in microseconds."""
     import torch
+    global LAST_STATS
     if PROFILE:
         return profile_calls(fn)
     side = torch.cuda.Stream()
@@ -238,17 +259,23 @@ def time_graph(fn, calls_per_graph: int, replays: int = 5):
         st = torch.cuda.current_stream().cuda_stream
         for i in range(calls_per_graph):
             fn(i, st)
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(replays):
+    for _ in range(3):
         g.replay()
-    e1.record()
     torch.cuda.synchronize()
-    t = e0.elapsed_time(e1) / 1e3 / (replays * calls_per_graph)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 1)]
+    ev[0].record()
+    for r in range(replays):
+        g.replay()
+        ev[r + 1].record()
+    torch.cuda.synchronize()
+    per_call = sorted(ev[r].elapsed_time(ev[r + 1]) / 1e3 / calls_per_graph for r in range(replays))
     del g
-    return t
+    LAST_STATS = {"median_us": round(statistics.median(per_call) * 1e6, 3), "min_us": round(per_call[0] * 1e6, 3),
+                  "max_us": round(per_call[-1] * 1e6, 3), "replays": replays, "calls_per_replay": calls_per_graph}
+    return statistics.median(per_call)
+
+
+LAST_STATS: dict = {}
 
 
 # ------------------------------------------------------------- the bench ---
@@ -268,9 +295,7 @@ def run_dsq(args, world, rank):
     W0 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w0"], N_PAIR, K_PAIR)
     W1 = quantized_weights(dsq, dsq.DSQ_Q8_0, seeds["w1"], N_PAIR, K_PAIR)
     bpc = paired_bytes_per_call()
-    R = copies_for(bpc["gemv"])
-    while (CALLS - 1) % R == 0:      # the last call of a step and the first of the
-        R += 1                       # next must not read the same weight copy
+    R = paired_copies()
     pairs = [(W0, W1)] + [(W0.clone(), W1.clone()) for _ in range(R - 1)]
     X_host = __import__("numpy").concatenate(
         [synth.activations(seeds["x_base"] + i, 1, K_PAIR) for i in range(CALLS)])
@@ -371,19 +396,20 @@ def run_dsq(args, world, rank):
     e2e_value = world * CALLS * bpc["total"] / e2e_t / 1e9
 
     # ---- the other rows of the path (each its own short timed loop)
-    rows = {}
+    rows, rows_clocks = {}, None
     if not args.skip_rows:
+        rs = ClockSampler(torch.cuda.current_device(), period=0.05)
+        rs.start()
         rows = measure_rows(dsq, L, stream, hbm_peak, bf16_peak,
                             only=set(args.rows.split(",")) if args.rows else None)
+        rs.stop()
+        rows_clocks = rs.summary()
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "weights": "N(0,0.02^2) fp32 quantized to Q8_0 on device, seeds 1/2",
-                   "activations": "N(0,1) fp32, seeds 1000..1063, quantized to Q8 per call",
-                   "l2": f"weights rotated over {R} copies ({R * bpc['gemv'] / 1e6:.0f} MB > 3x L2)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": bench_config(world),
         "us_per_call": round(ms_per_step * 1e3 / CALLS, 3),
         "hbm_frac": round(value / world / hbm_peak, 4),
         "timing": "CUDA graph of one step (64 x quantize + paired GEMV, programmatic launch) replayed "
@@ -401,22 +427,31 @@ def run_dsq(args, world, rank):
         "gpu_launches": int(launches),
         "clocks": sampler.summary(),
         "rows": rows,
+        "rows_clocks": rows_clocks,
+        "rows_timing": "each row: a CUDA graph of calls rotating over weight copies past 3x L2, replayed 21 "
+                       "times with CUDA events around every replay; median per call with min/max",
     }
     if rank == 0 and world == 1 and not args.skip_cpu:
         result["cpu_baseline"] = cpu_baseline(pairs[0], X_host, args.cpu_seconds)
+        result["cpu_oracle_rows"] = cpu_oracle_rows()
     return result
+
+
+PREFILL_SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048)
+NSWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
 
 
 def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
     """µs/call and GB/s (or TFLOP/s) for every other step of the path;
-    `only` restricts the run to the named rows."""
+    `only` restricts the run to the named rows (a row family such as
+    `prefill_sweep` or `gemv_nsweep` selects all of its points)."""
     import torch
 
     from block_quantized_dsq_b200 import synth
     rows = {}
 
     def want(name):
-        return only is None or name in only
+        return only is None or name in only or any(name.startswith(o + "_") for o in only)
 
     def act(seed, M, K):
         x = torch.from_numpy(synth.activations(seed, M, K)).cuda()
@@ -426,13 +461,24 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
         dsq.dsq_quantize_act_q8(x, M, K, xq, xd, xs)
         return x, xq, xd, xs
 
+    def stats_row(t, alg_bytes=None, flops=None):
+        """One row: median µs/call (with min/max over the replays) and the
+        rate of algorithmic bytes and/or flops against the measured peaks."""
+        r = {"us_per_call": round(t * 1e6, 3), **{k: v for k, v in LAST_STATS.items()}}
+        if alg_bytes is not None:
+            gbs = alg_bytes / t / 1e9
+            r.update({"GB/s": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes": alg_bytes})
+        if flops is not None:
+            tf = flops / t / 1e12
+            r.update({"TFLOP/s": round(tf, 1), "bf16_peak_frac": round(tf / bf16_peak, 4)})
+        return r
+
     # activation prequantization, one decode row of K = 4096
     if want("quantize_act_q8_1x4096"):
         x, xq, xd, xs = act(101, 1, 4096)
         px, pq, pd, ps = x.data_ptr(), xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
         t = time_graph(lambda i, st: L.dsq_quantize_act_q8(px, 1, 4096, pq, pd, ps, st), 500)
-        rows["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 3),
-                                          "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 2)}
+        rows["quantize_act_q8_1x4096"] = stats_row(t, 4096 * 4 + 4096 + 1024)
 
     def gemv_row(name, qtype, N, K, seed, xseed, G=1, fused=False):
         """fused: the *_f32 entry point (fp32 activation quantized in the
@@ -463,9 +509,7 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
             alg = nbytes + G * K * 4 + G * N * 4
         else:
             alg = nbytes + G * (K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1)) + G * N * 4
-        gbs = alg / t / 1e9
-        rows[name] = {"us_per_call": round(t * 1e6, 3), "GB/s": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4),
-                      "algorithmic_bytes": alg, "weight_copies": R}
+        rows[name] = {**stats_row(t, alg), "weight_copies": R}
         del ws
 
     seeds = synth.SEEDS
@@ -502,33 +546,91 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
         fn = lambda i, st: L.dsq_gemv_paired_f32(dsq.DSQ_Q8_0, pw[i % R][0], N_PAIR, pw[i % R][1], N_PAIR,  # noqa: E731
                                                  K_PAIR, px, py0, py1, st)
         t = time_graph(fn, R * max(1, 128 // R))
-        alg = nb2 + K_PAIR * 4 + 2 * N_PAIR * 4
-        gbs = alg / t / 1e9
-        rows["f32_paired_q8_0_2x8192x4096"] = {"us_per_call": round(t * 1e6, 3), "GB/s": round(gbs, 1),
-                                               "hbm_frac": round(gbs / hbm_peak, 4), "algorithmic_bytes": alg,
+        rows["f32_paired_q8_0_2x8192x4096"] = {**stats_row(t, nb2 + K_PAIR * 4 + 2 * N_PAIR * 4),
                                                "weight_copies": R}
         del keep, W0, W1
 
-    # prefill dequant-GEMM sweep
+    # decode GEMV N-sweep at K = 4096: the asymptotic HBM fraction once the
+    # launch and first-byte latency are amortised over more rows.  The rows
+    # of a 4096-row seeded matrix are repeated on the device (distinct
+    # addresses; the weight stream does not depend on the values).
     K = 4096
+    for qtype, tag in ((dsq.DSQ_Q8_0, "q8_0"), (dsq.DSQ_Q4_K, "q4_k")):
+        Ns = [N for N in NSWEEP_N if want(f"gemv_nsweep_{tag}_n{N}")]
+        if not Ns:
+            continue
+        base = quantized_weights(dsq, qtype, 600 + qtype, 4096, K)
+        x, xq, xd, xs = act(601, 1, K)
+        pq, pd, ps = xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
+        for N in Ns:
+            w = base.repeat((N + 4095) // 4096, 1)[:N].contiguous()
+            R = copies_for(w.numel())
+            ws = [w] + [w.clone() for _ in range(R - 1)]
+            ptrs = [c.data_ptr() for c in ws]
+            y = torch.empty(N, dtype=torch.float32, device="cuda")
+            py = y.data_ptr()
+            if qtype == dsq.DSQ_Q8_0:
+                fn = lambda i, st, ptrs=ptrs, R=R, N=N, py=py: L.dsq_gemv_q8_0(  # noqa: E731
+                    ptrs[i % R], N, K, pq, pd, py, st)
+            else:
+                fn = lambda i, st, ptrs=ptrs, R=R, N=N, py=py: L.dsq_gemv_q4_k(  # noqa: E731
+                    ptrs[i % R], N, K, pq, pd, ps, py, st)
+            t = time_graph(fn, R * max(1, 64 // R))
+            alg = w.numel() + K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1) + N * 4
+            rows[f"gemv_nsweep_{tag}_n{N}"] = {**stats_row(t, alg), "weight_copies": R}
+            del ws, w, y
+        del base
+
+    # prefill dequant-GEMM M sweep (1 .. 2048) for both weight types; for
+    # M <= 64 the same M tokens as M separate decode calls (quantize the M
+    # rows once, then one GEMV per token, each reading its weights from HBM)
     for qtype, N, tag in ((dsq.DSQ_Q4_K, 4096, "q4_k_n4096"), (dsq.DSQ_Q8_0, 8192, "q8_0_n8192")):
-        Ms = [M for M in (128, 512, 2048) if want(f"prefill_{tag}_m{M}")]
+        Ms = [M for M in PREFILL_SWEEP_M if want(f"prefill_{tag}_m{M}")]
         if not Ms:
             continue
         w = quantized_weights(dsq, qtype, seeds["prefill"]["w_q4_k" if qtype == dsq.DSQ_Q4_K else "w_q8_0"], N, K)
-        ws = [w, w.clone()]
+        wbytes = w.numel()
+        R = copies_for(wbytes)
+        ws = [w] + [w.clone() for _ in range(R - 1)]
+        pw = [c.data_ptr() for c in ws]
         for M in Ms:
             x = torch.from_numpy(synth.activations(seeds["prefill"]["x_base"] + M, M, K)).cuda()
             y = torch.empty((M, N), dtype=torch.float32, device="cuda")
             nb = dsq.dsq_prefill_workspace_bytes(qtype, N, K, M)
             wsp = torch.empty(nb, dtype=torch.uint8, device="cuda")
-            pw = [c.data_ptr() for c in ws]
             px, py, pws = x.data_ptr(), y.data_ptr(), wsp.data_ptr()
-            t = time_graph(lambda i, st: L.dsq_gemm_prefill(qtype, pw[i % 2], N, K, px, M, py, pws, nb, st), 10, 3)
-            tf = 2.0 * M * N * K / t / 1e12
-            rows[f"prefill_{tag}_m{M}"] = {"us_per_call": round(t * 1e6, 2), "TFLOP/s": round(tf, 1),
-                                           "bf16_peak_frac": round(tf / bf16_peak, 4)}
+            t = time_graph(lambda i, st: L.dsq_gemm_prefill(qtype, pw[i % R], N, K, px, M, py, pws, nb, st),
+                           R * max(1, 24 // R))
+            flops = 2.0 * M * N * K
+            alg = wbytes + 4 * M * K + 4 * M * N
+            bound_t = max(flops / (bf16_peak * 1e12), alg / (hbm_peak * 1e9))
+            row = {**stats_row(t, alg, flops), "weight_copies": R,
+                   "bound": "tensor" if flops / (bf16_peak * 1e12) >= alg / (hbm_peak * 1e9) else "hbm",
+                   "roofline_frac": round(bound_t / t, 4)}
+            if M <= 64:
+                xq = torch.empty((M, K), dtype=torch.int8, device="cuda")
+                xd = torch.empty((M, K // 32), dtype=torch.float32, device="cuda")
+                xs = torch.empty((M, K // 32), dtype=torch.int32, device="cuda")
+                pq, pd, ps = xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
+                rbq = K  # xq row stride (int8)
+                rbd = K // 32 * 4
+
+                def per_token(i, st, M=M, pq=pq, pd=pd, ps=ps, px=px, py=py):
+                    L.dsq_quantize_act_q8(px, M, K, pq, pd, ps, st)
+                    for m in range(M):
+                        wp = pw[(i * M + m) % R]
+                        if qtype == dsq.DSQ_Q8_0:
+                            L.dsq_gemv_q8_0(wp, N, K, pq + m * rbq, pd + m * rbd, py + m * N * 4, st)
+                        else:
+                            L.dsq_gemv_q4_k(wp, N, K, pq + m * rbq, pd + m * rbd, ps + m * rbd, py + m * N * 4,
+                                            st)
+                t2 = time_graph(per_token, max(1, 48 // M))
+                row["m_decode_calls_us"] = round(t2 * 1e6, 3)
+                row["m_decode_calls_stats"] = dict(LAST_STATS)
+                del xq, xd, xs
+            rows[f"prefill_{tag}_m{M}"] = row
             del x, y, wsp
+        del ws, w
     assert dsq.dsq_device_status() == 0
     return rows
 
@@ -588,6 +690,57 @@ def cpu_baseline(pair, X_host, budget_s: float):
             "cpu": platform.processor() or platform.machine(), "host_cores": os.cpu_count()}
 
 
+def cpu_oracle_rows(budget_s: float = 1.5) -> dict:
+    """The CPU oracle (single-threaded C, 1 core) per workload, each timed for
+    about budget_s seconds: activation quantize, the integer-form GEMV of the
+    three other decode workloads, and the fp64 prefill reference on a bounded
+    sample (256 weight rows x 128 tokens of the Q4_K N = 4096 workload)."""
+    import numpy as np
+
+    import oracle as ref
+    from block_quantized_dsq_b200 import synth
+    seeds = synth.SEEDS
+    out = {}
+
+    def timed(fn):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt > budget_s:
+                return dt / n
+
+    x1 = synth.activations(seeds["gemv_q4_k_4096"]["x"], 1, 4096)
+    t = timed(lambda: ref.quantize_act_q8(x1))
+    out["quantize_act_q8_1x4096"] = {"us_per_call": round(t * 1e6, 2),
+                                     "GB/s": round((4096 * 4 + 4096 + 1024) / t / 1e9, 4)}
+    for name, qtype, N, K, sw, sx, G in (
+            ("gemv_q8_0_1024x1024", 8, 1024, 1024, seeds["gemv_q8_0_1024"]["w"], seeds["gemv_q8_0_1024"]["x"], 1),
+            ("gemv_q4_k_4096x4096", 12, 4096, 4096, seeds["gemv_q4_k_4096"]["w"], seeds["gemv_q4_k_4096"]["x"], 1),
+            ("grouped_q8_0_8x1024x4096", 8, 1024, 4096, seeds["grouped_q8_0_8x1024x4096"]["w_base"],
+             seeds["grouped_q8_0_8x1024x4096"]["x_base"], 8)):
+        w = np.concatenate([ref.quantize(qtype, synth.weights(sw + g, N, K)) for g in range(G)])
+        xq, xd, xs = ref.quantize_act_q8(np.concatenate([synth.activations(sx + g, 1, K) for g in range(G)]))
+
+        def run(w=w, xq=xq, xd=xd, xs=xs, qtype=qtype, N=N, K=K, G=G):
+            for g in range(G):
+                ref.gemv(qtype, w[g * N:(g + 1) * N], K, xq[g], xd[g], xs[g])
+        t = timed(run)
+        alg = w.nbytes + G * (K + K // 32 * 4 * (2 if qtype == 12 else 1)) + G * N * 4
+        out[name] = {"us_per_call": round(t * 1e6, 1), "GB/s": round(alg / t / 1e9, 4)}
+    K, N, M, rows = 4096, 4096, 128, 256
+    w = ref.quantize(12, synth.weights(seeds["prefill"]["w_q4_k"], rows, K))
+    x = synth.activations(seeds["prefill"]["x_base"] + M, M, K)
+    t = timed(lambda: ref.prefill_f64(12, w, K, x))
+    out["prefill_q4_k_n4096_m128"] = {"sample": f"{rows} of {N} weight rows x {M} tokens, fp64",
+                                      "GFLOP/s": round(2.0 * M * rows * K / t / 1e9, 4),
+                                      "us_per_full_call": round(t * N / rows * 1e6, 1)}
+    out["cores"] = 1
+    out["kind"] = "oracle"
+    return out
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: same metric and workload, a bounded
     sample per step, host cores only (rank 0)."""
@@ -620,7 +773,7 @@ def run_reference(args, world, rank):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "host cores, rank 0"},
+            "data": "synthetic", "config": bench_config(world),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
