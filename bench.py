@@ -550,6 +550,47 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
                                                "weight_copies": R}
         del keep, W0, W1
 
+    # multi-token decode GEMV (dsq_gemv_tokens): M = 1..8 tokens per weight
+    # read, next to M single-token GEMV calls on the same weights
+    for qtype, tag, N, N1 in ((dsq.DSQ_Q4_K, "q4_k_4096x4096", 4096, 0),
+                              (dsq.DSQ_Q8_0, "paired_q8_0_2x8192x4096", N_PAIR, N_PAIR)):
+        Ms = [M for M in (1, 2, 4, 8) if want(f"tokens_{tag}_m{M}")]
+        if not Ms:
+            continue
+        K = 4096
+        w = quantized_weights(dsq, qtype, 620 + qtype, N + N1, K)
+        R = copies_for(w.numel())
+        ws = [w] + [w.clone() for _ in range(R - 1)]
+        rbw = dsq.dsq_row_bytes(qtype, K)
+        p0 = [c.data_ptr() for c in ws]
+        x, xq, xd, xs = act(621, 8, K)
+        pq, pd, ps = xq.data_ptr(), xd.data_ptr(), xs.data_ptr()
+        y = torch.empty((8, N + N1), dtype=torch.float32, device="cuda")
+        py = y.data_ptr()
+        for M in Ms:
+            fn = lambda i, st, M=M: L.dsq_gemv_tokens(  # noqa: E731
+                qtype, p0[i % R], N, p0[i % R] + N * rbw if N1 else None, N1, K, M, pq, pd, ps, py,
+                py + M * N * 4 if N1 else None, st)
+            t = time_graph(fn, R * max(1, 64 // R))
+            alg = w.numel() + M * (K + K // 32 * 4 * (2 if qtype == dsq.DSQ_Q4_K else 1)) + M * (N + N1) * 4
+            row = {**stats_row(t, alg), "weight_copies": R, "tokens": M}
+            # the same M tokens as M single-token calls, each reading its weights from HBM
+            if N1:
+                fn1 = lambda i, st, M=M: [L.dsq_gemv_paired(  # noqa: E731
+                    qtype, p0[(i * M + m) % R], N, p0[(i * M + m) % R] + N * rbw, N1, K, pq + m * K,
+                    pd + m * K // 8, ps + m * K // 8, py, py + N * 4, st) for m in range(M)]
+            elif qtype == dsq.DSQ_Q8_0:
+                fn1 = lambda i, st, M=M: [L.dsq_gemv_q8_0(p0[(i * M + m) % R], N, K, pq + m * K,  # noqa: E731
+                                                          pd + m * K // 8, py, st) for m in range(M)]
+            else:
+                fn1 = lambda i, st, M=M: [L.dsq_gemv_q4_k(p0[(i * M + m) % R], N, K, pq + m * K,  # noqa: E731
+                                                          pd + m * K // 8, ps + m * K // 8, py, st)
+                                          for m in range(M)]
+            t1 = time_graph(fn1, max(1, 64 // M))
+            row["m_single_calls_us"] = round(t1 * 1e6, 3)
+            rows[f"tokens_{tag}_m{M}"] = row
+        del ws, w
+
     # decode GEMV N-sweep at K = 4096: the asymptotic HBM fraction once the
     # launch and first-byte latency are amortised over more rows.  The rows
     # of a 4096-row seeded matrix are repeated on the device (distinct
@@ -627,6 +668,15 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
                 t2 = time_graph(per_token, max(1, 48 // M))
                 row["m_decode_calls_us"] = round(t2 * 1e6, 3)
                 row["m_decode_calls_stats"] = dict(LAST_STATS)
+                if M <= 8:
+                    # the same tokens through the multi-token GEMV: one
+                    # quantize of the M rows, one weight read for all of them
+                    def tokens(i, st, M=M, pq=pq, pd=pd, ps=ps, px=px, py=py):
+                        L.dsq_quantize_act_q8(px, M, K, pq, pd, ps, st)
+                        L.dsq_gemv_tokens(qtype, pw[i % R], N, None, 0, K, M, pq, pd, ps, py, None, st)
+                    t3 = time_graph(tokens, R * max(1, 24 // R))
+                    row["tokens_call_us"] = round(t3 * 1e6, 3)
+                    row["tokens_call_stats"] = dict(LAST_STATS)
                 del xq, xd, xs
             rows[f"prefill_{tag}_m{M}"] = row
             del x, y, wsp

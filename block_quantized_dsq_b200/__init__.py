@@ -16,10 +16,11 @@ import threading
 __all__ = [
     "DSQ_Q8_0", "DSQ_Q4_K", "DsqError", "lib", "dsq_row_bytes", "dsq_quantize_act_q8",
     "dsq_gemv_q8_0", "dsq_gemv_q4_k", "dsq_gemv_paired", "dsq_gemv_grouped", "dsq_gemv_f32",
-    "dsq_gemv_paired_f32", "dsq_gemv_grouped_f32", "dsq_gemm_prefill",
+    "dsq_gemv_paired_f32", "dsq_gemv_grouped_f32", "dsq_gemv_tokens", "dsq_gemm_prefill",
+    "dsq_gemm_prefill_grouped", "dsq_prefill_grouped_workspace_bytes",
     "dsq_prefill_workspace_bytes", "dsq_gemm_prefill_noalloc", "dsq_quantize_weights", "dsq_device_status", "dsq_last_error",
     "dsq_version", "dsq_launch_count", "dsq_test_block_sums", "dsq_test_set_wait_limit_ns",
-    "dsq_test_prefill_operands", "LIB_PATH",
+    "dsq_test_prefill_operands", "dsq_test_block_sums_tokens", "LIB_PATH",
 ]
 
 DSQ_Q8_0 = 8
@@ -47,8 +48,11 @@ _SIGS = {
     "dsq_gemv_f32": (_INT, [_INT, _P, _I64, _I64, _P, _P, _P]),
     "dsq_gemv_paired_f32": (_INT, [_INT, _P, _I64, _P, _I64, _I64, _P, _P, _P, _P]),
     "dsq_gemv_grouped_f32": (_INT, [_INT, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "dsq_gemv_tokens": (_INT, [_INT, _P, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "dsq_gemm_prefill": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P, _SZ, _P]),
     "dsq_prefill_workspace_bytes": (_SZ, [_INT, _I64, _I64, _I64]),
+    "dsq_gemm_prefill_grouped": (_INT, [_INT, _I64, _P, _P, _I64, _P, _I64, _P, _P, _SZ, _P]),
+    "dsq_prefill_grouped_workspace_bytes": (_SZ, [_INT, _I64, _P, _I64, _I64]),
     "dsq_gemm_prefill_noalloc": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P]),
     "dsq_quantize_weights": (_INT, [_INT, _P, _I64, _I64, _P, _P]),
     "dsq_device_status": (_INT, [_P]),
@@ -58,6 +62,7 @@ _SIGS = {
     "dsq_test_block_sums": (_INT, [_INT, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "dsq_test_set_wait_limit_ns": (_INT, [ctypes.c_uint64]),
     "dsq_test_prefill_operands": (_INT, [_INT, _P, _I64, _I64, _P, _I64, _P, _P, _P, _P]),
+    "dsq_test_block_sums_tokens": (_INT, [_INT, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
 }
 
 _lock = threading.Lock()
@@ -156,6 +161,14 @@ def dsq_gemv_grouped_f32(qtype, w, G, N, K, x, y, stream=None):
            lib().dsq_gemv_grouped_f32(qtype, _ptr(w), G, N, K, _ptr(x), _ptr(y), _stream(stream)))
 
 
+def dsq_gemv_tokens(qtype, w0, N0, w1, N1, K, M, xq, xd, xs, y0, y1, stream=None):
+    """M = 1..8 prequantized tokens against one weight (N1 = 0) or two that
+    share the input; every weight byte is read once for all M tokens."""
+    _check("dsq_gemv_tokens",
+           lib().dsq_gemv_tokens(qtype, _ptr(w0), N0, _ptr(w1), N1, K, M, _ptr(xq), _ptr(xd), _ptr(xs),
+                                 _ptr(y0), _ptr(y1), _stream(stream)))
+
+
 def dsq_gemm_prefill(qtype, w, N, K, x, M, y, workspace, workspace_bytes, stream=None):
     _check("dsq_gemm_prefill",
            lib().dsq_gemm_prefill(qtype, _ptr(w), N, K, _ptr(x), M, _ptr(y), _ptr(workspace),
@@ -164,6 +177,24 @@ def dsq_gemm_prefill(qtype, w, N, K, x, M, y, workspace, workspace_bytes, stream
 
 def dsq_prefill_workspace_bytes(qtype: int, N: int, K: int, M: int) -> int:
     return lib().dsq_prefill_workspace_bytes(qtype, N, K, M)
+
+
+def _host_array(ctype, values):
+    return (ctype * len(values))(*values)
+
+
+def dsq_gemm_prefill_grouped(qtype, ws, Ns, K, x, M, ys, workspace, workspace_bytes, stream=None):
+    """G weights (lists ws, Ns, ys of equal length) sharing one activation X."""
+    G = len(ws)
+    _check("dsq_gemm_prefill_grouped",
+           lib().dsq_gemm_prefill_grouped(qtype, G, _host_array(ctypes.c_void_p, [_ptr(w) for w in ws]),
+                                          _host_array(ctypes.c_int64, list(Ns)), K, _ptr(x), M,
+                                          _host_array(ctypes.c_void_p, [_ptr(y) for y in ys]), _ptr(workspace),
+                                          workspace_bytes, _stream(stream)))
+
+
+def dsq_prefill_grouped_workspace_bytes(qtype: int, Ns, K: int, M: int) -> int:
+    return lib().dsq_prefill_grouped_workspace_bytes(qtype, len(Ns), _host_array(ctypes.c_int64, list(Ns)), K, M)
 
 
 DSQ_PREFILL_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -215,3 +246,9 @@ def dsq_test_prefill_operands(qtype, w, N, K, x, M, x16, shift, w16, stream=None
     _check("dsq_test_prefill_operands",
            lib().dsq_test_prefill_operands(qtype, _ptr(w), N, K, _ptr(x), M, _ptr(x16), _ptr(shift), _ptr(w16),
                                            _stream(stream)))
+
+
+def dsq_test_block_sums_tokens(qtype, w, N, K, M, xq, xd, xs, y, isum, stream=None):
+    _check("dsq_test_block_sums_tokens",
+           lib().dsq_test_block_sums_tokens(qtype, _ptr(w), N, K, M, _ptr(xq), _ptr(xd), _ptr(xs), _ptr(y),
+                                            _ptr(isum), _stream(stream)))

@@ -1,0 +1,549 @@
+// gemv_tokens.cu -- multi-token decode GEMV: M = 1..8 prequantized activation
+// rows against one block-quantized weight, or against two weights that share
+// the same input (the paired Q / KV projections), reading every weight byte
+// once for all M tokens.
+//
+// Sources: "Support AProjQ4 GGUFs: Q4_K dense attention projections"
+// (antirez/ds4 PR #621), GB10 test report: short multi-token batches of up to
+// 8 tokens (the grouped-tok8 and QKV-pair decode paths) are worth a path of
+// their own only if they keep decode consistent and cost nothing; "ROCm:
+// restore DeepSeek V4 Flash decode performance" (antirez/ds4 PR #623),
+// Summary: the activation is prequantized to Q8 once and shared by the
+// projections that read it.
+//
+// Numerics: each token's output equals, bit for bit, what the single-token
+// entry points (dsq_gemv_q8_0 / dsq_gemv_q4_k / dsq_gemv_paired) give for that
+// token alone.  The block terms, the per-unit partial sums and the order in
+// which they are added are the single-token kernel's, so decoding M tokens
+// in one call is indistinguishable from M decode steps.
+//
+// B200 design (HBM-bound weight stream, M tokens per weight byte):
+//  * lane = weight row.  A warp handles a group of 32 consecutive rows of one
+//    weight, one 256-element unit at a time: the unit arrives as one 2-D TMA
+//    box (32 rows x 272 B for Q8_0, x 144 B for Q4_K) in the warp's ring of
+//    shared-memory slots.
+//  * All 32 lanes read the same activation bytes at the same moment, so the
+//    M tokens' codes and scales come out of shared memory as broadcasts:
+//    per unit and token, 20 16-byte reads for the whole warp.
+//  * A row is split into units the way the single-token kernel splits it
+//    across the lanes of a row: virtual lane j (j < G, G = units per row
+//    rounded up to a power of two, at most 32) owns units j, j+G, ...  The
+//    CTA's warps take virtual lanes j = warp + W*i.  Each virtual lane keeps
+//    its partial sum per token; the partials meet in the single-token
+//    kernel's butterfly order -- inside the warp for the strides >= W, then
+//    across warps through shared memory.
+//  * Persistent CTAs (one per SM) step through the row groups of both
+//    weights; weights are read once, activations stay in shared memory.
+#include <cudaTypedefs.h>
+
+#include "../../include/dsq_test.h"
+#include "dsq_host.h"
+
+namespace dsq {
+namespace {
+
+constexpr int kTokMaxM = 8;
+constexpr int kTokWarps = 8;          // warps per CTA
+constexpr int kTokRows = 32;          // rows per group (lane = row)
+constexpr int kTokMaxStages = 4;      // ring slots per warp
+constexpr size_t kTokSmemLimit = 227 * 1024;
+constexpr size_t kTokMaxActSmem = 64 * 1024;
+
+template <int TYPE> __host__ __device__ constexpr int tok_unit_bytes() { return TYPE == DSQ_Q8_0 ? 272 : 144; }
+
+struct TokArgs {
+  float *y[2];            // outputs [M][n[s]] of each weight
+  int64_t n[2];           // rows of each weight
+  int64_t groups0;        // 32-row groups of weight 0 (weight 1's follow)
+  int64_t total_groups;
+  int64_t K;
+  int nunits;             // K / 256
+  int G;                  // virtual lanes per row (power of two, <= 32)
+  int W;                  // warps with virtual lanes: min(8, G)
+  int stages;             // ring slots per warp
+  uint32_t box_bytes;     // one TMA box: 32 rows x one unit
+  uint32_t q_bytes, d_bytes, s_bytes;   // activation areas in shared memory
+  uint32_t ring_off, bar_off, red_off;  // shared-memory offsets
+  const int8_t *xq;       // [M][K]
+  const float *xd;        // [M][K/32]
+  const int32_t *xs;      // [M][K/32] (Q4_K)
+  int32_t *isum;          // test hook: [M][n0 + n1][K/32] block sums, or NULL
+  WaitCtl wait;
+};
+
+__device__ __forceinline__ float tok_half_lo(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+}
+__device__ __forceinline__ float tok_half_hi(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+// One Q8_0 unit (8 blocks, 272 bytes at p) of this lane's row against unit u
+// of the M tokens.  Block b starts at byte 34b: even b has its scale in the
+// low half of word 17b/2 and its codes two bytes later (realigned with a
+// funnel shift), odd b its scale in the high half of word (17b-1)/2 and its
+// codes word-aligned.  part[m] = sum over the 8 blocks, in block order from
+// 0, of (d_w * xd) * isum: the single-token kernel's unit partial.
+template <int M>
+__device__ __forceinline__ void tok_unit_q8_0(const uint8_t *p, const int8_t *sq, const float *sd, int64_t K, int u,
+                                              float (&part)[M], int32_t *isum, int64_t isum_tok_stride) {
+  uint32_t w[68];
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < 17; ++i) {
+    const uint4 v = p4[i];
+    w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+#pragma unroll
+  for (int m = 0; m < M; ++m) part[m] = 0.0f;
+  const int64_t nb = K / 32;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    uint32_t c[8];
+    float dw;
+    if ((b & 1) == 0) {
+      const int a0 = 17 * b / 2;
+      dw = tok_half_lo(w[a0]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = __funnelshift_r(w[a0 + i], w[a0 + i + 1], 16);
+    } else {
+      const int a0 = (17 * b - 1) / 2;
+      dw = tok_half_hi(w[a0]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = w[a0 + 1 + i];
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint4 *x4 = reinterpret_cast<const uint4 *>(sq + m * K + u * 256 + b * 32);
+      const uint4 x0 = x4[0], x1 = x4[1];
+      int32_t s = 0;
+      s = __dp4a(static_cast<int>(c[0]), static_cast<int>(x0.x), s);
+      s = __dp4a(static_cast<int>(c[1]), static_cast<int>(x0.y), s);
+      s = __dp4a(static_cast<int>(c[2]), static_cast<int>(x0.z), s);
+      s = __dp4a(static_cast<int>(c[3]), static_cast<int>(x0.w), s);
+      s = __dp4a(static_cast<int>(c[4]), static_cast<int>(x1.x), s);
+      s = __dp4a(static_cast<int>(c[5]), static_cast<int>(x1.y), s);
+      s = __dp4a(static_cast<int>(c[6]), static_cast<int>(x1.z), s);
+      s = __dp4a(static_cast<int>(c[7]), static_cast<int>(x1.w), s);
+      if (isum) isum[m * isum_tok_stride + u * 8 + b] = s;
+      part[m] += __fmul_rn(__fmul_rn(dw, sd[m * nb + u * 8 + b]), static_cast<float>(s));
+    }
+  }
+}
+
+// One Q4_K super-block (144 bytes at p: word 0 = d | dmin << 16, words 1..3
+// the packed 6-bit scales and mins, words 4..35 the nibbles) against unit u of
+// the M tokens: part[m] = sum over sub-blocks j, in order from 0, of
+// xd * ((d*sc_j)*isum_j - (dmin*m_j)*xs_j).
+template <int M>
+__device__ __forceinline__ void tok_unit_q4_k(const uint8_t *p, const int8_t *sq, const float *sd,
+                                              const int32_t *ss, int64_t K, int u, float (&part)[M],
+                                              int32_t *isum, int64_t isum_tok_stride) {
+  uint32_t w[36];
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < 9; ++i) {
+    const uint4 v = p4[i];
+    w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  const float d = tok_half_lo(w[0]), dmin = tok_half_hi(w[0]);
+  const uint32_t s0 = w[1], s1 = w[2], s2 = w[3];
+  const uint32_t scA = s0 & 0x3f3f3f3fu;
+  const uint32_t mA = s1 & 0x3f3f3f3fu;
+  const uint32_t scB = (s2 & 0x0f0f0f0fu) | ((s0 >> 2) & 0x30303030u);
+  const uint32_t mB = ((s2 >> 4) & 0x0f0f0f0fu) | ((s1 >> 2) & 0x30303030u);
+#pragma unroll
+  for (int m = 0; m < M; ++m) part[m] = 0.0f;
+  const int64_t nb = K / 32;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t scw = j < 4 ? scA : scB, mw = j < 4 ? mA : mB;
+    const int sh = 8 * (j & 3);
+    const float dsc = __fmul_rn(d, static_cast<float>((scw >> sh) & 0xffu));
+    const float dmm = __fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu));
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t byte4 = w[4 + 8 * (j >> 1) + i];
+      c[i] = (j & 1) ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint4 *x4 = reinterpret_cast<const uint4 *>(sq + m * K + u * 256 + j * 32);
+      const uint4 x0 = x4[0], x1 = x4[1];
+      int32_t s = 0;
+      s = __dp4a(static_cast<int>(c[0]), static_cast<int>(x0.x), s);
+      s = __dp4a(static_cast<int>(c[1]), static_cast<int>(x0.y), s);
+      s = __dp4a(static_cast<int>(c[2]), static_cast<int>(x0.z), s);
+      s = __dp4a(static_cast<int>(c[3]), static_cast<int>(x0.w), s);
+      s = __dp4a(static_cast<int>(c[4]), static_cast<int>(x1.x), s);
+      s = __dp4a(static_cast<int>(c[5]), static_cast<int>(x1.y), s);
+      s = __dp4a(static_cast<int>(c[6]), static_cast<int>(x1.z), s);
+      s = __dp4a(static_cast<int>(c[7]), static_cast<int>(x1.w), s);
+      if (isum) isum[m * isum_tok_stride + u * 8 + j] = s;
+      const int64_t bi = m * nb + u * 8 + j;
+      const float t = __fmul_rn(dsc, static_cast<float>(s));
+      const float v = __fmul_rn(dmm, static_cast<float>(ss[bi]));
+      part[m] += __fmul_rn(sd[bi], __fsub_rn(t, v));
+    }
+  }
+}
+
+// Position of a warp's work: row group g, virtual-lane slot i (virtual lane
+// v = warp + W*i), unit u (v, v+G, ...).  next() steps in consumption order.
+struct TokCursor {
+  int64_t g;
+  int i, u;
+  __device__ __forceinline__ void first(const TokArgs &a, int warp, int vpw) {
+    g = blockIdx.x;
+    i = 0;
+    u = warp;
+    if (vpw == 0 || u >= a.nunits) g = a.total_groups;   // this warp has no units
+  }
+  __device__ __forceinline__ void next(const TokArgs &a, int warp, int vpw) {
+    u += a.G;
+    if (u >= a.nunits) {
+      ++i;
+      u = warp + a.W * i;
+      if (i >= vpw || u >= a.nunits) {
+        g += gridDim.x;
+        i = 0;
+        u = warp;
+      }
+    }
+  }
+  __device__ __forceinline__ bool valid(const TokArgs &a) const { return g < a.total_groups; }
+};
+
+template <int UB>
+__device__ __forceinline__ void tok_issue(const CUtensorMap *map0, const CUtensorMap *map1, const TokArgs &a,
+                                          const TokCursor &c, uint8_t *dst, uint64_t *bar) {
+  const bool second = c.g >= a.groups0;
+  const int32_t row0 = static_cast<int32_t>((second ? c.g - a.groups0 : c.g) * kTokRows);
+  mbar_arrive_expect_tx(bar, a.box_bytes);
+  tma_load_2d(dst, second ? map1 : map0, c.u * (UB / 4), row0, bar);
+}
+
+template <int TYPE, int M>
+__global__ void __launch_bounds__(kTokWarps * 32, 1)
+    gemv_tokens_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
+                       const __grid_constant__ TokArgs a) {
+  constexpr int UB = tok_unit_bytes<TYPE>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int W = a.W, S = a.stages;
+  const int vpw = warp < W ? a.G / W : 0;   // virtual lanes of this warp
+  const int8_t *sq = reinterpret_cast<const int8_t *>(base);
+  const float *sd = reinterpret_cast<const float *>(base + a.q_bytes);
+  const int32_t *ss = reinterpret_cast<const int32_t *>(base + a.q_bytes + a.d_bytes);
+  uint8_t *ring = base + a.ring_off + static_cast<size_t>(warp) * S * a.box_bytes;
+  uint64_t *act_bar = reinterpret_cast<uint64_t *>(base + a.bar_off);
+  uint64_t *bars = act_bar + 1 + warp * kTokMaxStages;
+  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][8 warps][M][32 rows]
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(act_bar + 1 + kTokWarps * kTokMaxStages);
+
+  if (threadIdx.x == 0) {
+    mbar_init(act_bar, 1);
+    *abort_flag = 0u;
+    prefetch_tensormap(&map0);
+    prefetch_tensormap(&map1);
+  }
+  if (lane == 0)
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+  fence_barrier_init();
+  // weights are read-only: bring this warp's first boxes toward L2 while the
+  // kernel before us (usually the activation quantizer) finishes
+  TokCursor issue;
+  issue.first(a, warp, vpw);
+  if (lane == 0) {
+    TokCursor c = issue;
+    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp, vpw)) {
+      const bool second = c.g >= a.groups0;
+      prefetch_l2_tile_2d(second ? &map1 : &map0, c.u * (UB / 4),
+                          static_cast<int32_t>((second ? c.g - a.groups0 : c.g) * kTokRows));
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+
+  if (threadIdx.x == 0) {
+    // the M tokens' prequantized activations, once, into shared memory
+    const uint64_t keep = l2_policy_evict_last();
+    mbar_arrive_expect_tx(act_bar, a.q_bytes + a.d_bytes + a.s_bytes);
+    bulk_g2s(base, a.xq, a.q_bytes, act_bar, keep);
+    bulk_g2s(base + a.q_bytes, a.xd, a.d_bytes, act_bar, keep);
+    if (a.s_bytes) bulk_g2s(base + a.q_bytes + a.d_bytes, a.xs, a.s_bytes, act_bar, keep);
+  }
+  int64_t n_issued = 0, n_waited = 0;
+  if (lane == 0) {
+    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp, vpw), ++n_issued)
+      tok_issue<UB>(&map0, &map1, a, issue, ring + static_cast<size_t>(s) * a.box_bytes, &bars[s]);
+  }
+  bool ok = __all_sync(0xffffffffu, mbar_wait_for(act_bar, 0, a.wait.limit_ns));
+  if (!ok && lane == 0) {
+    *abort_flag = 1u;
+    record_timeout(a.wait);
+  }
+
+  int slot = 0;
+  uint32_t parity = 0;
+  int buf = 0;
+  const int64_t nb = a.K / 32;
+  const int64_t rows_total = a.n[0] + a.n[1];
+  for (int64_t g = blockIdx.x; g < a.total_groups; g += gridDim.x, buf ^= 1) {
+    const bool second = g >= a.groups0;
+    const int64_t rloc = (second ? g - a.groups0 : g) * kTokRows + lane;   // this lane's row in its weight
+    const int64_t vrow = (second ? a.n[0] : 0) + rloc;                   // in [weight 0 rows, weight 1 rows]
+    float acc[4][M];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[i][m] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i >= vpw) break;
+      for (int u = warp + W * i; u < a.nunits; u += a.G) {
+        ok = ok && *abort_flag == 0u;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
+        if (!ok) {
+          if (lane == 0 && *abort_flag == 0u) {
+            *abort_flag = 1u;
+            record_timeout(a.wait);
+          }
+        } else {
+          ++n_waited;
+          float part[M];
+          const uint8_t *rowp = ring + static_cast<size_t>(slot) * a.box_bytes + static_cast<size_t>(lane) * UB;
+          int32_t *isum = (a.isum && rloc < a.n[second ? 1 : 0]) ? a.isum + vrow * nb : nullptr;
+          if constexpr (TYPE == DSQ_Q8_0)
+            tok_unit_q8_0<M>(rowp, sq, sd, a.K, u, part, isum, rows_total * nb);
+          else
+            tok_unit_q4_k<M>(rowp, sq, sd, ss, a.K, u, part, isum, rows_total * nb);
+#pragma unroll
+          for (int m = 0; m < M; ++m) acc[i][m] += part[m];
+          __syncwarp();
+          if (lane == 0 && issue.valid(a)) {
+            fence_proxy_async_smem();
+            tok_issue<UB>(&map0, &map1, a, issue, ring + static_cast<size_t>(slot) * a.box_bytes, &bars[slot]);
+            issue.next(a, warp, vpw);
+            ++n_issued;
+          }
+        }
+        if (++slot == S) {
+          slot = 0;
+          parity ^= 1u;
+        }
+      }
+    }
+    // butterfly strides >= W stay inside the warp: virtual lane j = warp + W*i
+    // meets j ^ (W * st) = warp + W * (i ^ st)
+    float mine[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      if (vpw == 4) mine[m] = (acc[0][m] + acc[2][m]) + (acc[1][m] + acc[3][m]);
+      else if (vpw == 2) mine[m] = acc[0][m] + acc[1][m];
+      else mine[m] = acc[0][m];
+    }
+    float *rb = red + static_cast<size_t>(buf) * kTokWarps * M * 32;
+#pragma unroll
+    for (int m = 0; m < M; ++m) rb[(warp * M + m) * 32 + lane] = mine[m];
+    __syncthreads();
+    // strides < W cross warps: ((r0+r4)+(r2+r6)) + ((r1+r5)+(r3+r7)) for W = 8
+    for (int m = warp; m < M; m += kTokWarps) {
+      float r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r[k] = k < W ? rb[(k * M + m) * 32 + lane] : 0.0f;
+      float v;
+      if (W == 8) v = ((r[0] + r[4]) + (r[2] + r[6])) + ((r[1] + r[5]) + (r[3] + r[7]));
+      else if (W == 4) v = (r[0] + r[2]) + (r[1] + r[3]);
+      else if (W == 2) v = r[0] + r[1];
+      else v = r[0];
+      const int sgi = second ? 1 : 0;
+      if (rloc < a.n[sgi] && *abort_flag == 0u) a.y[sgi][m * a.n[sgi] + rloc] = v;
+    }
+  }
+  // after an abort: let this warp's copies still in flight land before exit
+  if (lane == 0) {
+    for (int64_t k = n_waited; k < n_issued; ++k)
+      mbar_wait_for(&bars[k % S], static_cast<uint32_t>((k / S) & 1), kDrainLimitNs);
+  }
+  if (threadIdx.x == 0 && !ok) mbar_wait_for(act_bar, 0, kDrainLimitNs);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tok_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// The weight rows viewed as uint32 [N][row_bytes / 4]; a box is one
+// 256-element unit (68 or 36 words) of 32 rows; rows past N read as zero.
+int tok_map(CUtensorMap *map, const void *w, int type, int64_t N, int64_t K, const char *name) {
+  auto enc = tok_encode_fn();
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+  const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
+  const cuuint32_t box[2] = {type == DSQ_Q8_0 ? 68u : 36u, static_cast<cuuint32_t>(kTokRows)};
+  const cuuint32_t estride[2] = {1u, 1u};
+  const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box, estride,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "%s: weight tensor map (%d)", name, (int)cr);
+  return DSQ_OK;
+}
+
+template <int TYPE, int M>
+cudaError_t tok_launch(const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a, unsigned grid, size_t smem,
+                       cudaStream_t st) {
+  return launch_pdl(gemv_tokens_kernel<TYPE, M>, dim3(grid), dim3(kTokWarps * 32), smem, st, m0, m1, a);
+}
+
+template <int TYPE>
+const void *tok_kernel(int M) {
+  switch (M) {
+    case 1: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 1>);
+    case 2: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 2>);
+    case 3: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 3>);
+    case 4: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 4>);
+    case 5: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 5>);
+    case 6: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 6>);
+    case 7: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 7>);
+    default: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 8>);
+  }
+}
+
+template <int TYPE>
+cudaError_t tok_dispatch(int M, const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a, unsigned grid,
+                         size_t smem, cudaStream_t st) {
+  switch (M) {
+    case 1: return tok_launch<TYPE, 1>(m0, m1, a, grid, smem, st);
+    case 2: return tok_launch<TYPE, 2>(m0, m1, a, grid, smem, st);
+    case 3: return tok_launch<TYPE, 3>(m0, m1, a, grid, smem, st);
+    case 4: return tok_launch<TYPE, 4>(m0, m1, a, grid, smem, st);
+    case 5: return tok_launch<TYPE, 5>(m0, m1, a, grid, smem, st);
+    case 6: return tok_launch<TYPE, 6>(m0, m1, a, grid, smem, st);
+    case 7: return tok_launch<TYPE, 7>(m0, m1, a, grid, smem, st);
+    default: return tok_launch<TYPE, 8>(m0, m1, a, grid, smem, st);
+  }
+}
+
+size_t tok_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int run_tokens(const char *name, int type, const void *w0, int64_t N0, const void *w1, int64_t N1, int64_t K,
+               int64_t M, const int8_t *xq, const float *xd, const int32_t *xs, float *y0, float *y1,
+               int32_t *isum, cudaStream_t stream) {
+  DSQ_REQUIRE(type == DSQ_Q8_0 || type == DSQ_Q4_K, DSQ_ERR_INVALID_ARG, "%s: unsupported type %d", name, type);
+  DSQ_REQUIRE(K > 0 && N0 >= 0 && N1 >= 0, DSQ_ERR_INVALID_ARG, "%s: negative size", name);
+  DSQ_REQUIRE(M >= 1 && M <= kTokMaxM, DSQ_ERR_SHAPE, "%s: M=%lld tokens (1..%d supported)", name, (long long)M,
+              kTokMaxM);
+  DSQ_REQUIRE(K % 256 == 0, DSQ_ERR_SHAPE, "%s: K=%lld must be a multiple of 256", name, (long long)K);
+  DSQ_REQUIRE(N0 + N1 <= (int64_t(1) << 31), DSQ_ERR_SHAPE, "%s: too many rows", name);
+  const size_t q_bytes = static_cast<size_t>(M) * K;
+  const size_t d_bytes = static_cast<size_t>(M) * (K / 32) * 4;
+  const size_t s_bytes = type == DSQ_Q4_K ? d_bytes : 0;
+  DSQ_REQUIRE(q_bytes + d_bytes + s_bytes <= kTokMaxActSmem, DSQ_ERR_SHAPE,
+              "%s: %lld tokens of K=%lld exceed the %zu bytes of shared memory kept for activations", name,
+              (long long)M, (long long)K, kTokMaxActSmem);
+  if (N0 + N1 == 0) return DSQ_OK;
+  DSQ_REQUIRE(xq && xd && (type == DSQ_Q8_0 || xs), DSQ_ERR_INVALID_ARG, "%s: null activation pointer", name);
+  DSQ_REQUIRE((N0 == 0 || (w0 && y0)) && (N1 == 0 || (w1 && y1)), DSQ_ERR_INVALID_ARG,
+              "%s: null weight/output pointer", name);
+  DSQ_REQUIRE(aligned(xq, 16) && aligned(xd, 16) && (type == DSQ_Q8_0 || aligned(xs, 16)), DSQ_ERR_ALIGNMENT,
+              "%s: xq/xd/xs must be 16-byte aligned", name);
+  DSQ_REQUIRE((N0 == 0 || (aligned(w0, 16) && aligned(y0, 4))) && (N1 == 0 || (aligned(w1, 16) && aligned(y1, 4))),
+              DSQ_ERR_ALIGNMENT, "%s: weights must be 16-byte and outputs 4-byte aligned", name);
+  WaitCtl ctl;
+  int sms = 0;
+  int rc = wait_ctl(&ctl, &sms);
+  if (rc != DSQ_OK) return rc;
+
+  TokArgs a{};
+  a.y[0] = y0;
+  a.y[1] = y1;
+  a.n[0] = N0;
+  a.n[1] = N1;
+  a.groups0 = (N0 + kTokRows - 1) / kTokRows;
+  a.total_groups = a.groups0 + (N1 + kTokRows - 1) / kTokRows;
+  a.K = K;
+  a.nunits = static_cast<int>(K / 256);
+  a.G = 1;
+  while (a.G < a.nunits && a.G < 32) a.G <<= 1;
+  a.W = a.G < kTokWarps ? a.G : kTokWarps;
+  a.box_bytes = static_cast<uint32_t>(kTokRows * (type == DSQ_Q8_0 ? 272 : 144));
+  a.q_bytes = static_cast<uint32_t>(q_bytes);
+  a.d_bytes = static_cast<uint32_t>(d_bytes);
+  a.s_bytes = static_cast<uint32_t>(s_bytes);
+  a.xq = xq;
+  a.xd = xd;
+  a.xs = xs;
+  a.isum = isum;
+  a.wait = ctl;
+  // shared memory: activations | ring (W warps x stages x box) | barriers | reduction
+  const size_t act = tok_align(q_bytes + d_bytes + s_bytes, 1024);
+  const size_t bars = (1 + kTokWarps * kTokMaxStages + 1) * sizeof(uint64_t);
+  const size_t red = 2 * static_cast<size_t>(kTokWarps) * M * 32 * sizeof(float);
+  const size_t fixed = 1024 + act + tok_align(bars, 16) + red;
+  const size_t per_stage = static_cast<size_t>(kTokWarps) * a.box_bytes;
+  int stages = static_cast<int>((kTokSmemLimit - fixed) / per_stage);
+  if (stages > kTokMaxStages) stages = kTokMaxStages;
+  DSQ_REQUIRE(stages >= 2, DSQ_ERR_SHAPE, "%s: no pipeline fits next to %lld tokens of K=%lld", name, (long long)M,
+              (long long)K);
+  a.stages = stages;
+  a.ring_off = static_cast<uint32_t>(act);
+  a.bar_off = static_cast<uint32_t>(act + per_stage * stages);
+  a.red_off = static_cast<uint32_t>(a.bar_off + tok_align(bars, 16));
+  const size_t smem = 1024 + a.red_off + red;
+
+  CUtensorMap m0, m1;
+  const void *wa = N0 > 0 ? w0 : w1;
+  rc = tok_map(&m0, wa, type, N0 > 0 ? N0 : N1, K, name);
+  if (rc != DSQ_OK) return rc;
+  if (N1 > 0) {
+    rc = tok_map(&m1, w1, type, N1, K, name);
+    if (rc != DSQ_OK) return rc;
+  } else {
+    m1 = m0;
+  }
+  const int64_t slots = sms;
+  const unsigned grid = static_cast<unsigned>(a.total_groups < slots ? a.total_groups : slots);
+  const int mi = static_cast<int>(M);
+  rc = set_smem_once(type == DSQ_Q8_0 ? tok_kernel<DSQ_Q8_0>(mi) : tok_kernel<DSQ_Q4_K>(mi), static_cast<int>(smem),
+                     name);
+  if (rc != DSQ_OK) return rc;
+  const cudaError_t e = type == DSQ_Q8_0 ? tok_dispatch<DSQ_Q8_0>(mi, m0, m1, a, grid, smem, stream)
+                                         : tok_dispatch<DSQ_Q4_K>(mi, m0, m1, a, grid, smem, stream);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: %s", name, cudaGetErrorString(e));
+  return after_launch(name);
+}
+
+}  // namespace
+}  // namespace dsq
+
+extern "C" {
+
+int dsq_gemv_tokens(int type, const void *w0, int64_t N0, const void *w1, int64_t N1, int64_t K, int64_t M,
+                    const int8_t *xq, const float *xd, const int32_t *xs, float *y0, float *y1, void *stream) {
+  using namespace dsq;
+  return run_tokens("dsq_gemv_tokens", type, w0, N0, w1, N1, K, M, xq, xd, xs, y0, y1, nullptr, as_stream(stream));
+}
+
+int dsq_test_block_sums_tokens(int type, const void *w, int64_t N, int64_t K, int64_t M, const int8_t *xq,
+                               const float *xd, const int32_t *xs, float *y, int32_t *isum, void *stream) {
+  using namespace dsq;
+  DSQ_REQUIRE(isum != nullptr || N == 0, DSQ_ERR_INVALID_ARG, "dsq_test_block_sums_tokens: null isum");
+  DSQ_REQUIRE(aligned(isum, 4), DSQ_ERR_ALIGNMENT, "dsq_test_block_sums_tokens: isum alignment");
+  return run_tokens("dsq_test_block_sums_tokens", type, w, N, nullptr, 0, K, M, xq, xd, xs, y, nullptr, isum,
+                    as_stream(stream));
+}
+
+}  // extern "C"

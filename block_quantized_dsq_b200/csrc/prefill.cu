@@ -60,12 +60,22 @@ constexpr int kConvWarps = 8;
 constexpr int kWarpEpi0 = kWarpConv0 + kConvWarps;   // warps 10..13: TMEM -> global epilogue
 constexpr int kWarpW = kWarpEpi0 + 4;                 // warp 14: TMA producer of raw weight units
 constexpr int kThreads = (kWarpW + 1) * 32;
+constexpr int kMaxGroup = DSQ_PREFILL_MAX_GROUP;   // weights sharing X in one launch
+
+// The weights' tensor maps (one per weight; unused entries repeat entry 0).
+struct WeightMaps {
+  CUtensorMap m[kMaxGroup];
+};
 
 struct PrefillArgs {
-  int64_t N, K, M;
+  int64_t K, M;
+  int G;                  // weights that share X
+  int64_t N[kMaxGroup];   // rows of each weight
+  float *y[kMaxGroup];    // [M][N_g] outputs, or [splits] x split_stride partials
+  int64_t split_stride[kMaxGroup];   // floats between two splits' partials (a multiple of 4)
+  int64_t tile_n0[kMaxGroup + 1];    // first 256-row tile of each weight in the tile order
   const __half *x16;      // fp16 activations, tile-major and swizzled (see x_to_f16_kernel)
   const int32_t *shift;   // [M] activation row shifts
-  float *y;               // [M][N], or [splits][M][N] partials
   int units_per_split;    // 256-element units of K per split
   int splits;
   int tn;                 // tokens per pair tile (MMA N): 32..256, multiple of 32
@@ -334,20 +344,30 @@ __device__ __forceinline__ bool wait_or_abort(const Smem &s, uint64_t *bar, uint
 // at the same time on the same activation tile (other weight rows) or the
 // same weight tile (other tokens) then read different units instead of the
 // same lines at the same moment.
+// The weight-row tiles of the G weights follow one another in the tile
+// order; g is the tile's weight and n0 its first row within that weight.  The
+// K rotation depends only on the tile's place within its own weight, so a
+// weight computed inside a group gets exactly the sums it gets alone when
+// the split plan is the same.
 struct Tile {
   int64_t mt, n0;
   int u0, u1, rot;
-  int split;
+  int split, g;
 };
 __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   Tile tl;
   tl.mt = t % a.tiles_m;
   const int64_t rest = t / a.tiles_m;
   tl.split = static_cast<int>(rest % a.splits);
-  tl.n0 = (rest / a.splits) * kTileN;
+  const int64_t nt = rest / a.splits;
+  int g = 0;
+  while (g + 1 < a.G && nt >= a.tile_n0[g + 1]) ++g;
+  tl.g = g;
+  const int64_t ntl = nt - a.tile_n0[g];
+  tl.n0 = ntl * kTileN;
   tl.u0 = tl.split * a.units_per_split;
   tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
-  tl.rot = static_cast<int>((rest / a.splits + 7 * tl.mt) % (tl.u1 - tl.u0));
+  tl.rot = static_cast<int>((ntl + 7 * tl.mt) % (tl.u1 - tl.u0));
   return tl;
 }
 
@@ -417,7 +437,7 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
 // by the number of pairs); rank r = this CTA's rank in the cluster.
 template <int TYPE>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ PrefillArgs a) {
+    prefill_kernel(const __grid_constant__ WeightMaps maps, const __grid_constant__ PrefillArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
   constexpr uint32_t RAW_BYTES = kRows * UB;   // one unit of this CTA's 128 rows
   extern __shared__ uint8_t smem_raw[];
@@ -448,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(s.drain, 1);
     *s.abort = 0u;
     fence_barrier_init();
-    prefetch_tensormap(&tmap_w);
+    for (int g = 0; g < a.G; ++g) prefetch_tensormap(&maps.m[g]);
   }
   if (warp == kWarpW && lane == 0 && pair < a.total_tiles) {
     // weights are read-only: start this CTA's first units toward L2 while
@@ -456,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Tile tl = tile_of(a, pair);
     for (int k = 0; k < 2 && k < tl.u1 - tl.u0; ++k) {
       const int u = tl.u0 + (tl.rot + k) % (tl.u1 - tl.u0);
-      prefetch_l2_tile_2d(&tmap_w, u * (UB / 4), static_cast<int32_t>(tl.n0 + kRows * rank));
+      prefetch_l2_tile_2d(&maps.m[tl.g], u * (UB / 4), static_cast<int32_t>(tl.n0 + kRows * rank));
     }
   }
   if (warp == kWarpMma) {
@@ -595,7 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&s.rfull[rs], RAW_BYTES);
-          tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &tmap_w, u * (UB / 4), row0, &s.rfull[rs]);
+          tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &maps.m[tl.g], u * (UB / 4), row0,
+                      &s.rfull[rs]);
           if (++rs == SR) {
             rs = 0;
             ++rnd;
@@ -623,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t t = pair; t < a.total_tiles; t += npairs, ++i) {
       const Tile tl = tile_of(a, t);
       const int64_t n = tl.n0 + r;
-      const bool n_ok = n < a.N;
+      const int64_t Ng = a.N[tl.g];
+      const bool n_ok = n < Ng;
       const int64_t m0 = tl.mt * a.tn;
       // before the wait: lane j holds 2^-s of token m0 + 32c + j for every
       // chunk c (0 for padding tokens), so the drain below has no loads
@@ -654,14 +676,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xffffffffu, my_scale[c], j)));
         const int64_t mc = m0 + 32 * c;
-        float *yp = a.y + (static_cast<int64_t>(tl.split) * a.M + mc) * a.N + n;
+        float *yp = a.y[tl.g] + static_cast<int64_t>(tl.split) * a.split_stride[tl.g] + mc * Ng + n;
         if (n_ok && mc + 32 <= a.M) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) yp[static_cast<int64_t>(j) * a.N] = __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) yp[static_cast<int64_t>(j) * Ng] = __uint_as_float(v[j]);
         } else if (n_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (mc + j < a.M) yp[static_cast<int64_t>(j) * a.N] = __uint_as_float(v[j]);
+            if (mc + j < a.M) yp[static_cast<int64_t>(j) * Ng] = __uint_as_float(v[j]);
         }
       }
     }
@@ -744,26 +766,28 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__
   }
 }
 
-// Split-K partials -> output, summed in split order (deterministic).
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ part, int64_t total, int splits,
-                                                            float *__restrict__ y) {
+// Split-K partials -> output, summed in split order (deterministic).  Split
+// s's partial of the M x N outputs starts at part + s * sstride, sstride =
+// total rounded up to a multiple of 4, so every split is float4-aligned.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restrict__ part, int64_t total,
+                                                            int64_t sstride, int splits, float *__restrict__ y) {
   pdl_trigger();
   pdl_wait();
-  const int64_t n4 = total / 4;
+  const int64_t n4 = total / 4, s4 = sstride / 4;
   const float4 *p4 = reinterpret_cast<const float4 *>(part);
   float4 *y4 = reinterpret_cast<float4 *>(y);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
     float4 acc = __ldg(p4 + i);
     for (int s = 1; s < splits; ++s) {
-      const float4 v = __ldg(p4 + static_cast<int64_t>(s) * n4 + i);
+      const float4 v = __ldg(p4 + static_cast<int64_t>(s) * s4 + i);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     y4[i] = acc;
   }
   for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     float acc = part[i];
-    for (int s = 1; s < splits; ++s) acc += part[static_cast<int64_t>(s) * total + i];
+    for (int s = 1; s < splits; ++s) acc += part[static_cast<int64_t>(s) * sstride + i];
     y[i] = acc;
   }
 }
@@ -807,6 +831,8 @@ struct Plan {
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
   unsigned grid;   // CTAs (2 per pair)
   size_t smem, x16_bytes, shift_off, part_off, total;
+  int64_t split_stride[kMaxGroup];   // floats per split of each weight's partials
+  size_t part_g_off[kMaxGroup];      // byte offset of each weight's partials
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -814,7 +840,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 constexpr size_t kSmemLimit = 227 * 1024;
 
 template <int TYPE>
-cudaError_t launch_pair(const CUtensorMap &map_w, const PrefillArgs &args, unsigned grid, size_t smem,
+cudaError_t launch_pair(const WeightMaps &maps, const PrefillArgs &args, unsigned grid, size_t smem,
                         cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
@@ -830,7 +856,7 @@ cudaError_t launch_pair(const CUtensorMap &map_w, const PrefillArgs &args, unsig
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<TYPE>, map_w, args);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<TYPE>, maps, args);
 }
 
 // How many CTA pairs of the GEMM kernel can be resident at once (clusters
@@ -872,13 +898,15 @@ int resident_pairs(int type, int tn, size_t smem, int sms) {
 }
 
 // pairs < 0: ask the device (needs a current device), else use that count
-Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
+// G weights of N[0..G-1] rows share the M x K activation.
+Plan make_plan(int type, int G, const int64_t *N, int64_t K, int64_t M, int sms, int pairs) {
   Plan p{};
   // tokens per pair tile: the smallest multiple of 32 that covers M, at most
   // 256 (the MMA's N; each CTA holds tn/2 of them)
   p.tn = M <= 256 ? static_cast<int>((M + 31) / 32 * 32) : 256;
   p.tiles_m = (M + p.tn - 1) / p.tn;
-  p.tiles_n = (N + kTileN - 1) / kTileN;
+  p.tiles_n = 0;
+  for (int g = 0; g < G; ++g) p.tiles_n += (N[g] + kTileN - 1) / kTileN;
   const int units = static_cast<int>(K / 256);
   // TMEM: tn accumulator columns, then up to 8 (an even number of) 32-column
   // weight stages
@@ -911,7 +939,14 @@ Plan make_plan(int type, int64_t N, int64_t K, int64_t M, int sms, int pairs) {
   p.x16_bytes = align_up(static_cast<size_t>(p.m_pad) * K * 2, 1024);
   p.shift_off = p.x16_bytes;
   p.part_off = align_up(p.shift_off + static_cast<size_t>(p.m_pad) * 4, 1024);
-  p.total = p.part_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * 4 : 0);
+  // split-K partials: per weight, splits x (M x N_g rounded up to 4 floats)
+  size_t off = p.part_off;
+  for (int g = 0; g < G; ++g) {
+    p.split_stride[g] = static_cast<int64_t>(align_up(static_cast<size_t>(M) * N[g], 4));
+    p.part_g_off[g] = off;
+    if (p.splits > 1) off += static_cast<size_t>(p.splits) * p.split_stride[g] * 4;
+  }
+  p.total = off;
   return p;
 }
 
@@ -940,11 +975,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int TYPE>
-int launch_gemm(const CUtensorMap &map_w, const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
+int launch_gemm(const WeightMaps &maps, const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
   const void *kern = reinterpret_cast<const void *>(prefill_kernel<TYPE>);
   const int rc = set_smem_once(kern, static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  const cudaError_t e = launch_pair<TYPE>(map_w, args, p.grid, p.smem, stream);
+  const cudaError_t e = launch_pair<TYPE>(maps, args, p.grid, p.smem, stream);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
@@ -952,70 +987,105 @@ int launch_gemm(const CUtensorMap &map_w, const PrefillArgs &args, const Plan &p
 }  // namespace
 }  // namespace dsq
 
-extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M) {
-  using namespace dsq;
-  if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || N < 1 || M < 1 || K < 256 || K % 256 != 0) return 0;
-  int sms = 148;
-  if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
-  return make_plan(type, N, K, M, sms, -1).total;
+namespace dsq {
+namespace {
+
+// Argument checks shared by the prefill entry points (nothing launched on
+// failure).
+int validate_group(const char *name, int type, int64_t G, const void *const *w, const int64_t *N, int64_t K,
+                   const float *x, int64_t M, float *const *y) {
+  DSQ_REQUIRE(G >= 1 && G <= kMaxGroup, DSQ_ERR_INVALID_ARG, "%s: G=%lld weights (1..%d supported)", name,
+              (long long)G, kMaxGroup);
+  DSQ_REQUIRE(w && N && y, DSQ_ERR_INVALID_ARG, "%s: null weight, size or output array", name);
+  int64_t total = 0;
+  for (int64_t g = 0; g < G; ++g) {
+    const int rc = validate(name, type, w[g], N[g], K, x, M);
+    if (rc != DSQ_OK) return rc;
+    DSQ_REQUIRE(y[g] != nullptr, DSQ_ERR_INVALID_ARG, "%s: null output %lld", name, (long long)g);
+    DSQ_REQUIRE(aligned(y[g], 16), DSQ_ERR_ALIGNMENT, "%s: y must be 16-byte aligned", name);
+    total += N[g];
+  }
+  DSQ_REQUIRE(total <= (int64_t(1) << 24), DSQ_ERR_SHAPE, "%s: the weights hold more than 2^24 rows", name);
+  return DSQ_OK;
 }
 
-extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
-                                void *workspace, size_t workspace_bytes, void *stream) {
-  using namespace dsq;
-  int rc = validate("dsq_gemm_prefill", type, w, N, K, x, M);
+size_t group_workspace_bytes(int type, int64_t G, const int64_t *N, int64_t K, int64_t M) {
+  if ((type != DSQ_Q8_0 && type != DSQ_Q4_K) || G < 1 || G > kMaxGroup || N == nullptr || M < 1 || K < 256 ||
+      K % 256 != 0)
+    return 0;
+  for (int64_t g = 0; g < G; ++g)
+    if (N[g] < 1) return 0;
+  int sms = 148;
+  if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
+  return make_plan(type, static_cast<int>(G), N, K, M, sms, -1).total;
+}
+
+// One activation conversion, one GEMM launch over the tiles of all G weights,
+// and (when K is split) one in-order reduction per weight.
+int run_prefill(const char *name, int type, int64_t G, const void *const *w, const int64_t *N, int64_t K,
+                const float *x, int64_t M, float *const *y, void *workspace, size_t workspace_bytes,
+                cudaStream_t st) {
+  int rc = validate_group(name, type, G, w, N, K, x, M, y);
   if (rc != DSQ_OK) return rc;
-  DSQ_REQUIRE(y != nullptr, DSQ_ERR_INVALID_ARG, "dsq_gemm_prefill: null output");
-  DSQ_REQUIRE(aligned(y, 16), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: y must be 16-byte aligned");
   WaitCtl ctl;
   int sms = 0;
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
-  const Plan p = make_plan(type, N, K, M, sms, -1);
+  const int Gi = static_cast<int>(G);
+  const Plan p = make_plan(type, Gi, N, K, M, sms, -1);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
-              "dsq_gemm_prefill: workspace of %zu bytes needed, %zu given", p.total, workspace_bytes);
-  DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "dsq_gemm_prefill: workspace must be 256-byte aligned");
-  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots >= 2 && p.slots_raw >= 2, DSQ_ERR_SHAPE,
-              "dsq_gemm_prefill: no pipeline fits");
+              "%s: workspace of %zu bytes needed, %zu given", name, p.total, workspace_bytes);
+  DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "%s: workspace must be 256-byte aligned", name);
+  DSQ_REQUIRE(p.smem <= kSmemLimit && p.slots >= 2 && p.slots_raw >= 2, DSQ_ERR_SHAPE, "%s: no pipeline fits",
+              name);
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   __half *x16 = reinterpret_cast<__half *>(ws);
   int32_t *shift = reinterpret_cast<int32_t *>(ws + p.shift_off);
-  float *part = reinterpret_cast<float *>(ws + p.part_off);
 
   // raw weight units: the packed rows viewed as uint32 [N][row_bytes/4], one
   // 256-element unit (68 or 36 words) x 128 rows per box; rows past N read as
   // zero (a zero block dequantizes to zero).  The kernel reads the weights
-  // only through this map.
+  // only through these maps.
   auto enc = encode_fn();
-  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "dsq_gemm_prefill: cuTensorMapEncodeTiled unavailable");
-  CUtensorMap map_w;
-  {
-    const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+  WeightMaps maps;
+  const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  for (int g = 0; g < Gi; ++g) {
     const cuuint32_t unit_words = type == DSQ_Q8_0 ? 68u : 36u;
-    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N)};
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N[g])};
     const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
     const cuuint32_t box[2] = {unit_words, static_cast<cuuint32_t>(kRows)};
     const cuuint32_t estride[2] = {1u, 1u};
-    const CUresult cr = enc(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w), gdim, gstride, box,
-                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    const CUresult cr = enc(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w[g]), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "dsq_gemm_prefill: weight tensor map (%d)", (int)cr);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "%s: weight tensor map %d (%d)", name, g, (int)cr);
   }
-  cudaStream_t st = as_stream(stream);
+  for (int g = Gi; g < kMaxGroup; ++g) maps.m[g] = maps.m[0];
+
   cudaError_t e = launch_pdl(x_to_f16_kernel<true>, dim3(static_cast<unsigned>(p.m_pad)), dim3(256), 0, st, x, M, K,
                              static_cast<int64_t>(p.tn / 2), x16, shift);
-  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: x_to_f16: %s", cudaGetErrorString(e));
-  rc = after_launch("dsq_gemm_prefill: x_to_f16");
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: x_to_f16: %s", name, cudaGetErrorString(e));
+  rc = after_launch(name);
   if (rc != DSQ_OK) return rc;
 
   PrefillArgs args{};
-  args.N = N;
   args.K = K;
   args.M = M;
+  args.G = Gi;
+  int64_t t0 = 0;
+  for (int g = 0; g < kMaxGroup; ++g) {
+    const bool used = g < Gi;
+    args.N[g] = used ? N[g] : 1;
+    args.y[g] = used ? (p.splits > 1 ? reinterpret_cast<float *>(ws + p.part_g_off[g]) : y[g]) : nullptr;
+    args.split_stride[g] = used ? p.split_stride[g] : 0;
+    args.tile_n0[g] = t0;
+    if (used) t0 += (N[g] + kTileN - 1) / kTileN;
+  }
+  args.tile_n0[kMaxGroup] = t0;
   args.x16 = x16;
   args.shift = shift;
-  args.y = p.splits > 1 ? part : y;
   args.units_per_split = p.units_per_split;
   args.splits = p.splits;
   args.tn = p.tn;
@@ -1025,18 +1095,51 @@ extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, c
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
   args.wait = ctl;
-  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(map_w, args, p, st) : launch_gemm<DSQ_Q4_K>(map_w, args, p, st);
+  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(maps, args, p, st) : launch_gemm<DSQ_Q4_K>(maps, args, p, st);
   if (rc != DSQ_OK) return rc;
   if (p.splits > 1) {
-    const int64_t total = M * N;
-    const int64_t blocks = (total / 4 + 255) / 256 + 1;
-    const unsigned grid = static_cast<unsigned>(blocks < 8 * sms ? blocks : 8 * sms);
-    e = launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(256), 0, st, static_cast<const float *>(part), total,
-                   p.splits, y);
-    if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: reduce: %s", cudaGetErrorString(e));
-    rc = after_launch("dsq_gemm_prefill: split-k reduce");
+    for (int g = 0; g < Gi; ++g) {
+      const int64_t total = M * N[g];
+      const int64_t blocks = (total / 4 + 255) / 256 + 1;
+      const unsigned grid = static_cast<unsigned>(blocks < 8 * sms ? blocks : 8 * sms);
+      e = launch_pdl(splitk_reduce_kernel, dim3(grid), dim3(256), 0, st,
+                     static_cast<const float *>(reinterpret_cast<float *>(ws + p.part_g_off[g])), total,
+                     p.split_stride[g], p.splits, y[g]);
+      if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: reduce: %s", name, cudaGetErrorString(e));
+      rc = after_launch(name);
+      if (rc != DSQ_OK) return rc;
+    }
   }
-  return rc;
+  return DSQ_OK;
+}
+
+}  // namespace
+}  // namespace dsq
+
+extern "C" size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M) {
+  return dsq::group_workspace_bytes(type, 1, &N, K, M);
+}
+
+extern "C" size_t dsq_prefill_grouped_workspace_bytes(int type, int64_t G, const int64_t *N, int64_t K, int64_t M) {
+  return dsq::group_workspace_bytes(type, G, N, K, M);
+}
+
+extern "C" int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M, float *y,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+  using namespace dsq;
+  DSQ_REQUIRE(y != nullptr, DSQ_ERR_INVALID_ARG, "dsq_gemm_prefill: null output");
+  const void *ws_[1] = {w};
+  float *ys_[1] = {y};
+  return run_prefill("dsq_gemm_prefill", type, 1, ws_, &N, K, x, M, ys_, workspace, workspace_bytes,
+                     as_stream(stream));
+}
+
+extern "C" int dsq_gemm_prefill_grouped(int type, int64_t G, const void *const *w, const int64_t *N, int64_t K,
+                                        const float *x, int64_t M, float *const *y, void *workspace,
+                                        size_t workspace_bytes, void *stream) {
+  using namespace dsq;
+  return run_prefill("dsq_gemm_prefill_grouped", type, G, w, N, K, x, M, y, workspace, workspace_bytes,
+                     as_stream(stream));
 }
 
 extern "C" int dsq_test_prefill_operands(int type, const void *w, int64_t N, int64_t K, const float *x, int64_t M,

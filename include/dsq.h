@@ -157,6 +157,26 @@ int dsq_gemv_grouped_f32(int type, const void *w, int64_t G, int64_t N,
                          int64_t K, const float *x, float *y, void *stream);
 
 /*
+ * Multi-token decode GEMV [ds4-621 GB10 report: the grouped-tok8 and
+ * QKV-pair paths for short batches of up to 8 tokens; ds4-623 Summary: the
+ * activation is prequantized to Q8 once and shared]: M = 1..8 prequantized
+ * activation rows against W0 (N0 rows) and, optionally, a second weight W1
+ * (N1 rows, same type and K; the Q / KV projections that read one input),
+ * in one launch that reads every weight byte once for all M tokens:
+ *   y0[m][n] = (W0 x_m)[n],  y1[m][n] = (W1 x_m)[n],  m < M.
+ * xq [M][K], xd [M][K/32], xs [M][K/32] (Q4_K only; may be NULL for Q8_0),
+ * y0 [M][N0], y1 [M][N1] (row-major, fp32).  Each token's outputs equal bit
+ * for bit those of dsq_gemv_q8_0 / dsq_gemv_q4_k / dsq_gemv_paired called
+ * for that token alone.  Either N may be 0 (its pointers are then unused).
+ * Requires K % 256 == 0, 1 <= M <= 8 and M * (K + K/8 (+ K/8 for Q4_K)) <=
+ * 65536 bytes (e.g. 8 tokens of K = 4096); otherwise DSQ_ERR_SHAPE and
+ * nothing is launched.  Weights 16-byte aligned, as for every GEMV.
+ */
+int dsq_gemv_tokens(int type, const void *w0, int64_t N0, const void *w1, int64_t N1,
+                    int64_t K, int64_t M, const int8_t *xq, const float *xd,
+                    const int32_t *xs, float *y0, float *y1, void *stream);
+
+/*
  * Prefill dequantize-into-dense-GEMM [ds4-621 GB10 report: "dequant + GEMM
  * prefill path"]:  Y[M][N] = X[M][K] * deq(W)^T, X fp32 row-major, Y fp32
  * row-major.  Tensor-core contraction with 16-bit float operands and fp32
@@ -187,6 +207,28 @@ int dsq_gemm_prefill(int type, const void *w, int64_t N, int64_t K,
                      void *workspace, size_t workspace_bytes, void *stream);
 
 size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M);
+
+/*
+ * Grouped prefill [ds4-621 consolidated results: the grouped attention-A
+ * prefill path, which computes several attention-A projections that read the
+ * same input in one launch]: G = 1..DSQ_PREFILL_MAX_GROUP weights of the same
+ * type and K (weight g: N[g] rows at w[g]) against ONE activation X [M][K]:
+ *   y[g][m][n] = (X * deq(W_g)^T)[m][n],   y[g] row-major [M][N[g]].
+ * X is converted to binary16 once and one GEMM launch covers the weight-row
+ * tiles of all G weights.  Numerics, layouts, alignment and errors are those
+ * of dsq_gemm_prefill for every weight; w, N and y are HOST arrays of G
+ * entries (the pointers in them are device pointers).  When the split of K
+ * is the same as for a weight alone (always for M > 256 on 148 SMs), each
+ * y[g] equals dsq_gemm_prefill's result for that weight bit for bit.
+ * workspace: at least dsq_prefill_grouped_workspace_bytes(type, G, N, K, M)
+ * bytes, 256-byte aligned.
+ */
+#define DSQ_PREFILL_MAX_GROUP 4
+int dsq_gemm_prefill_grouped(int type, int64_t G, const void *const *w, const int64_t *N,
+                             int64_t K, const float *x, int64_t M, float *const *y,
+                             void *workspace, size_t workspace_bytes, void *stream);
+size_t dsq_prefill_grouped_workspace_bytes(int type, int64_t G, const int64_t *N, int64_t K,
+                                           int64_t M);
 
 /*
  * Allocation-free prefill: dsq_gemm_prefill without a workspace argument.

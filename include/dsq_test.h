@@ -25,6 +25,14 @@ int dsq_test_block_sums(int type, const void *w, int64_t N, int64_t K,
                         float *y, int32_t *isum, void *stream);
 
 /*
+ * The multi-token GEMV (dsq_gemv_tokens, one weight) with its per-block int32
+ * dot products written out by the same device code: isum [M][N][K/32].
+ */
+int dsq_test_block_sums_tokens(int type, const void *w, int64_t N, int64_t K, int64_t M,
+                               const int8_t *xq, const float *xd, const int32_t *xs,
+                               float *y, int32_t *isum, void *stream);
+
+/*
  * Limit, in nanoseconds, of every bounded device wait launched from now on
  * (default 1e9).  0 makes each pipeline wait expire at once without
  * waiting, which exercises the timeout path: the kernel records

@@ -98,6 +98,26 @@ def test_host_side_validation(dsq):
     assert L.dsq_gemv_grouped_f32(8, A16, -1, 8, 256, A16, A16, None) == 1
     assert L.dsq_gemv_paired_f32(12, A16, 8, A16, 8, 256, A16 + 8, A16, A16, None) == 2
     assert L.dsq_gemv_paired_f32(8, None, 0, None, 0, 256, None, None, None, None) == 0   # empty: no-op
+    # the multi-token GEMV: token count, activation area, K, pointers
+    assert L.dsq_gemv_tokens(8, A16, 8, None, 0, 4096, 9, A16, A16, None, A16, None, None) == 3
+    assert L.dsq_gemv_tokens(8, A16, 8, None, 0, 4096, 0, A16, A16, None, A16, None, None) == 3
+    assert L.dsq_gemv_tokens(8, A16, 8, None, 0, 8192, 8, A16, A16, None, A16, None, None) == 3
+    assert L.dsq_gemv_tokens(12, A16, 8, None, 0, 288, 2, A16, A16, A16, A16, None, None) == 3
+    assert L.dsq_gemv_tokens(12, A16, 8, None, 0, 256, 2, A16, A16, None, A16, None, None) == 1
+    assert L.dsq_gemv_tokens(8, A16 + 8, 8, None, 0, 256, 2, A16, A16, None, A16, None, None) == 2
+    assert L.dsq_gemv_tokens(8, A16, 8, A16, 4, 256, 2, A16, A16, None, A16, None, None) == 1   # null y1
+    assert L.dsq_gemv_tokens(8, None, 0, None, 0, 256, 2, None, None, None, None, None, None) == 0
+    # the grouped prefill: weight count, sizes, host arrays
+    arr_p = (ctypes.c_void_p * 5)(*([A16] * 5))
+    arr_n = (ctypes.c_int64 * 5)(*([128] * 5))
+    assert L.dsq_gemm_prefill_grouped(8, 0, arr_p, arr_n, 256, A16, 4, arr_p, A16, 1 << 30, None) == 1
+    assert L.dsq_gemm_prefill_grouped(8, 5, arr_p, arr_n, 256, A16, 4, arr_p, A16, 1 << 30, None) == 1
+    assert L.dsq_gemm_prefill_grouped(8, 2, None, arr_n, 256, A16, 4, arr_p, A16, 1 << 30, None) == 1
+    assert L.dsq_gemm_prefill_grouped(8, 2, arr_p, arr_n, 96, A16, 4, arr_p, A16, 1 << 30, None) == 3
+    bad_n = (ctypes.c_int64 * 2)(128, 0)
+    assert L.dsq_gemm_prefill_grouped(8, 2, arr_p, bad_n, 256, A16, 4, arr_p, A16, 1 << 30, None) == 1
+    assert L.dsq_prefill_grouped_workspace_bytes(8, 2, bad_n, 256, 4) == 0
+    assert L.dsq_prefill_grouped_workspace_bytes(8, 5, arr_n, 256, 4) == 0
     # the allocation-free prefill names a bad argument before it looks at the
     # scratch size, even for a problem too large for its scratch
     big_m = 8192                                    # 8192 x 8192 x 2 B of fp16 activations > 32 MiB

@@ -33,13 +33,18 @@ def test_expired_waits_report_timeout_and_context_survives(dsq, ref):
         assert dsq.dsq_device_status() == 7
         dsq.dsq_gemv_paired(8, wg, N, wg, N, K, xqg, xdg, xsg, y, y)
         assert dsq.dsq_device_status() == 7
+        dsq.dsq_gemv_tokens(8, wg, N, None, 0, K, 1, xqg, xdg, None, y, None)
+        assert dsq.dsq_device_status() == 7
     finally:
         dsq.dsq_test_set_wait_limit_ns(2 ** 64 - 1)   # back to the default limit
     assert dsq.dsq_device_status() == 0                # the word was cleared
 
     dsq.dsq_gemv_q8_0(wg, N, K, xqg, xdg, y)
+    y_tok = torch.empty(N, dtype=torch.float32, device="cuda")
+    dsq.dsq_gemv_tokens(8, wg, N, None, 0, K, 1, xqg, xdg, None, y_tok, None)
     dsq.dsq_gemm_prefill(8, wg, N, K, xg, M, Y, ws, nbytes)
     assert dsq.dsq_device_status() == 0
+    assert torch.equal(y, y_tok)
     y_ref, absum = ref.gemv(8, w8, K, xq, xd, xs)
     assert gemv_error(y.cpu().numpy(), y_ref, absum, K // 32) <= GEMV_TOL
     Y64 = ref.prefill_f64(8, w8, K, x)

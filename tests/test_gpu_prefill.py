@@ -214,3 +214,71 @@ def test_prefill_weight_range_fails_closed(dsq, ref, qtype, args, bad):
     assert dsq.dsq_device_status() == (9 if bad else 0)
     assert np.isfinite(np.delete(y, 5, axis=1)).all()
     assert np.isfinite(y[:, 5]).all() != bad
+
+
+@pytest.mark.parametrize("qtype,N,K,M", [(8, 129, 4096, 3), (12, 255, 2048, 5), (8, 33, 1024, 1)])
+def test_prefill_split_k_ragged_outputs(dsq, ref, qtype, N, K, M):
+    """K split across many pair tiles with M x N not a multiple of 4: every
+    split's partials must be summed from the right place."""
+    w = ref.quantize(qtype, synth.weights(340 + N, N, K))
+    x = synth.activations(341 + M, M, K)
+    y = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    assert (M * N) % 4 != 0
+    assert rel_l2(y, ref.prefill_rounded(qtype, w, K, x, "f16")) <= PREFILL_ROUNDED_TOL
+    assert rel_l2(y, ref.prefill_f64(qtype, w, K, x)) <= PREFILL_TOL
+
+
+def _grouped(dsq, qtype, wgs, Ns, K, xg, M):
+    ys = [torch.full((M, n), float("nan"), dtype=torch.float32, device="cuda") for n in Ns]
+    nb = dsq.dsq_prefill_grouped_workspace_bytes(qtype, Ns, K, M)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    dsq.dsq_gemm_prefill_grouped(qtype, wgs, Ns, K, xg, M, ys, ws, nb)
+    torch.cuda.synchronize()
+    return ys
+
+
+@pytest.mark.parametrize("qtype,Ns,K,M", [(12, [300, 129, 256], 1024, 7), (8, [512, 64], 512, 40),
+                                          (8, [128, 200, 256, 77], 256, 300), (12, [1536], 1024, 33)])
+def test_prefill_grouped_parity(dsq, ref, qtype, Ns, K, M):
+    """Several weights sharing X in one launch (grouped attention-A prefill):
+    each output against the oracle's references for that weight."""
+    ws = [ref.quantize(qtype, synth.weights(350 + g, n, K)) for g, n in enumerate(Ns)]
+    x = synth.activations(351 + M, M, K)
+    x[min(1, M - 1)] *= 1e3
+    ys = _grouped(dsq, qtype, [to_dev(w) for w in ws], Ns, K, to_dev(x), M)
+    for w, y in zip(ws, ys):
+        yc = y.cpu().numpy()
+        assert np.isfinite(yc).all()
+        assert rel_l2(yc, ref.prefill_rounded(qtype, w, K, x, "f16")) <= PREFILL_ROUNDED_TOL
+        assert rel_l2(yc, ref.prefill_f64(qtype, w, K, x)) <= PREFILL_TOL
+
+
+@pytest.mark.parametrize("qtype", [8, 12])
+def test_prefill_grouped_equals_single_calls(dsq, ref, qtype):
+    """With the same split plan (no K split at M = 2048) a weight computed in a
+    group gets exactly the bits it gets alone; a sample is also checked against
+    the oracle."""
+    K, M, Ns = 4096, 2048, [2048, 1024]
+    ws = [ref.quantize(qtype, synth.weights(360 + g, n, K)) for g, n in enumerate(Ns)]
+    x = synth.activations(361, M, K)
+    wgs, xg = [to_dev(w) for w in ws], to_dev(x)
+    ys = _grouped(dsq, qtype, wgs, Ns, K, xg, M)
+    rng = np.random.default_rng(362)
+    ms = np.sort(rng.choice(M, size=24, replace=False))
+    for g, (w, n) in enumerate(zip(ws, Ns)):
+        y1 = torch.from_numpy(run_prefill(dsq, qtype, wgs[g], n, K, xg, M)).cuda()
+        assert torch.equal(ys[g], y1)
+        ns = np.sort(rng.choice(n, size=128, replace=False))
+        ys_c = ys[g].cpu().numpy()[np.ix_(ms, ns)]
+        assert rel_l2(ys_c, ref.prefill_rounded(qtype, w[ns], K, x[ms], "f16")) <= PREFILL_ROUNDED_TOL
+
+
+def test_prefill_grouped_refusals(dsq):
+    from block_quantized_dsq_b200 import DsqError
+    t = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    before = dsq.dsq_launch_count()
+    for ws, Ns, status in [([t] * 5, [128] * 5, 1), ([t, t], [128, 0], 1), ([t], [128], 5)]:
+        with pytest.raises(DsqError) as ei:
+            dsq.dsq_gemm_prefill_grouped(8, ws, Ns, 256, t, 4, [t] * len(ws), t, 0)
+        assert ei.value.status == status
+    assert dsq.dsq_launch_count() == before

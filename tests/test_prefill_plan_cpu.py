@@ -63,3 +63,23 @@ def test_workspace_grows_with_tokens_once_unsplit(dsq, qtype):
     sizes = [dsq.dsq_prefill_workspace_bytes(qtype, N, K, M) for M in (512, 1024, 2048, 4096)]
     assert all(a < b for a, b in zip(sizes, sizes[1:]))
     assert all(s >= M * K * 2 for s, M in zip(sizes, (512, 1024, 2048, 4096)))
+
+
+def test_split_partials_are_padded_to_whole_float4s(dsq):
+    # one 32-token tile x 1 weight tile, K = 4096: split 16 ways; M x N = 387
+    # floats per split are padded to 388 so every split starts float4-aligned
+    M, N, K = 3, 129, 4096
+    got = dsq.dsq_prefill_workspace_bytes(Q8, N, K, M)
+    assert got == _align(32 * K * 2, 1024) + _align(32 * 4, 1024) + 16 * 388 * 4
+
+
+def test_grouped_workspace_sums_the_weights_partials(dsq):
+    # G = 2 weights of 512 and 128 rows at M = 64: one 64-token tile x 3
+    # weight tiles, K split 16 ways (3 x 16 x 2 = 96 > 74 pairs stops the
+    # doubling at 16 = the 16 units of K); each weight's partials apart
+    M, K, Ns = 64, 4096, [512, 128]
+    got = dsq.dsq_prefill_grouped_workspace_bytes(Q8, Ns, K, M)
+    base = _align(M * K * 2, 1024) + _align(M * 4, 1024)
+    assert got == base + 16 * (M * 512 + M * 128) * 4
+    # a group of one is the single-weight plan
+    assert dsq.dsq_prefill_grouped_workspace_bytes(Q8, [512], K, M) == dsq.dsq_prefill_workspace_bytes(Q8, 512, K, M)
