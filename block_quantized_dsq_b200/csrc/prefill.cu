@@ -825,6 +825,273 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
   pair_to_f16<TYPE, 1>(unit, dst, status);
 }
 
+// ------------------------------------------------------ small-M bridge --
+// For one to three tokens the tensor-core pipeline is all fill and drain: the
+// weights stream once, but three launches (activation rounding, GEMM, split
+// reduction) and the pair pipeline's start-up dominate.  Those token counts
+// (small_max_m below, chosen from the measured sweep) take this CUDA-core
+// kernel instead, with the same operands: every
+// activation row rounded to binary16 after the same exact 2^s_m scaling,
+// every weight element dequantized by the converter's own functions, each
+// product exact in fp32, fp32 sums, the result scaled back by 2^-s_m.
+//  * One launch.  Each CTA copies the M fp32 activation rows into shared
+//    memory, finds the row shifts and rounds the rows in place, while its
+//    first weight boxes are in flight.
+//  * lane = weight row: a warp takes 32 rows of one weight, one 256-element
+//    unit at a time (a 2-D TMA box of 32 rows x 272 / 144 B); warp w takes the
+//    units u = w, w+8, ...; all lanes read the same activation values
+//    (broadcast), two K elements per paired fp32 FMA.
+//  * The 8 warps' partial sums meet in shared memory in a fixed order.
+constexpr int kSmallMaxM = 3;
+constexpr int kSmallWarps = 8;
+constexpr int kSmallRows = 32;
+constexpr size_t kSmallMaxActSmem = 128 * 1024;
+constexpr size_t kSmallPipeSmem = 227 * 1024;   // dynamic shared memory the kernel may take
+
+struct SmallArgs {
+  int64_t K, M;
+  int G;
+  int64_t N[kMaxGroup];
+  float *y[kMaxGroup];
+  int64_t group0[kMaxGroup + 1];   // first 32-row group of each weight
+  int64_t total_groups;
+  const float *x;                  // [M][K] fp32
+  int nunits, stages;
+  uint32_t box_bytes, ring_off, bar_off, red_off;
+  WaitCtl wait;
+};
+
+// Item position of a warp: row group g, unit u (warp, warp + 8, ...).
+struct SmallCursor {
+  int64_t g;
+  int u;
+  __device__ __forceinline__ void first(const SmallArgs &a, int warp) {
+    g = blockIdx.x;
+    u = warp;
+    if (u >= a.nunits) g = a.total_groups;
+  }
+  __device__ __forceinline__ void next(const SmallArgs &a, int warp) {
+    u += kSmallWarps;
+    if (u >= a.nunits) {
+      u = warp;
+      g += gridDim.x;
+    }
+  }
+  __device__ __forceinline__ bool valid(const SmallArgs &a) const { return g < a.total_groups; }
+};
+
+__device__ __forceinline__ int small_weight_of(const SmallArgs &a, int64_t g) {
+  int w = 0;
+  while (w + 1 < a.G && g >= a.group0[w + 1]) ++w;
+  return w;
+}
+
+template <int UB>
+__device__ __forceinline__ void small_issue(const WeightMaps &maps, const SmallArgs &a, const SmallCursor &c,
+                                            uint8_t *dst, uint64_t *bar) {
+  const int w = small_weight_of(a, c.g);
+  const int32_t row0 = static_cast<int32_t>((c.g - a.group0[w]) * kSmallRows);
+  mbar_arrive_expect_tx(bar, a.box_bytes);
+  tma_load_2d(dst, &maps.m[w], c.u * (UB / 4), row0, bar);
+}
+
+// acc2[m] (two fp32 lanes: even and odd K) += w16[k .. k+63] * x[m][k .. k+63]
+// for one 64-element piece whose binary16 weights are the 32 words `piece`.
+template <int M>
+__device__ __forceinline__ void small_piece_fma(const uint32_t (&piece)[32], const float *xk, int64_t K,
+                                                uint64_t (&acc2)[M]) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {   // 4 elements per step
+    const float2 w01 = __half22float2(bits_h2(piece[2 * c]));
+    const float2 w23 = __half22float2(bits_h2(piece[2 * c + 1]));
+    const uint64_t wa = pack2(w01.x, w01.y), wb = pack2(w23.x, w23.y);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const float4 xv = *reinterpret_cast<const float4 *>(xk + m * K + 4 * c);
+      acc2[m] = fma2_rn(wa, pack2(xv.x, xv.y), acc2[m]);
+      acc2[m] = fma2_rn(wb, pack2(xv.z, xv.w), acc2[m]);
+    }
+  }
+}
+
+// The binary16 range guard of pair_in_range for a whole 256-element unit
+// held as NV uint4 granules.
+template <int TYPE, int NV>
+__device__ __forceinline__ bool unit_in_range(const uint4 (&v)[NV]) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+    uint32_t worst = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int wd = (b & 1) ? (17 * b - 1) / 2 : 17 * b / 2;   // word holding block b's scale
+      const uint32_t w = word4(v[wd >> 2], wd & 3);
+      worst = max(worst, ((b & 1) ? (w >> 16) : w) & 0x7fffu);
+    }
+    return worst < 0x6008u;
+  } else {
+    PairRegs<DSQ_Q4_K> r;
+    r.hdr = v[0];
+    return pair_in_range<DSQ_Q4_K, 0>(r) && pair_in_range<DSQ_Q4_K, 1>(r);
+  }
+}
+
+template <int TYPE, int M>
+__device__ __forceinline__ void small_unit(const uint8_t *p, const float *xf, int64_t K, int u, uint64_t (&acc2)[M],
+                                           uint32_t *status) {
+  constexpr int NV = TYPE == DSQ_Q8_0 ? 17 : 9;
+  uint4 v[NV];
+  const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = p4[i];
+  if (!unit_in_range<TYPE, NV>(v)) record_range(status);
+  const float *xu = xf + static_cast<int64_t>(u) * 256;
+#pragma unroll
+  for (int P = 0; P < 4; ++P) {
+    uint32_t piece[32];
+    if constexpr (TYPE == DSQ_Q8_0) {
+      piece_q8_0([&](int i) { return word4(v[(17 * P + i) >> 2], (17 * P + i) & 3); }, piece);
+    } else {
+      if (P == 0) piece_q4_k<0>(v[0], [&](int i) { return word4(v[1 + (i >> 2)], i & 3); }, piece);
+      if (P == 1) piece_q4_k<1>(v[0], [&](int i) { return word4(v[3 + (i >> 2)], i & 3); }, piece);
+      if (P == 2) piece_q4_k<2>(v[0], [&](int i) { return word4(v[5 + (i >> 2)], i & 3); }, piece);
+      if (P == 3) piece_q4_k<3>(v[0], [&](int i) { return word4(v[7 + (i >> 2)], i & 3); }, piece);
+    }
+    small_piece_fma<M>(piece, xu + 64 * P, K, acc2);
+  }
+}
+
+template <int TYPE, int M>
+__global__ void __launch_bounds__(kSmallWarps * 32, 1)
+    prefill_small_kernel(const __grid_constant__ WeightMaps maps, const __grid_constant__ SmallArgs a) {
+  constexpr int UB = unit_bytes<TYPE>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.stages;
+  const int64_t K = a.K;
+  float *xf = reinterpret_cast<float *>(base);   // [M][K]
+  uint8_t *ring = base + a.ring_off + static_cast<size_t>(warp) * S * a.box_bytes;
+  uint64_t *act_bar = reinterpret_cast<uint64_t *>(base + a.bar_off);
+  uint64_t *bars = act_bar + 1 + warp * 2;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(act_bar + 1 + 2 * kSmallWarps);
+  __shared__ float row_scale[kSmallMaxM], scale_back[kSmallMaxM];   // 2^s_m and 2^-s_m
+  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][8 warps][M][32]
+
+  if (threadIdx.x == 0) {
+    mbar_init(act_bar, 1);
+    *abort_flag = 0u;
+    for (int w = 0; w < a.G; ++w) prefetch_tensormap(&maps.m[w]);
+  }
+  if (lane == 0)
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+  fence_barrier_init();
+  SmallCursor issue;
+  issue.first(a, warp);
+  if (lane == 0) {
+    // weights are read-only: this warp's first boxes toward L2 while the
+    // kernel before us finishes
+    SmallCursor c = issue;
+    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp)) {
+      const int w = small_weight_of(a, c.g);
+      prefetch_l2_tile_2d(&maps.m[w], c.u * (UB / 4), static_cast<int32_t>((c.g - a.group0[w]) * kSmallRows));
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(act_bar, static_cast<uint32_t>(M * K * 4));
+    bulk_g2s(xf, a.x, static_cast<uint32_t>(M * K * 4), act_bar, l2_policy_evict_last());
+  }
+  int64_t n_issued = 0, n_waited = 0;
+  if (lane == 0)
+    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp), ++n_issued)
+      small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(s) * a.box_bytes, &bars[s]);
+  bool ok = __all_sync(0xffffffffu, mbar_wait_for(act_bar, 0, a.wait.limit_ns));
+  if (!ok && lane == 0 && *abort_flag == 0u) {
+    *abort_flag = 1u;
+    record_timeout(a.wait);
+  }
+  // row shifts (warp m takes row m), then every element rounded in place:
+  // float(binary16_rne(x * 2^s_m)), exactly as the tensor-core path rounds it
+  if (warp < M) {
+    float amax = 0.0f;
+    if (ok)
+      for (int64_t k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(xf[warp * K + k]));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int sft = 0;
+    if (amax > 0.0f && !isinf(amax)) {
+      int e;
+      frexpf(amax, &e);
+      sft = min(126, max(-113, 15 - e));
+    }
+    if (lane == 0) {
+      row_scale[warp] = __int_as_float((127 + sft) << 23);
+      scale_back[warp] = __int_as_float((127 - sft) << 23);
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    for (int m = 0; m < M; ++m) {
+      const float sc = row_scale[m];
+      for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
+        xf[m * K + k] = __half2float(__float2half_rn(__fmul_rn(xf[m * K + k], sc)));
+    }
+  }
+  __syncthreads();
+
+  int slot = 0;
+  uint32_t parity = 0;
+  int buf = 0;
+  for (int64_t g = blockIdx.x; g < a.total_groups; g += gridDim.x, buf ^= 1) {
+    uint64_t acc2[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) acc2[m] = 0ull;
+    for (int u = warp; u < a.nunits; u += kSmallWarps) {
+      ok = ok && *abort_flag == 0u;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
+      if (!ok) {
+        if (lane == 0 && *abort_flag == 0u) {
+          *abort_flag = 1u;
+          record_timeout(a.wait);
+        }
+      } else {
+        ++n_waited;
+        small_unit<TYPE, M>(ring + static_cast<size_t>(slot) * a.box_bytes + static_cast<size_t>(lane) * UB, xf, K,
+                            u, acc2, a.wait.status);
+        __syncwarp();
+        if (lane == 0 && issue.valid(a)) {
+          fence_proxy_async_smem();
+          small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(slot) * a.box_bytes, &bars[slot]);
+          issue.next(a, warp);
+          ++n_issued;
+        }
+      }
+      if (++slot == S) {
+        slot = 0;
+        parity ^= 1u;
+      }
+    }
+    float *rb = red + static_cast<size_t>(buf) * kSmallWarps * M * 32;
+#pragma unroll
+    for (int m = 0; m < M; ++m) rb[(warp * M + m) * 32 + lane] = __fadd_rn(lo_of(acc2[m]), hi_of(acc2[m]));
+    __syncthreads();
+    for (int m = warp; m < M; m += kSmallWarps) {
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kSmallWarps; ++w) v += rb[(w * M + m) * 32 + lane];
+      const int wi = small_weight_of(a, g);
+      const int64_t row = (g - a.group0[wi]) * kSmallRows + lane;
+      if (row < a.N[wi] && *abort_flag == 0u) a.y[wi][m * a.N[wi] + row] = __fmul_rn(v, scale_back[m]);
+    }
+  }
+  if (lane == 0)
+    for (int64_t k = n_waited; k < n_issued; ++k)
+      mbar_wait_for(&bars[k % S], static_cast<uint32_t>((k / S) & 1), kDrainLimitNs);
+  if (threadIdx.x == 0 && !ok) mbar_wait_for(act_bar, 0, kDrainLimitNs);
+}
+
 // ------------------------------------------------------------------- host --
 struct Plan {
   int tn, slots, slots_raw, splits, units_per_split;
@@ -990,6 +1257,115 @@ int launch_gemm(const WeightMaps &maps, const PrefillArgs &args, const Plan &p, 
 namespace dsq {
 namespace {
 
+// ---- small-M bridge: plan and launch ----
+// The workspace the small-M kernel asks for (it keeps its activations in
+// shared memory and needs none; a token amount keeps the API uniform).
+constexpr size_t kSmallWorkspace = 256;
+
+size_t small_act_bytes(int64_t K, int64_t M) { return static_cast<size_t>(M) * K * 4; }
+
+// Where the small-M kernel beats the tensor-core pipeline (measured on B200
+// with K = 4096: Q4_K up to 3 tokens, 8.6 / 10.6 us against 15.7 us at 1 / 2
+// tokens for 4096 rows; Q8_0 up to 2 tokens, 13.9 / 17.2 us against 19.2 /
+// 19.5 us for 8192 rows; from 4 tokens on its CUDA-core products cost more
+// than the tensor-core pipeline's fixed start-up).
+int small_max_m(int type) { return type == DSQ_Q4_K ? 3 : 2; }   // at most kSmallMaxM
+
+bool small_fits(int type, int64_t K, int64_t M) {
+  return M >= 1 && M <= small_max_m(type) && small_act_bytes(K, M) <= kSmallMaxActSmem;
+}
+
+template <int TYPE, int M>
+cudaError_t small_launch(const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem, cudaStream_t st) {
+  return launch_pdl(prefill_small_kernel<TYPE, M>, dim3(grid), dim3(kSmallWarps * 32), smem, st, maps, a);
+}
+
+template <int TYPE>
+const void *small_kernel_ptr(int M) {
+  switch (M) {
+    case 1: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 1>);
+    case 2: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 2>);
+    default: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 3>);
+  }
+}
+
+template <int TYPE>
+cudaError_t small_dispatch(int M, const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem,
+                           cudaStream_t st) {
+  switch (M) {
+    case 1: return small_launch<TYPE, 1>(maps, a, grid, smem, st);
+    case 2: return small_launch<TYPE, 2>(maps, a, grid, smem, st);
+    default: return small_launch<TYPE, 3>(maps, a, grid, smem, st);
+  }
+}
+
+int run_prefill_small(const char *name, int type, int G, const void *const *w, const int64_t *N, int64_t K,
+                      const float *x, int64_t M, float *const *y, void *workspace, size_t workspace_bytes,
+                      const WaitCtl &ctl, int sms, cudaStream_t st) {
+  DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= kSmallWorkspace, DSQ_ERR_WORKSPACE,
+              "%s: workspace of %zu bytes needed, %zu given", name, kSmallWorkspace, workspace_bytes);
+  DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "%s: workspace must be 256-byte aligned", name);
+  SmallArgs a{};
+  a.K = K;
+  a.M = M;
+  a.G = G;
+  int64_t g0 = 0;
+  for (int g = 0; g < kMaxGroup; ++g) {
+    const bool used = g < G;
+    a.N[g] = used ? N[g] : 1;
+    a.y[g] = used ? y[g] : nullptr;
+    a.group0[g] = g0;
+    if (used) g0 += (N[g] + kSmallRows - 1) / kSmallRows;
+  }
+  a.group0[kMaxGroup] = g0;
+  a.total_groups = g0;
+  a.x = x;
+  a.nunits = static_cast<int>(K / 256);
+  a.box_bytes = static_cast<uint32_t>(kSmallRows * (type == DSQ_Q8_0 ? 272 : 144));
+  a.wait = ctl;
+  // shared memory: activations [M][K] fp32 | ring (8 warps x stages x box) |
+  // barriers | reduction [2][8][M][32]
+  const size_t act = align_up(small_act_bytes(K, M), 1024);
+  const size_t bars = align_up((1 + 2 * kSmallWarps + 1) * sizeof(uint64_t), 128);
+  const size_t red = 2 * static_cast<size_t>(kSmallWarps) * M * 32 * sizeof(float);
+  const size_t fixed = 1024 + act + bars + red + 2 * kSmallMaxM * sizeof(float);
+  const size_t per_stage = static_cast<size_t>(kSmallWarps) * a.box_bytes;
+  int stages = fixed < kSmallPipeSmem ? static_cast<int>((kSmallPipeSmem - fixed) / per_stage) : 0;
+  if (stages > 2) stages = 2;
+  DSQ_REQUIRE(stages >= 1, DSQ_ERR_SHAPE, "%s: no pipeline fits next to %lld tokens of K=%lld", name, (long long)M,
+              (long long)K);
+  a.stages = stages;
+  a.ring_off = static_cast<uint32_t>(act);
+  a.bar_off = static_cast<uint32_t>(act + per_stage * stages);
+  a.red_off = static_cast<uint32_t>(a.bar_off + bars);
+  const size_t smem = 1024 + a.red_off + red;
+
+  auto enc = encode_fn();
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+  WeightMaps maps;
+  const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  for (int g = 0; g < G; ++g) {
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N[g])};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {type == DSQ_Q8_0 ? 68u : 36u, static_cast<cuuint32_t>(kSmallRows)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w[g]), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "%s: weight tensor map %d (%d)", name, g, (int)cr);
+  }
+  for (int g = G; g < kMaxGroup; ++g) maps.m[g] = maps.m[0];
+  const int mi = static_cast<int>(M);
+  const int rc = set_smem_once(type == DSQ_Q8_0 ? small_kernel_ptr<DSQ_Q8_0>(mi) : small_kernel_ptr<DSQ_Q4_K>(mi),
+                               static_cast<int>(smem), name);
+  if (rc != DSQ_OK) return rc;
+  const unsigned grid = static_cast<unsigned>(a.total_groups < sms ? a.total_groups : sms);
+  const cudaError_t e = type == DSQ_Q8_0 ? small_dispatch<DSQ_Q8_0>(mi, maps, a, grid, smem, st)
+                                         : small_dispatch<DSQ_Q4_K>(mi, maps, a, grid, smem, st);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: %s", name, cudaGetErrorString(e));
+  return after_launch(name);
+}
+
 // Argument checks shared by the prefill entry points (nothing launched on
 // failure).
 int validate_group(const char *name, int type, int64_t G, const void *const *w, const int64_t *N, int64_t K,
@@ -1015,6 +1391,7 @@ size_t group_workspace_bytes(int type, int64_t G, const int64_t *N, int64_t K, i
     return 0;
   for (int64_t g = 0; g < G; ++g)
     if (N[g] < 1) return 0;
+  if (small_fits(type, K, M)) return kSmallWorkspace;
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
   return make_plan(type, static_cast<int>(G), N, K, M, sms, -1).total;
@@ -1032,6 +1409,8 @@ int run_prefill(const char *name, int type, int64_t G, const void *const *w, con
   rc = wait_ctl(&ctl, &sms);
   if (rc != DSQ_OK) return rc;
   const int Gi = static_cast<int>(G);
+  if (small_fits(type, K, M))
+    return run_prefill_small(name, type, Gi, w, N, K, x, M, y, workspace, workspace_bytes, ctl, sms, st);
   const Plan p = make_plan(type, Gi, N, K, M, sms, -1);
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "%s: workspace of %zu bytes needed, %zu given", name, p.total, workspace_bytes);

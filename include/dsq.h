@@ -217,8 +217,9 @@ size_t dsq_prefill_workspace_bytes(int type, int64_t N, int64_t K, int64_t M);
  * X is converted to binary16 once and one GEMM launch covers the weight-row
  * tiles of all G weights.  Numerics, layouts, alignment and errors are those
  * of dsq_gemm_prefill for every weight; w, N and y are HOST arrays of G
- * entries (the pointers in them are device pointers).  When the split of K
- * is the same as for a weight alone (always for M > 256 on 148 SMs), each
+ * entries (the pointers in them are device pointers).  The split of K (if
+ * any) is planned over all G weights' tiles together; whenever it comes out
+ * the same as for a weight alone -- in particular when neither splits K --
  * y[g] equals dsq_gemm_prefill's result for that weight bit for bit.
  * workspace: at least dsq_prefill_grouped_workspace_bytes(type, G, N, K, M)
  * bytes, 256-byte aligned.

@@ -31,6 +31,8 @@ def test_expired_waits_report_timeout_and_context_survives(dsq, ref):
         assert dsq.dsq_device_status() == 7            # DSQ_ERR_TIMEOUT
         dsq.dsq_gemm_prefill(8, wg, N, K, xg, M, Y, ws, nbytes)
         assert dsq.dsq_device_status() == 7
+        dsq.dsq_gemm_prefill(8, wg, N, K, xg, 2, Y, ws, nbytes)      # the small-M kernel
+        assert dsq.dsq_device_status() == 7
         dsq.dsq_gemv_paired(8, wg, N, wg, N, K, xqg, xdg, xsg, y, y)
         assert dsq.dsq_device_status() == 7
         dsq.dsq_gemv_tokens(8, wg, N, None, 0, K, 1, xqg, xdg, None, y, None)
@@ -42,9 +44,13 @@ def test_expired_waits_report_timeout_and_context_survives(dsq, ref):
     dsq.dsq_gemv_q8_0(wg, N, K, xqg, xdg, y)
     y_tok = torch.empty(N, dtype=torch.float32, device="cuda")
     dsq.dsq_gemv_tokens(8, wg, N, None, 0, K, 1, xqg, xdg, None, y_tok, None)
+    Y4 = torch.empty((2, N), dtype=torch.float32, device="cuda")
+    dsq.dsq_gemm_prefill(8, wg, N, K, xg, 2, Y4, ws, nbytes)
     dsq.dsq_gemm_prefill(8, wg, N, K, xg, M, Y, ws, nbytes)
     assert dsq.dsq_device_status() == 0
     assert torch.equal(y, y_tok)
+    Y64_4 = ref.prefill_f64(8, w8, K, x[:2])
+    assert np.linalg.norm(Y4.cpu().numpy() - Y64_4) / np.linalg.norm(Y64_4) <= PREFILL_TOL
     y_ref, absum = ref.gemv(8, w8, K, xq, xd, xs)
     assert gemv_error(y.cpu().numpy(), y_ref, absum, K // 32) <= GEMV_TOL
     Y64 = ref.prefill_f64(8, w8, K, x)

@@ -32,7 +32,11 @@ def run_prefill(dsq, qtype, wg, N, K, xg, M):
 
 
 CASES = [(8, 128, 256, 1), (8, 256, 512, 5), (12, 300, 512, 33), (8, 128, 4096, 128), (12, 384, 1024, 200),
-         (8, 640, 2048, 70), (12, 128, 768, 257), (8, 200, 256, 513), (12, 4096, 4096, 3), (8, 1024, 512, 1100)]
+         (8, 640, 2048, 70), (12, 128, 768, 257), (8, 200, 256, 513), (12, 4096, 4096, 3), (8, 1024, 512, 1100),
+         # M <= 2 (Q8_0) / 3 (Q4_K) takes the small-M kernel; up to 32 the
+         # narrowest tensor-core tile
+         (8, 4096, 4096, 8), (12, 1000, 2048, 3), (8, 33, 16384, 2), (12, 300, 512, 9), (8, 256, 512, 17),
+         (8, 700, 1024, 2), (12, 64, 256, 1)]
 
 
 @pytest.mark.parametrize("qtype,N,K,M", CASES)
@@ -68,7 +72,7 @@ def test_prefill_operands_bit_exact(dsq, ref, qtype, N, K, M):
 
 
 @pytest.mark.parametrize("qtype,N,M", [(12, 4096, 128), (12, 4096, 512), (12, 4096, 2048),
-                                       (8, 8192, 128), (8, 8192, 512), (8, 8192, 2048)])
+                                       (8, 8192, 128), (8, 8192, 512), (8, 8192, 2048), (12, 4096, 3), (8, 8192, 2)])
 def test_prefill_workload_sampled(dsq, ref, qtype, N, M):
     """Full workload sizes (K = 4096), in the configuration the bench times;
     the oracle recomputes a sample of 48 tokens x 256 weight rows."""
@@ -196,12 +200,13 @@ RANGE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("M", [2, 40])            # the small-M kernel and the tensor-core kernel
 @pytest.mark.parametrize("qtype,args,bad", RANGE_CASES)
-def test_prefill_weight_range_fails_closed(dsq, ref, qtype, args, bad):
+def test_prefill_weight_range_fails_closed(dsq, ref, qtype, args, bad, M):
     """A weight block whose dequantized values leave the binary16 range makes
     the kernels record DSQ_ERR_RANGE; a block just inside the bound does not.
     Either way the operand bits equal the oracle's (inf where it overflows)."""
-    N, K, M = 128, 256, 8
+    N, K = 128, 256
     w = _q8_0_row_with_block(ref, N, K, *args) if qtype == 8 else _q4_k_row_with_subblock(ref, N, K, *args)
     x = synth.activations(336, M, K)
     got, want, status = _operands_and_status(dsq, ref, qtype, w, K, x)
@@ -216,7 +221,7 @@ def test_prefill_weight_range_fails_closed(dsq, ref, qtype, args, bad):
     assert np.isfinite(y[:, 5]).all() != bad
 
 
-@pytest.mark.parametrize("qtype,N,K,M", [(8, 129, 4096, 3), (12, 255, 2048, 5), (8, 33, 1024, 1)])
+@pytest.mark.parametrize("qtype,N,K,M", [(8, 129, 4096, 9), (12, 255, 2048, 11), (8, 33, 1024, 13)])
 def test_prefill_split_k_ragged_outputs(dsq, ref, qtype, N, K, M):
     """K split across many pair tiles with M x N not a multiple of 4: every
     split's partials must be summed from the right place."""
@@ -238,7 +243,8 @@ def _grouped(dsq, qtype, wgs, Ns, K, xg, M):
 
 
 @pytest.mark.parametrize("qtype,Ns,K,M", [(12, [300, 129, 256], 1024, 7), (8, [512, 64], 512, 40),
-                                          (8, [128, 200, 256, 77], 256, 300), (12, [1536], 1024, 33)])
+                                          (8, [128, 200, 256, 77], 256, 300), (12, [1536], 1024, 33),
+                                          (12, [300, 129, 256], 1024, 19), (8, [64, 1000], 4096, 2)])
 def test_prefill_grouped_parity(dsq, ref, qtype, Ns, K, M):
     """Several weights sharing X in one launch (grouped attention-A prefill):
     each output against the oracle's references for that weight."""
@@ -255,10 +261,11 @@ def test_prefill_grouped_parity(dsq, ref, qtype, Ns, K, M):
 
 @pytest.mark.parametrize("qtype", [8, 12])
 def test_prefill_grouped_equals_single_calls(dsq, ref, qtype):
-    """With the same split plan (no K split at M = 2048) a weight computed in a
-    group gets exactly the bits it gets alone; a sample is also checked against
-    the oracle."""
-    K, M, Ns = 4096, 2048, [2048, 1024]
+    """With the same split plan a weight computed in a group gets exactly the
+    bits it gets alone: at M = 2048 neither 2048 rows (64 pair tiles) nor 2304
+    rows (72) nor both together split K on 74 SM pairs.  A sample is also
+    checked against the oracle."""
+    K, M, Ns = 4096, 2048, [2048, 2304]
     ws = [ref.quantize(qtype, synth.weights(360 + g, n, K)) for g, n in enumerate(Ns)]
     x = synth.activations(361, M, K)
     wgs, xg = [to_dev(w) for w in ws], to_dev(x)
@@ -282,3 +289,18 @@ def test_prefill_grouped_refusals(dsq):
             dsq.dsq_gemm_prefill_grouped(8, ws, Ns, 256, t, 4, [t] * len(ws), t, 0)
         assert ei.value.status == status
     assert dsq.dsq_launch_count() == before
+
+
+@pytest.mark.parametrize("qtype,N,K,M", [(12, 4000, 1024, 300), (8, 2000, 2048, 700)])
+def test_prefill_two_way_split_is_deterministic(dsq, ref, qtype, N, K, M):
+    """K split in two: the partials are summed in split order, so two calls
+    give the same bits."""
+    tiles = -(-M // 256) * -(-N // 256)
+    assert 2 * tiles <= 74 < 4 * tiles          # the planner splits K in two on 74 SM pairs
+    w = ref.quantize(qtype, synth.weights(370 + N, N, K))
+    x = synth.activations(371 + M, M, K)
+    y1 = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    y2 = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    assert np.array_equal(y1, y2)
+    assert rel_l2(y1, ref.prefill_rounded(qtype, w, K, x, "f16")) <= PREFILL_ROUNDED_TOL
+    assert rel_l2(y1, ref.prefill_f64(qtype, w, K, x)) <= PREFILL_TOL

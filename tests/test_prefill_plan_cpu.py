@@ -66,11 +66,24 @@ def test_workspace_grows_with_tokens_once_unsplit(dsq, qtype):
 
 
 def test_split_partials_are_padded_to_whole_float4s(dsq):
-    # one 32-token tile x 1 weight tile, K = 4096: split 16 ways; M x N = 387
-    # floats per split are padded to 388 so every split starts float4-aligned
-    M, N, K = 3, 129, 4096
+    # one 32-token tile x 1 weight tile, K = 4096: split 16 ways; M x N = 1161
+    # floats per split are padded to 1164 so every split starts float4-aligned
+    M, N, K = 9, 129, 4096
     got = dsq.dsq_prefill_workspace_bytes(Q8, N, K, M)
-    assert got == _align(32 * K * 2, 1024) + _align(32 * 4, 1024) + 16 * 388 * 4
+    assert got == _align(32 * K * 2, 1024) + _align(32 * 4, 1024) + 16 * 1164 * 4
+
+
+@pytest.mark.parametrize("qtype,max_m", [(Q8, 2), (Q4, 3)])
+def test_a_few_tokens_take_the_small_kernel(dsq, qtype, max_m):
+    # up to 2 (Q8_0) or 3 (Q4_K) tokens, with M x K x 4 bytes of activations
+    # <= 128 KB, run the CUDA-core kernel, which keeps its activations in
+    # shared memory: the workspace is a token 256 bytes
+    for M in range(1, max_m + 1):
+        assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 4096, M) == 256
+    assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 4096, max_m + 1) > 256
+    assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 16384, 2) == 256     # exactly 128 KB
+    assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 16640, 2) > 256      # 130 KB of activations
+    assert dsq.dsq_prefill_grouped_workspace_bytes(qtype, [512, 64], 4096, 2) == 256
 
 
 def test_grouped_workspace_sums_the_weights_partials(dsq):
