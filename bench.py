@@ -15,6 +15,7 @@ dequant-GEMM TFLOP/s sweep, the CPU oracle baseline and clock samples.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -681,6 +682,43 @@ def measure_rows(dsq, L, stream, hbm_peak, bf16_peak, only=None):
             rows[f"prefill_{tag}_m{M}"] = row
             del x, y, wsp
         del ws, w
+    # grouped attention-A prefill: two Q4_K weights (4096 and 1024 rows) that
+    # read the same X, one launch against two back-to-back single calls
+    for M in (512, 2048):
+        name = f"prefill_grouped_q4_k_4096+1024_m{M}"
+        if not want(name):
+            continue
+        Ns = [4096, 1024]
+        wl = [quantized_weights(dsq, dsq.DSQ_Q4_K, 630 + g, n, K) for g, n in enumerate(Ns)]
+        wbytes = sum(w.numel() for w in wl)
+        R = copies_for(wbytes)
+        copies = [wl] + [[w.clone() for w in wl] for _ in range(R - 1)]
+        x = torch.from_numpy(synth.activations(631 + M, M, K)).cuda()
+        ys = [torch.empty((M, n), dtype=torch.float32, device="cuda") for n in Ns]
+        nbg = dsq.dsq_prefill_grouped_workspace_bytes(dsq.DSQ_Q4_K, Ns, K, M)
+        wsg = torch.empty(nbg, dtype=torch.uint8, device="cuda")
+        nbs = [dsq.dsq_prefill_workspace_bytes(dsq.DSQ_Q4_K, n, K, M) for n in Ns]
+        wss = [torch.empty(b, dtype=torch.uint8, device="cuda") for b in nbs]
+        pw = [[w.data_ptr() for w in c] for c in copies]
+        arr_n = (ctypes.c_int64 * 2)(*Ns)
+        arr_y = (ctypes.c_void_p * 2)(*[y.data_ptr() for y in ys])
+        arr_w = [(ctypes.c_void_p * 2)(*p) for p in pw]
+        px = x.data_ptr()
+
+        def grouped(i, st):
+            L.dsq_gemm_prefill_grouped(dsq.DSQ_Q4_K, 2, arr_w[i % R], arr_n, K, px, M, arr_y, wsg.data_ptr(), nbg, st)
+
+        def singles(i, st):
+            for g in range(2):
+                L.dsq_gemm_prefill(dsq.DSQ_Q4_K, pw[i % R][g], Ns[g], K, px, M, ys[g].data_ptr(), wss[g].data_ptr(),
+                                   nbs[g], st)
+        t = time_graph(grouped, R * max(1, 24 // R))
+        flops = 2.0 * M * sum(Ns) * K
+        row = {**stats_row(t, wbytes + 4 * M * K + 4 * M * sum(Ns), flops), "weight_copies": R}
+        t2 = time_graph(singles, R * max(1, 24 // R))
+        row["single_calls_us"] = round(t2 * 1e6, 3)
+        rows[name] = row
+        del copies, wl, wsg, wss
     assert dsq.dsq_device_status() == 0
     return rows
 

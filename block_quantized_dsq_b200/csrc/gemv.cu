@@ -240,22 +240,6 @@ __device__ __forceinline__ void locate(const GemvArgs &a, int64_t r, int &seg, i
   if (r < a.rows0) { seg = 0; local = r; } else { seg = 1; local = r - a.rows0; }
 }
 
-// Activation group of a row within its segment (grouped form: group_rows
-// rows per group; other forms: one group).  A lane's rows only increase, so
-// the group is tracked across calls and the 64-bit division runs only when a
-// row leaves the current group's range.
-struct GroupTracker {
-  int64_t group = 0, lo = 0, hi = -1;   // hi < lo: nothing cached yet
-  __device__ __forceinline__ int64_t of(const GemvArgs &a, int64_t local) {
-    if (local >= lo && local < hi) return group;
-    group = local < a.group_rows ? 0 : local / a.group_rows;
-    lo = group * a.group_rows;
-    hi = lo + a.group_rows;
-    if (hi < lo) hi = INT64_MAX;   // one group: the bound overflowed
-    return group;
-  }
-};
-
 // Issue the bulk copy of virtual rows [ra, rb) into a slot (split when the
 // range crosses from segment 0 into segment 1).
 __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_t rb, uint8_t *dst, uint64_t *bar,
@@ -353,30 +337,23 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   const int sub = lane / G, j = lane % G;
   ActSlice act;
   int64_t cached = -1;  // (group * nunits + unit) currently in registers
-  GroupTracker gt;
+  {
+    // the slice of this lane's first (group, unit), loaded now so its
+    // latency overlaps the first weight slot's instead of following it
+    const int64_t row = r0 + static_cast<int64_t>(warp) * RPC + sub;
+    if (row < min(r0 + static_cast<int64_t>(warp) * RPC + RPC, r1) && j < a.nunits) {
+      int seg;
+      int64_t local;
+      locate(a, row, seg, local);
+      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
+      const int64_t e0 = group * a.K + static_cast<int64_t>(j) * 256;
+      load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
+      cached = group * a.nunits + j;
+    }
+  }
   int slot = 0;         // ring position kept incrementally (no division per chunk)
   uint32_t parity = 0;
   for (int64_t k = 0; k < mine; ++k) {
-    if (a.nunits <= G) {
-      // one unit per lane: (re)load the slice of this chunk's (group, unit)
-      // before waiting for the weight slot, so its latency overlaps the
-      // slot's flight (the first chunk, and every change of group in the
-      // grouped form) instead of following it
-      const int64_t ra = r0 + (warp + k * W) * RPC;
-      const int64_t row = ra + sub;
-      if (row < min(ra + RPC, r1) && j < a.nunits) {
-        int seg;
-        int64_t local;
-        locate(a, row, seg, local);
-        const int64_t group = gt.of(a, local);
-        const int64_t key = group * a.nunits + j;
-        if (key != cached) {
-          const int64_t e0 = group * a.K + static_cast<int64_t>(j) * 256;
-          load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
-          cached = key;
-        }
-      }
-    }
     const bool ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
     if (!ok) {
       if (lane == 0) {
@@ -395,7 +372,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       int seg;
       int64_t local;
       locate(a, row, seg, local);
-      const int64_t group = gt.of(a, local);
+      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
       const uint8_t *rowp = ring + static_cast<size_t>(slot) * a.slot_bytes + static_cast<size_t>(sub) * a.row_bytes;
       for (int u = j; u < a.nunits; u += G) {
         const int64_t key = group * a.nunits + u;
