@@ -19,6 +19,13 @@ namespace {
 __global__ void __launch_bounds__(256) act_q8_kernel(const float4 *__restrict__ x, int64_t nblocks,
                                                      int8_t *__restrict__ xq, float *__restrict__ xd,
                                                      int32_t *__restrict__ xs) {
+  if (threadIdx.x == 0) {
+    // this CTA's slice of x toward L2 while the previous kernel finishes (a
+    // hint: L2 is the point of coherence, so the predecessor's writes win)
+    const int64_t f0 = static_cast<int64_t>(blockIdx.x) * blockDim.x;
+    const int64_t nf = min(static_cast<int64_t>(blockDim.x), nblocks * 8 - f0);
+    if (nf > 0) prefetch_l2(x + f0, static_cast<uint32_t>(nf * 16));
+  }
   pdl_trigger();
   pdl_wait();
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
