@@ -354,20 +354,26 @@ struct Tile {
   int u0, u1, rot;
   int split, g;
 };
+// Every tile index, count and divisor here fits in 32 bits (the host refuses
+// a plan of 2^31 tiles or more), and 32-bit division costs a fraction of
+// 64-bit division, which sits at the start of every role's tile.
 __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   Tile tl;
-  tl.mt = t % a.tiles_m;
-  const int64_t rest = t / a.tiles_m;
-  tl.split = static_cast<int>(rest % a.splits);
-  const int64_t nt = rest / a.splits;
+  const uint32_t t32 = static_cast<uint32_t>(t);
+  const uint32_t tm = static_cast<uint32_t>(a.tiles_m), sp = static_cast<uint32_t>(a.splits);
+  const uint32_t rest = t32 / tm;
+  const uint32_t mt = t32 - rest * tm;
+  const uint32_t nt = rest / sp;
+  tl.mt = mt;
+  tl.split = static_cast<int>(rest - nt * sp);
   int g = 0;
-  while (g + 1 < a.G && nt >= a.tile_n0[g + 1]) ++g;
+  while (g + 1 < a.G && nt >= static_cast<uint32_t>(a.tile_n0[g + 1])) ++g;
   tl.g = g;
-  const int64_t ntl = nt - a.tile_n0[g];
-  tl.n0 = ntl * kTileN;
+  const uint32_t ntl = nt - static_cast<uint32_t>(a.tile_n0[g]);
+  tl.n0 = static_cast<int64_t>(ntl) * kTileN;
   tl.u0 = tl.split * a.units_per_split;
   tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
-  tl.rot = static_cast<int>((ntl + 7 * tl.mt) % (tl.u1 - tl.u0));
+  tl.rot = static_cast<int>((ntl + 7u * mt) % static_cast<uint32_t>(tl.u1 - tl.u0));
   return tl;
 }
 
@@ -1412,6 +1418,8 @@ int run_prefill(const char *name, int type, int64_t G, const void *const *w, con
   if (small_fits(type, K, M))
     return run_prefill_small(name, type, Gi, w, N, K, x, M, y, workspace, workspace_bytes, ctl, sms, st);
   const Plan p = make_plan(type, Gi, N, K, M, sms, -1);
+  DSQ_REQUIRE(p.total_tiles < (int64_t(1) << 31), DSQ_ERR_SHAPE, "%s: %lld tiles exceed one launch", name,
+              static_cast<long long>(p.total_tiles));
   DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= p.total, DSQ_ERR_WORKSPACE,
               "%s: workspace of %zu bytes needed, %zu given", name, p.total, workspace_bytes);
   DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "%s: workspace must be 256-byte aligned", name);
