@@ -494,7 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after_sync();
   pdl_trigger();
-  pdl_wait();
+  // The launch-dependency wait sits in each role, just before its first read
+  // of memory a predecessor may write (the activation and weight copies, the
+  // row shifts) or its first write of the outputs; the converters and the
+  // MMA issuer touch only shared and tensor memory and never wait.  All the
+  // set-up before a role's first copy then overlaps the previous kernel.
   const uint32_t tmem_base = *s.tmem;
   const uint32_t a_col0 = static_cast<uint32_t>(a.tn);   // first weight-stage column
 
@@ -521,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&s.ready[sq], slot_b_bytes);
+            if (gs == 0) pdl_wait();
             bulk_g2s(s.b + static_cast<size_t>(sq) * slot_b_bytes,
                      reinterpret_cast<const uint8_t *>(a.x16) +
                          ((xt * units + u) * 4 + kb4) * static_cast<int64_t>(stage_b_bytes),
@@ -621,6 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&s.rfull[rs], RAW_BYTES);
+          if (gu == 0) pdl_wait();
           tma_load_2d(s.raw + static_cast<size_t>(rs) * RAW_BYTES, &maps.m[tl.g], u * (UB / 4), row0,
                       &s.rfull[rs]);
           if (++rs == SR) {
@@ -653,8 +659,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t Ng = a.N[tl.g];
       const bool n_ok = n < Ng;
       const int64_t m0 = tl.mt * a.tn;
-      // before the wait: lane j holds 2^-s of token m0 + 32c + j for every
+      // before the accumulator wait: lane j holds 2^-s of token m0 + 32c + j for every
       // chunk c (0 for padding tokens), so the drain below has no loads
+      if (i == 0) pdl_wait();
       float my_scale[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
