@@ -294,14 +294,32 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
     }
     prefetch_l2(a.x32 + ga * a.K, static_cast<uint32_t>((gb - ga + 1) * a.K * 4));
   }
-  pdl_trigger();
-  pdl_wait();
-  if (!FUSED && mine == 0) return;
-
+  // Everything that needs nothing from a predecessor is set up before the
+  // wait: the slot barriers, the copy policy, and where this lane's first
+  // activation slice lives.
   const uint64_t policy = l2_policy_evict_first();
   if (lane == 0 && mine > 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
+  }
+  const int sub = lane / G, j = lane % G;
+  int64_t first_e0 = -1, first_key = -1;   // element offset and (group * nunits + unit) of that slice
+  {
+    const int64_t row = r0 + static_cast<int64_t>(warp) * RPC + sub;
+    if (row < min(r0 + static_cast<int64_t>(warp) * RPC + RPC, r1) && j < a.nunits) {
+      int seg;
+      int64_t local;
+      locate(a, row, seg, local);
+      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
+      first_e0 = group * a.K + static_cast<int64_t>(j) * 256;
+      first_key = group * a.nunits + j;
+    }
+  }
+  pdl_trigger();
+  pdl_wait();
+  if (!FUSED && mine == 0) return;
+
+  if (lane == 0 && mine > 0) {
     for (int64_t k = 0; k < mine && k < S; ++k) {
       const int64_t c = warp + k * W;
       const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
@@ -334,22 +352,13 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   }
   __syncwarp();
 
-  const int sub = lane / G, j = lane % G;
   ActSlice act;
   int64_t cached = -1;  // (group * nunits + unit) currently in registers
-  {
+  if (first_e0 >= 0) {
     // the slice of this lane's first (group, unit), loaded now so its
     // latency overlaps the first weight slot's instead of following it
-    const int64_t row = r0 + static_cast<int64_t>(warp) * RPC + sub;
-    if (row < min(r0 + static_cast<int64_t>(warp) * RPC + RPC, r1) && j < a.nunits) {
-      int seg;
-      int64_t local;
-      locate(a, row, seg, local);
-      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
-      const int64_t e0 = group * a.K + static_cast<int64_t>(j) * 256;
-      load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
-      cached = group * a.nunits + j;
-    }
+    load_act<TYPE, FUSED>(act, xq + first_e0, xd + first_e0 / 32, TYPE == DSQ_Q4_K ? xs + first_e0 / 32 : nullptr);
+    cached = first_key;
   }
   int slot = 0;         // ring position kept incrementally (no division per chunk)
   uint32_t parity = 0;
