@@ -381,7 +381,9 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       int seg;
       int64_t local;
       locate(a, row, seg, local);
-      const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
+      // rows and group sizes are below 2^31 (checked on the host): 32-bit division
+      const int64_t group =
+          local < a.group_rows ? 0 : static_cast<uint32_t>(local) / static_cast<uint32_t>(a.group_rows);
       const uint8_t *rowp = ring + static_cast<size_t>(slot) * a.slot_bytes + static_cast<size_t>(sub) * a.row_bytes;
       for (int u = j; u < a.nunits; u += G) {
         const int64_t key = group * a.nunits + u;
