@@ -96,29 +96,96 @@ struct ActSlice {
   int32_t s[8];     // 8 block code sums (Q4_K only)
 };
 
-// SMEM: the slice lives in this CTA's shared memory (fused mode), else in
-// global memory (read-only path).
-template <int TYPE, bool SMEM>
+// The slice of one unit from the prequantized rows in global memory
+// (read-only path): codes, scales and sums are contiguous.
+template <int TYPE>
 __device__ __forceinline__ void load_act(ActSlice &act, const int8_t *xq, const float *xd, const int32_t *xs) {
   const uint4 *q4 = reinterpret_cast<const uint4 *>(xq);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint4 v = SMEM ? q4[i] : __ldg(q4 + i);
+    const uint4 v = __ldg(q4 + i);
     act.q[4 * i + 0] = v.x; act.q[4 * i + 1] = v.y; act.q[4 * i + 2] = v.z; act.q[4 * i + 3] = v.w;
   }
   const float4 *d4 = reinterpret_cast<const float4 *>(xd);
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const float4 v = SMEM ? d4[i] : __ldg(d4 + i);
+    const float4 v = __ldg(d4 + i);
     act.d[4 * i + 0] = v.x; act.d[4 * i + 1] = v.y; act.d[4 * i + 2] = v.z; act.d[4 * i + 3] = v.w;
   }
   if (TYPE == DSQ_Q4_K) {
     const int4 *s4 = reinterpret_cast<const int4 *>(xs);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int4 v = SMEM ? s4[i] : __ldg(s4 + i);
+      const int4 v = __ldg(s4 + i);
       act.s[4 * i + 0] = v.x; act.s[4 * i + 1] = v.y; act.s[4 * i + 2] = v.z; act.s[4 * i + 3] = v.w;
     }
+  }
+}
+
+// Shared-memory activation area (fused and staged modes), per activation
+// row: the codes as [16][nunits] 16-byte words (word i of unit u at
+// i * nunits + u) and the scales and sums each as [2][nunits] 16-byte words.
+// The G lanes of a row read G consecutive units at once, so they touch
+// consecutive 16-byte words instead of the same bank 16 times.
+__device__ __forceinline__ uint32_t act_q_word(uint32_t w, uint32_t nunits) {   // w: 4-code word of the row
+  return (((w & 63u) >> 2) * nunits + (w >> 6)) * 4u + (w & 3u);
+}
+__device__ __forceinline__ uint32_t act_s_word(uint32_t b, uint32_t nunits) {   // b: 32-block of the row
+  return (((b & 7u) >> 2) * nunits + (b >> 3)) * 4u + (b & 3u);
+}
+
+template <int TYPE>
+__device__ __forceinline__ void load_act_smem(ActSlice &act, const int8_t *qrow, const float *drow,
+                                              const int32_t *srow, int u, int nunits) {
+  const uint4 *q4 = reinterpret_cast<const uint4 *>(qrow) + u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint4 v = q4[i * nunits];
+    act.q[4 * i + 0] = v.x; act.q[4 * i + 1] = v.y; act.q[4 * i + 2] = v.z; act.q[4 * i + 3] = v.w;
+  }
+  const float4 *d4 = reinterpret_cast<const float4 *>(drow) + u;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float4 v = d4[i * nunits];
+    act.d[4 * i + 0] = v.x; act.d[4 * i + 1] = v.y; act.d[4 * i + 2] = v.z; act.d[4 * i + 3] = v.w;
+  }
+  if (TYPE == DSQ_Q4_K) {
+    const int4 *s4 = reinterpret_cast<const int4 *>(srow) + u;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int4 v = s4[i * nunits];
+      act.s[4 * i + 0] = v.x; act.s[4 * i + 1] = v.y; act.s[4 * i + 2] = v.z; act.s[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// Where the dot loop reads its activation slices: global memory (the
+// prequantized rows), shared memory quantized by the CTA itself from fp32 (the
+// fused entry points), or shared memory copied once from the prequantized
+// groups (the grouped form: a warp whose rows cross into the next group then
+// reloads its slice from shared memory instead of waiting on L2).
+enum : int { kActGlobal = 0, kActFused = 1, kActStaged = 2 };
+
+// Staged mode: the CTA's threads copy prequantized activation groups
+// [g0, g0 + rows) into the shared-memory area (at most 64 KB, so 32-bit
+// indices suffice).
+__device__ __forceinline__ void copy_act_to_smem(const GemvArgs &a, int64_t g0, int64_t rows, int8_t *sq,
+                                                 float *sd, int32_t *ss) {
+  const uint32_t nunits = static_cast<uint32_t>(a.nunits);
+  const uint32_t q_row = nunits * 16u, s_row = nunits * 2u;   // 16-byte words per row: codes, scales
+  const uint32_t nq = static_cast<uint32_t>(rows) * q_row, ns = static_cast<uint32_t>(rows) * s_row;
+  const uint4 *q = reinterpret_cast<const uint4 *>(a.xq + g0 * a.K);
+  for (uint32_t g = threadIdx.x; g < nq; g += blockDim.x) {
+    const uint32_t r = g / q_row, gg = g - r * q_row;   // row; word gg = 16 codes of unit gg / 16
+    reinterpret_cast<uint4 *>(sq)[r * q_row + (gg & 15u) * nunits + (gg >> 4)] = __ldg(q + g);
+  }
+  const uint4 *d = reinterpret_cast<const uint4 *>(a.xd + g0 * (a.K / 32));
+  const uint4 *x = a.xs ? reinterpret_cast<const uint4 *>(a.xs + g0 * (a.K / 32)) : nullptr;
+  for (uint32_t f = threadIdx.x; f < ns; f += blockDim.x) {
+    const uint32_t r = f / s_row, ff = f - r * s_row;   // row; word ff = 4 blocks of unit ff / 2
+    const uint32_t dst = r * s_row + (ff & 1u) * nunits + (ff >> 1);
+    reinterpret_cast<uint4 *>(sd)[dst] = __ldg(d + f);
+    if (x) reinterpret_cast<uint4 *>(ss)[dst] = __ldg(x + f);
   }
 }
 
@@ -132,6 +199,7 @@ __device__ __forceinline__ void quantize_act_to_smem(const GemvArgs &a, int64_t 
                                                      float *sd, int32_t *ss) {
   constexpr int kBatch = 4;
   const int64_t tasks = rows * a.K / 4;   // float4s
+  const uint32_t row_words = static_cast<uint32_t>(a.K / 4), nunits = static_cast<uint32_t>(a.nunits);
   const float4 *x4 = reinterpret_cast<const float4 *>(a.x32 + g0 * a.K);
   const int64_t step = static_cast<int64_t>(blockDim.x) * kBatch;
   for (int64_t base = 0; base < tasks; base += step) {
@@ -148,10 +216,13 @@ __device__ __forceinline__ void quantize_act_to_smem(const GemvArgs &a, int64_t 
       int sum;
       const uint32_t packed = q8_block_lanes(v[i], d, sum);
       if (t < tasks) {
-        reinterpret_cast<uint32_t *>(sq)[t] = packed;
-        if ((t & 7) == 0) {
-          sd[t >> 3] = d;
-          ss[t >> 3] = sum;
+        // the area is at most 64 KB: 32-bit indices
+        const uint32_t r = static_cast<uint32_t>(t) / row_words, w = static_cast<uint32_t>(t) - r * row_words;
+        reinterpret_cast<uint32_t *>(sq)[r * row_words + act_q_word(w, nunits)] = packed;
+        if ((w & 7u) == 0) {
+          const uint32_t b = r * (row_words / 8u) + act_s_word(w >> 3, nunits);
+          sd[b] = d;
+          ss[b] = sum;
         }
       }
     }
@@ -257,7 +328,7 @@ __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_
   }
 }
 
-template <int TYPE, int G, bool ISUM, bool FUSED>
+template <int TYPE, int G, bool ISUM, int ACT>
 __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
   constexpr int RPC = 32 / G;  // rows per slot
   extern __shared__ __align__(128) uint8_t smem[];
@@ -284,7 +355,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       }
     }
   }
-  if (FUSED && threadIdx.x == 0) {
+  if (ACT == kActFused && threadIdx.x == 0) {
     // the fp32 activation rows this CTA will quantize, toward L2 (a hint:
     // the predecessor's writes still win, L2 being the point of coherence)
     int64_t ga = 0, gb = 0;
@@ -303,7 +374,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
     fence_barrier_init();
   }
   const int sub = lane / G, j = lane % G;
-  int64_t first_e0 = -1, first_key = -1;   // element offset and (group * nunits + unit) of that slice
+  int64_t first_group = -1, first_key = -1;   // group and (group * nunits + unit) of that slice
   {
     const int64_t row = r0 + static_cast<int64_t>(warp) * RPC + sub;
     if (row < min(r0 + static_cast<int64_t>(warp) * RPC + RPC, r1) && j < a.nunits) {
@@ -311,13 +382,13 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       int64_t local;
       locate(a, row, seg, local);
       const int64_t group = local < a.group_rows ? 0 : local / a.group_rows;
-      first_e0 = group * a.K + static_cast<int64_t>(j) * 256;
+      first_group = group;
       first_key = group * a.nunits + j;
     }
   }
   pdl_trigger();
   pdl_wait();
-  if (!FUSED && mine == 0) return;
+  if (ACT == kActGlobal && mine == 0) return;
 
   if (lane == 0 && mine > 0) {
     for (int64_t k = 0; k < mine && k < S; ++k) {
@@ -331,7 +402,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   const int8_t *xq = a.xq;
   const float *xd = a.xd;
   const int32_t *xs = a.xs;
-  if (FUSED) {
+  if (ACT != kActGlobal) {
     // only the activation groups this CTA's rows read: [g0, g1]
     int64_t g0 = 0, g1 = 0;
     if (r1 > r0 && a.act_rows > 1) {
@@ -342,7 +413,8 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
     int8_t *sq = reinterpret_cast<int8_t *>(smem + a.act_off);
     float *sd = reinterpret_cast<float *>(sq + rows * a.K);
     int32_t *ss = reinterpret_cast<int32_t *>(sd + rows * (a.K / 32));
-    quantize_act_to_smem(a, g0, rows, sq, sd, ss);
+    if (ACT == kActFused) quantize_act_to_smem(a, g0, rows, sq, sd, ss);
+    else copy_act_to_smem(a, g0, rows, sq, sd, ss);
     __syncthreads();
     if (mine == 0) return;
     // indexed by absolute group below: shift the bases by g0 rows
@@ -352,12 +424,21 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
   }
   __syncwarp();
 
+  // the activation slice of (group, unit u) into registers
+  auto fetch_act = [&](ActSlice &dst, int64_t group, int u) {
+    if (ACT == kActGlobal) {
+      const int64_t e0 = group * a.K + static_cast<int64_t>(u) * 256;
+      load_act<TYPE>(dst, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
+    } else {
+      load_act_smem<TYPE>(dst, xq + group * a.K, xd + group * (a.K / 32), xs + group * (a.K / 32), u, a.nunits);
+    }
+  };
   ActSlice act;
   int64_t cached = -1;  // (group * nunits + unit) currently in registers
-  if (first_e0 >= 0) {
+  if (first_group >= 0) {
     // the slice of this lane's first (group, unit), loaded now so its
     // latency overlaps the first weight slot's instead of following it
-    load_act<TYPE, FUSED>(act, xq + first_e0, xd + first_e0 / 32, TYPE == DSQ_Q4_K ? xs + first_e0 / 32 : nullptr);
+    fetch_act(act, first_group, j);
     cached = first_key;
   }
   int slot = 0;         // ring position kept incrementally (no division per chunk)
@@ -388,8 +469,7 @@ __global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM)
       for (int u = j; u < a.nunits; u += G) {
         const int64_t key = group * a.nunits + u;
         if (key != cached) {
-          const int64_t e0 = group * a.K + static_cast<int64_t>(u) * 256;
-          load_act<TYPE, FUSED>(act, xq + e0, xd + e0 / 32, TYPE == DSQ_Q4_K ? xs + e0 / 32 : nullptr);
+          fetch_act(act, group, u);
           cached = key;
         }
         int32_t is[8];
@@ -467,17 +547,17 @@ constexpr size_t kSmemBudget = DSQ_GEMV_SMEM_KB * 1024;
 // scales and int32 sums per 32-block.
 size_t act_smem_bytes(int64_t rows, int64_t K) { return static_cast<size_t>(rows) * (K + 8 * (K / 32)); }
 
-template <int TYPE, int G, bool ISUM, bool FUSED>
+template <int TYPE, int G, bool ISUM, int ACT>
 int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   constexpr int RPC = 32 / G;
   size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
                 static_cast<size_t>(a.warps) * a.stages * sizeof(uint64_t);
-  if (FUSED) {
+  if (ACT != kActGlobal) {
     smem = (smem + 15) / 16 * 16;
     a.act_off = static_cast<int>(smem);
     smem += act_smem_bytes(a.act_rows, a.K);
   }
-  auto kern = gemv_kernel<TYPE, G, ISUM, FUSED>;
+  auto kern = gemv_kernel<TYPE, G, ISUM, ACT>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
   if (rc != DSQ_OK) return rc;
   const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
@@ -488,16 +568,23 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   return after_launch("gemv");
 }
 
-template <int TYPE, bool ISUM, bool FUSED>
+template <int TYPE, bool ISUM, int ACT>
 int dispatch_g(GemvArgs &a, int G, int num_sms, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_fast<TYPE, 1, ISUM, FUSED>(a, num_sms, stream);
-    case 2: return launch_fast<TYPE, 2, ISUM, FUSED>(a, num_sms, stream);
-    case 4: return launch_fast<TYPE, 4, ISUM, FUSED>(a, num_sms, stream);
-    case 8: return launch_fast<TYPE, 8, ISUM, FUSED>(a, num_sms, stream);
-    case 16: return launch_fast<TYPE, 16, ISUM, FUSED>(a, num_sms, stream);
-    default: return launch_fast<TYPE, 32, ISUM, FUSED>(a, num_sms, stream);
+    case 1: return launch_fast<TYPE, 1, ISUM, ACT>(a, num_sms, stream);
+    case 2: return launch_fast<TYPE, 2, ISUM, ACT>(a, num_sms, stream);
+    case 4: return launch_fast<TYPE, 4, ISUM, ACT>(a, num_sms, stream);
+    case 8: return launch_fast<TYPE, 8, ISUM, ACT>(a, num_sms, stream);
+    case 16: return launch_fast<TYPE, 16, ISUM, ACT>(a, num_sms, stream);
+    default: return launch_fast<TYPE, 32, ISUM, ACT>(a, num_sms, stream);
   }
+}
+
+template <int TYPE, bool ISUM>
+int dispatch_act(GemvArgs &a, int G, int act, int num_sms, cudaStream_t stream) {
+  if (act == kActFused) return dispatch_g<TYPE, ISUM, kActFused>(a, G, num_sms, stream);
+  if (act == kActStaged) return dispatch_g<TYPE, ISUM, kActStaged>(a, G, num_sms, stream);
+  return dispatch_g<TYPE, ISUM, kActGlobal>(a, G, num_sms, stream);
 }
 
 // Largest activation area the fused mode keeps in shared memory (e.g. 8 rows
@@ -568,22 +655,21 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   int G = 1;
   while (G < a.nunits && G < 32) G <<= 1;
   a.slot_bytes = static_cast<int>((32 / G) * rb);
-  // the ring gets the shared memory the fused activation area leaves
-  const size_t budget = kSmemBudget - (x32 ? act_smem_bytes(groups, K) + 16 : 0);
+  // the grouped form copies its CTA's activation groups into shared memory
+  // when they fit; the ring gets the shared memory the activation area leaves
+  const int act = x32 ? kActFused : (groups > 1 && act_smem_bytes(groups, K) <= kMaxActSmem ? kActStaged : kActGlobal);
+  const size_t budget = kSmemBudget - (act != kActGlobal ? act_smem_bytes(groups, K) + 16 : 0);
   a.warps = kMaxWarps;
   while (a.warps > 1 && static_cast<size_t>(a.warps) * 2 * a.slot_bytes > budget) a.warps >>= 1;
   DSQ_REQUIRE(static_cast<size_t>(a.warps) * 2 * a.slot_bytes <= budget, DSQ_ERR_SHAPE,
               "%s: K=%lld rows do not fit the shared-memory pipeline", name, (long long)K);
   a.stages = static_cast<int>(budget / (static_cast<size_t>(a.warps) * a.slot_bytes));
   if (a.stages > DSQ_GEMV_MAX_STAGES) a.stages = DSQ_GEMV_MAX_STAGES;
-  if (x32)
-    return type == DSQ_Q8_0 ? dispatch_g<DSQ_Q8_0, false, true>(a, G, num_sms, stream)
-                            : dispatch_g<DSQ_Q4_K, false, true>(a, G, num_sms, stream);
   if (type == DSQ_Q8_0)
-    return isum ? dispatch_g<DSQ_Q8_0, true, false>(a, G, num_sms, stream)
-                : dispatch_g<DSQ_Q8_0, false, false>(a, G, num_sms, stream);
-  return isum ? dispatch_g<DSQ_Q4_K, true, false>(a, G, num_sms, stream)
-              : dispatch_g<DSQ_Q4_K, false, false>(a, G, num_sms, stream);
+    return isum ? dispatch_act<DSQ_Q8_0, true>(a, G, act, num_sms, stream)
+                : dispatch_act<DSQ_Q8_0, false>(a, G, act, num_sms, stream);
+  return isum ? dispatch_act<DSQ_Q4_K, true>(a, G, act, num_sms, stream)
+              : dispatch_act<DSQ_Q4_K, false>(a, G, act, num_sms, stream);
 }
 
 constexpr int64_t kOneGroup = int64_t(1) << 62;
