@@ -3,7 +3,9 @@
 
 One step = the paired Q8_0 decode projection workload: 64 back-to-back calls,
 each quantizing a fresh fp32 activation (1 x 4096) to Q8 and running the
-paired GEMV of two Q8_0 weights (8192 x 4096 each) against it.  Weights are
+paired GEMV of two Q8_0 weights (8192 x 4096 each) against it, both in one
+launch (dsq_gemv_paired_f32); the same calls as two launches each
+(dsq_quantize_act_q8, then dsq_gemv_paired) are timed beside it.  Weights are
 rotated over enough copies that L2 (126 MB) cannot serve them.  The headline
 value is HBM GB/s of algorithmic bytes; the same JSON line also carries
 us/call, the roofline of the dominant kernel, an end-to-end figure through
@@ -35,11 +37,14 @@ WORKLOAD = "paired Q8_0 decode projection: 2 x (8192 x 4096) weights, shared 1 x
 
 
 def paired_bytes_per_call() -> dict:
-    """Algorithmic bytes of one call: the quantize step and the paired GEMV."""
+    """Algorithmic bytes of one call.  fused: the one-launch form (weights,
+    the fp32 activation, the outputs); two_call: the quantize step (x in,
+    codes, scales and sums out) plus the paired GEMV on the codes (gemv)."""
     rb = K_PAIR // 32 * 34
-    gemv = 2 * N_PAIR * rb + K_PAIR + (K_PAIR // 32) * 4 + 2 * N_PAIR * 4
+    weights, out = 2 * N_PAIR * rb, 2 * N_PAIR * 4
+    gemv = weights + K_PAIR + (K_PAIR // 32) * 4 + out
     quant = K_PAIR * 4 + K_PAIR + 2 * (K_PAIR // 32) * 4
-    return {"gemv": gemv, "quant": quant, "total": gemv + quant}
+    return {"fused": weights + K_PAIR * 4 + out, "gemv": gemv, "quant": quant, "two_call": gemv + quant}
 
 
 def measured_peaks():
@@ -203,7 +208,7 @@ def bench_config(world: int) -> dict:
     """The workload description both arms print."""
     R = paired_copies()
     return {"workload": WORKLOAD, "weights": "N(0,0.02^2) fp32 quantized to Q8_0, seeds 1/2",
-            "activations": "N(0,1) fp32, seeds 1000..1063, quantized to Q8 per call",
+            "activations": "N(0,1) fp32, seeds 1000..1063, quantized to Q8 per call inside the GEMV launch",
             "l2": f"weights rotated over {R} copies ({R * paired_bytes_per_call()['gemv'] / 1e6:.0f} MB > 3x L2)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -312,23 +317,29 @@ def run_dsq(args, world, rank):
     p_y0 = [Y[i, 0].data_ptr() for i in range(CALLS)]
     p_y1 = [Y[i, 1].data_ptr() for i in range(CALLS)]
     p_w = [(a.data_ptr(), b.data_ptr()) for a, b in pairs]
-    quant, paired = L.dsq_quantize_act_q8, L.dsq_gemv_paired
+    quant, paired, fused = L.dsq_quantize_act_q8, L.dsq_gemv_paired, L.dsq_gemv_paired_f32
 
-    def one_call(c, st, with_quant=True):
-        rc = quant(p_x[c], 1, K_PAIR, p_xq[c], p_xd[c], p_xs[c], st) if with_quant else 0
+    def one_call(c, st, form):
+        """form: "fused" (the step: one launch quantizes x and runs the paired
+        GEMV), "two_call" (quantize, then the GEMV on the codes) or "gemv"
+        (the GEMV alone on codes already made)."""
         w0, w1 = p_w[c % R]
-        rc |= paired(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_xq[c], p_xd[c], p_xs[c], p_y0[c], p_y1[c], st)
+        if form == "fused":
+            rc = fused(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_x[c], p_y0[c], p_y1[c], st)
+        else:
+            rc = quant(p_x[c], 1, K_PAIR, p_xq[c], p_xd[c], p_xs[c], st) if form == "two_call" else 0
+            rc |= paired(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_xq[c], p_xd[c], p_xs[c], p_y0[c], p_y1[c], st)
         if rc:
             raise RuntimeError(dsq.dsq_last_error())
 
-    def capture(with_quant):
+    def capture(form):
         """One step (64 calls) as a CUDA graph: the decode loop's launch
         pattern without host launch overhead between the kernels."""
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
             for c in range(CALLS):
-                one_call(c, side.cuda_stream, with_quant)
+                one_call(c, side.cuda_stream, form)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -336,10 +347,22 @@ def run_dsq(args, world, rank):
         with torch.cuda.graph(g):
             st = torch.cuda.current_stream().cuda_stream
             for c in range(CALLS):
-                one_call(c, st, with_quant)
+                one_call(c, st, form)
         return g, dsq.dsq_launch_count() - n0
 
-    step_graph, launches_per_step = capture(True)
+    def replay_avg(graph, reps):
+        """Average time of one replay over `reps` back-to-back replays."""
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    step_graph, launches_per_step = capture("fused")
     for _ in range(args.warmup):
         step_graph.replay()
     torch.cuda.synchronize()
@@ -361,22 +384,19 @@ def run_dsq(args, world, rank):
     launches = launches_per_step * args.steps
     assert dsq.dsq_device_status() == 0, "a device wait timed out during the bench"
     ms_per_step = elapsed / args.steps * 1e3
-    value = world * args.steps * CALLS * bpc["total"] / elapsed / 1e9
+    value = world * args.steps * CALLS * bpc["fused"] / elapsed / 1e9
+    # the step is one kernel launch per call: the dominant kernel's average
+    # launch duration is the timed region over its launches
+    kern_avg = elapsed / launches
 
-    # ---- the dominant kernel alone: 64 back-to-back paired GEMV launches
-    # (same launch pattern, no quantize in between), CUDA events on its stream
-    gemv_graph, _ = capture(False)
-    gemv_graph.replay()
-    torch.cuda.synchronize()
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- the same step as two launches per call (quantize, then the GEMV on
+    # the codes), and the GEMV alone, for comparison
     reps = max(3, args.steps // 4)
-    g0.record()
-    for _ in range(reps):
-        gemv_graph.replay()
-    g1.record()
-    torch.cuda.synchronize()
-    gemv_avg = g0.elapsed_time(g1) / 1e3 / (reps * CALLS)
-    del gemv_graph, step_graph
+    two_graph, _ = capture("two_call")
+    two_avg = replay_avg(two_graph, reps) / CALLS
+    gemv_graph, _ = capture("gemv")
+    gemv_avg = replay_avg(gemv_graph, reps) / CALLS
+    del gemv_graph, two_graph, step_graph
 
     # ---- end to end through the public API with host buffers
     X_pin = torch.from_numpy(X_host).pin_memory()
@@ -386,15 +406,13 @@ def run_dsq(args, world, rank):
     def e2e_step(s):
         X.copy_(X_pin, non_blocking=True)
         for c in range(CALLS):
-            dsq.dsq_quantize_act_q8(p_x[c], 1, K_PAIR, p_xq[c], p_xd[c], p_xs[c], stream)
             w0, w1 = p_w[c % R]
-            dsq.dsq_gemv_paired(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_xq[c], p_xd[c], p_xs[c], p_y0[c], p_y1[c],
-                                stream)
+            dsq.dsq_gemv_paired_f32(8, w0, N_PAIR, w1, N_PAIR, K_PAIR, p_x[c], p_y0[c], p_y1[c], stream)
         Y_pin.copy_(Y, non_blocking=True)
 
     e2e_t = time_calls(lambda s_, st_: e2e_step(s_), e2e_steps, warmup=2)
     e2e_t = max_over_ranks(world, e2e_t)
-    e2e_value = world * CALLS * bpc["total"] / e2e_t / 1e9
+    e2e_value = world * CALLS * bpc["fused"] / e2e_t / 1e9
 
     # ---- the other rows of the path (each its own short timed loop)
     rows, rows_clocks = {}, None
@@ -413,16 +431,22 @@ def run_dsq(args, world, rank):
         "config": bench_config(world),
         "us_per_call": round(ms_per_step * 1e3 / CALLS, 3),
         "hbm_frac": round(value / world / hbm_peak, 4),
-        "timing": "CUDA graph of one step (64 x quantize + paired GEMV, programmatic launch) replayed "
+        "timing": "CUDA graph of one step (64 calls of dsq_gemv_paired_f32: each quantizes its fp32 "
+                  "activation and runs the paired GEMV in one launch, programmatic launch) replayed "
                   f"{args.steps} times; CUDA events on the replay stream",
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (paired Q8_0)",
-                     "achieved": round(bpc["gemv"] / gemv_avg / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(bpc["gemv"] / gemv_avg / 1e9 / hbm_peak, 4),
-                     "traffic": traffic_record("gemv_kernel", "paired_q8_0_2x8192x4096"),
-                     "algorithmic_bytes": bpc["gemv"], "avg_launch_us": round(gemv_avg * 1e6, 3),
-                     "measured": f"{reps} replays of a graph of 64 back-to-back paired GEMV launches",
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (paired Q8_0, activation quantized in the kernel)",
+                     "achieved": round(bpc["fused"] / kern_avg / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(bpc["fused"] / kern_avg / 1e9 / hbm_peak, 4),
+                     "traffic": traffic_record("gemv_kernel", "paired_f32_q8_0_2x8192x4096"),
+                     "algorithmic_bytes": bpc["fused"], "avg_launch_us": round(kern_avg * 1e6, 3),
+                     "measured": "the timed region over its launches (one per call)",
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                      else "fallback"},
+        "two_call": {"us_per_call": round(two_avg * 1e6, 3), "GB/s": round(bpc["two_call"] / two_avg / 1e9, 1),
+                     "gemv_us_per_call": round(gemv_avg * 1e6, 3),
+                     "gemv_GB/s": round(bpc["gemv"] / gemv_avg / 1e9, 1),
+                     "measured": f"{reps} replays of a graph of the 64 calls as dsq_quantize_act_q8 + "
+                                 "dsq_gemv_paired, and of the 64 paired GEMVs alone"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": CALLS * K_PAIR * 4,
                 "d2h_bytes_per_step": CALLS * 2 * N_PAIR * 4, "us_per_call": round(e2e_t / CALLS * 1e6, 3)},
         "gpu_launches": int(launches),
@@ -746,6 +770,8 @@ def run_profile(args):
         xs = torch.empty(K_PAIR // 32, dtype=torch.int32, device="cuda")
         y = torch.empty((2, N_PAIR), dtype=torch.float32, device="cuda")
         for _ in range(3):
+            dsq.dsq_gemv_paired_f32(8, W0, N_PAIR, W1, N_PAIR, K_PAIR, x, y[0], y[1], stream)
+        for _ in range(3):
             dsq.dsq_quantize_act_q8(x, 1, K_PAIR, xq, xd, xs, stream)
             dsq.dsq_gemv_paired(8, W0, N_PAIR, W1, N_PAIR, K_PAIR, xq, xd, xs, y[0], y[1], stream)
         torch.cuda.synchronize()
@@ -773,7 +799,7 @@ def cpu_baseline(pair, X_host, budget_s: float):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(n * bpc["total"] / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    return {"value": round(n * bpc["fused"] / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} of the 64 paired calls (oracle act-quantize + two integer-form GEMVs), {dt:.1f} s",
             "cpu": platform.processor() or platform.machine(), "host_cores": os.cpu_count()}
 
@@ -856,7 +882,7 @@ def run_reference(args, world, rank):
     for s in range(args.steps):
         step(s)
     dt = time.perf_counter() - t0
-    value = args.steps * per_step * bpc["total"] / dt / 1e9
+    value = args.steps * per_step * bpc["fused"] / dt / 1e9
     sample = f"{per_step} of the 64 paired calls per step (oracle act-quantize + two integer-form GEMVs)"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
