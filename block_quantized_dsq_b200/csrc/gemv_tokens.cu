@@ -64,6 +64,7 @@ struct TokArgs {
   uint32_t box_bytes;     // one TMA box: 32 rows x one unit
   uint32_t q_bytes, d_bytes, s_bytes;   // activation areas in shared memory
   uint32_t ring_off, bar_off, red_off;  // shared-memory offsets
+  uint32_t sc_off;        // tensor-core form, Q4_K: per-warp scale scratch
   const int8_t *xq;       // [M][K]
   const float *xd;        // [M][K/32]
   const int32_t *xs;      // [M][K/32] (Q4_K)
@@ -372,6 +373,319 @@ __global__ void __launch_bounds__(kTokWarps * 32, 1)
   if (threadIdx.x == 0 && !ok) mbar_wait_for(act_bar, 0, kDrainLimitNs);
 }
 
+// ------------------------------------------------------- 5 to 8 tokens ---
+// From 5 (Q8_0) or 7 (Q4_K) tokens on, the block dots run on the tensor cores: one
+// mma.sync.m16n8k32 (int8 x int8 -> int32) gives the exact block sums of one
+// 32-element block for 16 weight rows x 8 tokens.  Integer sums are exact
+// whoever forms them, and the lanes then form each fp32 block term and add
+// it in the single-token kernel's order, so every output stays bit-identical
+// to the single-token entry points; only the lane that computes a term
+// changes.  Per block a warp issues two MMAs (rows 0..15, 16..31) where the
+// CUDA-core form issues 64 dp4a per lane, and no lane holds a whole row.
+//
+// Fragments of m16n8k32 (lane = 4 grp + t): A rows grp and grp + 8, codes
+// 4t..4t+3 and 16+4t..16+4t+3 of the block; B token grp, the same codes; D
+// rows grp and grp + 8, tokens 2t and 2t + 1.
+//
+// Activations in shared memory (tokens padded to 8 with zeros):
+//   codes as 32-bit words [unit][block][chunk kc][token] -- lane (grp, t)
+//   reads chunk t (and t + 4) of token grp: 32 consecutive words;
+//   scales and sums as [unit * 8 + block][token] -- lane reads tokens 2t, 2t+1.
+// The tensor-core form does the work of 8 tokens whatever M is, so it pays
+// only from a type-dependent token count on (interleaved A/B on one B200:
+// paired 2 x 8192 x 4096 Q8_0 at 4 / 6 / 8 tokens 21.9 / 22.9 / 22.7 us
+// against 20.3 / 26.7 / 33.9 on the CUDA cores; Q4_K 4096 x 4096 8.8 / 9.4 /
+// 9.3 us against 7.0 / 8.7 / 10.4).
+constexpr int kTokMmaMinM = 5;   // the smallest count any type takes it at
+__host__ __device__ constexpr int tok_mma_min_m(int type) { return type == DSQ_Q8_0 ? 5 : 7; }
+constexpr int kTokScStride = 18;   // words per row of the Q4_K scale scratch (8 pairs + pad)
+
+__device__ __forceinline__ void mma_s8_m16n8k32(int32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// Value v of a lane's 8 (row, token) terms: m-tile mt = v / 4, row half h =
+// (v / 2) % 2, token e = v % 2 -> row grp + 8h + 16mt, token 2t + e.
+__device__ __forceinline__ int mma_row(int v, int grp) { return grp + 8 * ((v >> 1) & 1) + 16 * (v >> 2); }
+__device__ __forceinline__ int mma_tok(int v, int t) { return 2 * t + (v & 1); }
+
+// One Q8_0 unit of the warp's 32-row box against unit u of the tokens:
+// part[v] = sum over the 8 blocks, in order, of (d_w * xd) * isum.
+template <int M>
+__device__ __forceinline__ void tok_mma_q8_0(const uint8_t *box, const uint32_t *qt, const float *dt, int u,
+                                             int lane, float (&part)[8], int32_t *isum, int64_t isum_row,
+                                             int64_t isum_tok, int64_t rows_left) {
+  const int grp = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) part[v] = 0.0f;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    uint32_t A[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint8_t *p = box + (grp + 8 * h + 16 * mt) * 272 + 34 * b + 2 + 4 * t + 16 * kk;
+          // codes of even blocks sit 2 bytes past a word boundary
+          A[mt][h + 2 * kk] = (b & 1) ? lds32(p) : __funnelshift_r(lds32(p - 2), lds32(p + 2), 16);
+        }
+    const uint32_t *q = qt + (u * 8 + b) * 64;
+    const uint32_t b0 = q[t * 8 + grp], b1 = q[(t + 4) * 8 + grp];
+    int32_t D[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    mma_s8_m16n8k32(D[0], A[0], b0, b1);
+    mma_s8_m16n8k32(D[1], A[1], b0, b1);
+    const float2 x = *reinterpret_cast<const float2 *>(dt + (u * 8 + b) * 8 + 2 * t);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int row = mma_row(v, grp);
+      const float dw = __half2float(*reinterpret_cast<const __half *>(box + row * 272 + 34 * b));
+      const int32_t sum = D[v >> 2][v & 3];
+      if (isum != nullptr && row < rows_left && mma_tok(v, t) < M)
+        isum[mma_tok(v, t) * isum_tok + row * isum_row + u * 8 + b] = sum;
+      part[v] += __fmul_rn(__fmul_rn(dw, (v & 1) ? x.y : x.x), static_cast<float>(sum));
+    }
+  }
+}
+
+// One Q4_K super-block of the warp's box against unit u: part[v] = sum over
+// sub-blocks j, in order, of xd * ((d*sc_j)*isum_j - (dmin*m_j)*xs_j).  The
+// lanes first decode their own row's eight (d*sc_j, dmin*m_j) into the warp's
+// scratch (lane = row), then read the pairs of the rows they hold.
+template <int M>
+__device__ __forceinline__ void tok_mma_q4_k(const uint8_t *box, const uint32_t *qt, const float *dt,
+                                             const int32_t *st, float *scr, int u, int lane, float (&part)[8],
+                                             int32_t *isum, int64_t isum_row, int64_t isum_tok,
+                                             int64_t rows_left) {
+  const int grp = lane >> 2, t = lane & 3;
+  {
+    const uint4 hdr = *reinterpret_cast<const uint4 *>(box + lane * 144);
+    const float d = tok_half_lo(hdr.x), dmin = tok_half_hi(hdr.x);
+    const uint32_t scA = hdr.y & 0x3f3f3f3fu, mA = hdr.z & 0x3f3f3f3fu;
+    const uint32_t scB = (hdr.w & 0x0f0f0f0fu) | ((hdr.y >> 2) & 0x30303030u);
+    const uint32_t mB = ((hdr.w >> 4) & 0x0f0f0f0fu) | ((hdr.z >> 2) & 0x30303030u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t scw = j < 4 ? scA : scB, mw = j < 4 ? mA : mB;
+      const int sh = 8 * (j & 3);
+      *reinterpret_cast<float2 *>(scr + lane * kTokScStride + 2 * j) =
+          make_float2(__fmul_rn(d, static_cast<float>((scw >> sh) & 0xffu)),
+                      __fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu)));
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int v = 0; v < 8; ++v) part[v] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t A[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t w = lds32(box + (grp + 8 * h + 16 * mt) * 144 + 16 + 32 * (j >> 1) + 4 * t + 16 * kk);
+          A[mt][h + 2 * kk] = (j & 1) ? ((w >> 4) & 0x0f0f0f0fu) : (w & 0x0f0f0f0fu);
+        }
+    const uint32_t *q = qt + (u * 8 + j) * 64;
+    const uint32_t b0 = q[t * 8 + grp], b1 = q[(t + 4) * 8 + grp];
+    int32_t D[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    mma_s8_m16n8k32(D[0], A[0], b0, b1);
+    mma_s8_m16n8k32(D[1], A[1], b0, b1);
+    const float2 x = *reinterpret_cast<const float2 *>(dt + (u * 8 + j) * 8 + 2 * t);
+    const int2 xs = *reinterpret_cast<const int2 *>(st + (u * 8 + j) * 8 + 2 * t);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int row = mma_row(v, grp);
+      const float2 sc = *reinterpret_cast<const float2 *>(scr + row * kTokScStride + 2 * j);
+      const int32_t sum = D[v >> 2][v & 3];
+      if (isum != nullptr && row < rows_left && mma_tok(v, t) < M)
+        isum[mma_tok(v, t) * isum_tok + row * isum_row + u * 8 + j] = sum;
+      const float tv = __fmul_rn(sc.x, static_cast<float>(sum));
+      const float vv = __fmul_rn(sc.y, static_cast<float>((v & 1) ? xs.y : xs.x));
+      part[v] += __fmul_rn((v & 1) ? x.y : x.x, __fsub_rn(tv, vv));
+    }
+  }
+  __syncwarp();   // the scratch is rewritten by the next unit
+}
+
+template <int TYPE, int M>
+__global__ void __launch_bounds__(kTokWarps * 32, 1)
+    gemv_tokens_mma_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
+                           const __grid_constant__ TokArgs a) {
+  constexpr int UB = tok_unit_bytes<TYPE>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, t = lane & 3;
+  const int W = a.W, S = a.stages;
+  const int vpw = warp < W ? a.G / W : 0;   // virtual lanes of this warp
+  uint32_t *qt = reinterpret_cast<uint32_t *>(base);
+  float *dt = reinterpret_cast<float *>(base + a.q_bytes);
+  int32_t *st = reinterpret_cast<int32_t *>(base + a.q_bytes + a.d_bytes);
+  uint8_t *ring = base + a.ring_off + static_cast<size_t>(warp) * S * a.box_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + a.bar_off) + 1 + warp * kTokMaxStages;
+  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][8 warps][M][32 rows]
+  float *scr = reinterpret_cast<float *>(base + a.sc_off) + warp * kTokRows * kTokScStride;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(
+      reinterpret_cast<uint64_t *>(base + a.bar_off) + 1 + kTokWarps * kTokMaxStages);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0u;
+    prefetch_tensormap(&map0);
+    prefetch_tensormap(&map1);
+  }
+  if (lane == 0)
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+  fence_barrier_init();
+  TokCursor issue;
+  issue.first(a, warp, vpw);
+  if (lane == 0) {
+    TokCursor c = issue;
+    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp, vpw)) {
+      const bool second = c.g >= a.groups0;
+      prefetch_l2_tile_2d(second ? &map1 : &map0, c.u * (UB / 4),
+                          static_cast<int32_t>((second ? c.g - a.groups0 : c.g) * kTokRows));
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+
+  int64_t n_issued = 0, n_waited = 0;
+  if (lane == 0) {
+    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp, vpw), ++n_issued)
+      tok_issue<UB>(&map0, &map1, a, issue, ring + static_cast<size_t>(s) * a.box_bytes, &bars[s]);
+  }
+  {
+    // the M tokens' prequantized activations, once, into the layout above
+    // (tokens M..7 zero), while the first weight boxes are in flight.  Each
+    // thread issues all of its 16-byte loads (one per token, unrolled) before
+    // it stores, so the copy costs about one L2 round trip.
+    const uint32_t q16 = static_cast<uint32_t>(a.K / 16), nb = static_cast<uint32_t>(a.K / 32);
+    const uint4 *xq4 = reinterpret_cast<const uint4 *>(a.xq);
+    for (uint32_t w4 = threadIdx.x; w4 < q16; w4 += blockDim.x) {
+      uint4 v[M];
+#pragma unroll
+      for (int tok = 0; tok < M; ++tok) v[tok] = __ldg(xq4 + tok * q16 + w4);
+#pragma unroll
+      for (int tok = 0; tok < 8; ++tok) {
+        const uint4 z = tok < M ? v[tok < M ? tok : 0] : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t *dst = qt + 4 * w4 * 8 + tok;   // words 4 w4 .. 4 w4 + 3 of this token
+        dst[0] = z.x; dst[8] = z.y; dst[16] = z.z; dst[24] = z.w;
+      }
+    }
+    for (uint32_t blk = threadIdx.x; blk < nb; blk += blockDim.x) {
+      float d[M];
+      int32_t sm[M];
+#pragma unroll
+      for (int tok = 0; tok < M; ++tok) {
+        d[tok] = __ldg(a.xd + tok * nb + blk);
+        sm[tok] = TYPE == DSQ_Q4_K ? __ldg(a.xs + tok * nb + blk) : 0;
+      }
+#pragma unroll
+      for (int tok = 0; tok < 8; ++tok) {
+        dt[blk * 8 + tok] = tok < M ? d[tok < M ? tok : 0] : 0.0f;
+        if (TYPE == DSQ_Q4_K) st[blk * 8 + tok] = tok < M ? sm[tok < M ? tok : 0] : 0;
+      }
+    }
+  }
+  __syncthreads();
+
+  bool ok = true;
+  int slot = 0;
+  uint32_t parity = 0;
+  int buf = 0;
+  const int64_t nb = a.K / 32;
+  const int64_t rows_total = a.n[0] + a.n[1];
+  for (int64_t g = blockIdx.x; g < a.total_groups; g += gridDim.x, buf ^= 1) {
+    const bool second = g >= a.groups0;
+    const int sgi = second ? 1 : 0;
+    const int64_t rbase = (second ? g - a.groups0 : g) * kTokRows;   // first row of the group in its weight
+    const int64_t vbase = (second ? a.n[0] : 0) + rbase;               // in [weight 0 rows, weight 1 rows]
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int v = 0; v < 8; ++v) acc[i][v] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i >= vpw) break;
+      for (int u = warp + W * i; u < a.nunits; u += a.G) {
+        ok = ok && *abort_flag == 0u;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
+        if (!ok) {
+          if (lane == 0 && *abort_flag == 0u) {
+            *abort_flag = 1u;
+            record_timeout(a.wait);
+          }
+        } else {
+          ++n_waited;
+          float part[8];
+          const uint8_t *box = ring + static_cast<size_t>(slot) * a.box_bytes;
+          int32_t *isum = a.isum ? a.isum + vbase * nb : nullptr;
+          const int64_t rows_left = a.n[sgi] - rbase;
+          if constexpr (TYPE == DSQ_Q8_0)
+            tok_mma_q8_0<M>(box, qt, dt, u, lane, part, isum, nb, rows_total * nb, rows_left);
+          else
+            tok_mma_q4_k<M>(box, qt, dt, st, scr, u, lane, part, isum, nb, rows_total * nb, rows_left);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) acc[i][v] += part[v];
+          __syncwarp();
+          if (lane == 0 && issue.valid(a)) {
+            fence_proxy_async_smem();
+            tok_issue<UB>(&map0, &map1, a, issue, ring + static_cast<size_t>(slot) * a.box_bytes, &bars[slot]);
+            issue.next(a, warp, vpw);
+            ++n_issued;
+          }
+        }
+        if (++slot == S) {
+          slot = 0;
+          parity ^= 1u;
+        }
+      }
+    }
+    // butterfly strides >= W inside the warp, as in the CUDA-core form
+    float *rb = red + static_cast<size_t>(buf) * kTokWarps * M * 32;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      float mine;
+      if (vpw == 4) mine = (acc[0][v] + acc[2][v]) + (acc[1][v] + acc[3][v]);
+      else if (vpw == 2) mine = acc[0][v] + acc[1][v];
+      else mine = acc[0][v];
+      const int tok = mma_tok(v, t);
+      if (tok < M) rb[(warp * M + tok) * 32 + mma_row(v, grp)] = mine;
+    }
+    __syncthreads();
+    // strides < W cross warps: ((r0+r4)+(r2+r6)) + ((r1+r5)+(r3+r7)) for W = 8
+    for (int m = warp; m < M; m += kTokWarps) {
+      float r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r[k] = k < W ? rb[(k * M + m) * 32 + lane] : 0.0f;
+      float v;
+      if (W == 8) v = ((r[0] + r[4]) + (r[2] + r[6])) + ((r[1] + r[5]) + (r[3] + r[7]));
+      else if (W == 4) v = (r[0] + r[2]) + (r[1] + r[3]);
+      else if (W == 2) v = r[0] + r[1];
+      else v = r[0];
+      const int64_t rloc = rbase + lane;
+      if (rloc < a.n[sgi] && *abort_flag == 0u) a.y[sgi][m * a.n[sgi] + rloc] = v;
+    }
+  }
+  if (lane == 0) {
+    for (int64_t k = n_waited; k < n_issued; ++k)
+      mbar_wait_for(&bars[k % S], static_cast<uint32_t>((k / S) & 1), kDrainLimitNs);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tok_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -402,38 +716,50 @@ int tok_map(CUtensorMap *map, const void *w, int type, int64_t N, int64_t K, con
   return DSQ_OK;
 }
 
+// The CUDA-core kernel below tok_mma_min_m(type) tokens; from there on the
+// tensor-core one, whenever its padded activation layout fits.
 template <int TYPE, int M>
-cudaError_t tok_launch(const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a, unsigned grid, size_t smem,
-                       cudaStream_t st) {
+const void *tok_kernel_m(bool mma) {
+  if constexpr (M >= kTokMmaMinM)
+    if (mma) return reinterpret_cast<const void *>(gemv_tokens_mma_kernel<TYPE, M>);
+  return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, M>);
+}
+
+template <int TYPE, int M>
+cudaError_t tok_launch(bool mma, const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a, unsigned grid,
+                       size_t smem, cudaStream_t st) {
+  if constexpr (M >= kTokMmaMinM)
+    if (mma)
+      return launch_pdl(gemv_tokens_mma_kernel<TYPE, M>, dim3(grid), dim3(kTokWarps * 32), smem, st, m0, m1, a);
   return launch_pdl(gemv_tokens_kernel<TYPE, M>, dim3(grid), dim3(kTokWarps * 32), smem, st, m0, m1, a);
 }
 
 template <int TYPE>
-const void *tok_kernel(int M) {
+const void *tok_kernel(int M, bool mma) {
   switch (M) {
-    case 1: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 1>);
-    case 2: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 2>);
-    case 3: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 3>);
-    case 4: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 4>);
-    case 5: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 5>);
-    case 6: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 6>);
-    case 7: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 7>);
-    default: return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, 8>);
+    case 1: return tok_kernel_m<TYPE, 1>(mma);
+    case 2: return tok_kernel_m<TYPE, 2>(mma);
+    case 3: return tok_kernel_m<TYPE, 3>(mma);
+    case 4: return tok_kernel_m<TYPE, 4>(mma);
+    case 5: return tok_kernel_m<TYPE, 5>(mma);
+    case 6: return tok_kernel_m<TYPE, 6>(mma);
+    case 7: return tok_kernel_m<TYPE, 7>(mma);
+    default: return tok_kernel_m<TYPE, 8>(mma);
   }
 }
 
 template <int TYPE>
-cudaError_t tok_dispatch(int M, const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a, unsigned grid,
-                         size_t smem, cudaStream_t st) {
+cudaError_t tok_dispatch(int M, bool mma, const CUtensorMap &m0, const CUtensorMap &m1, const TokArgs &a,
+                         unsigned grid, size_t smem, cudaStream_t st) {
   switch (M) {
-    case 1: return tok_launch<TYPE, 1>(m0, m1, a, grid, smem, st);
-    case 2: return tok_launch<TYPE, 2>(m0, m1, a, grid, smem, st);
-    case 3: return tok_launch<TYPE, 3>(m0, m1, a, grid, smem, st);
-    case 4: return tok_launch<TYPE, 4>(m0, m1, a, grid, smem, st);
-    case 5: return tok_launch<TYPE, 5>(m0, m1, a, grid, smem, st);
-    case 6: return tok_launch<TYPE, 6>(m0, m1, a, grid, smem, st);
-    case 7: return tok_launch<TYPE, 7>(m0, m1, a, grid, smem, st);
-    default: return tok_launch<TYPE, 8>(m0, m1, a, grid, smem, st);
+    case 1: return tok_launch<TYPE, 1>(mma, m0, m1, a, grid, smem, st);
+    case 2: return tok_launch<TYPE, 2>(mma, m0, m1, a, grid, smem, st);
+    case 3: return tok_launch<TYPE, 3>(mma, m0, m1, a, grid, smem, st);
+    case 4: return tok_launch<TYPE, 4>(mma, m0, m1, a, grid, smem, st);
+    case 5: return tok_launch<TYPE, 5>(mma, m0, m1, a, grid, smem, st);
+    case 6: return tok_launch<TYPE, 6>(mma, m0, m1, a, grid, smem, st);
+    case 7: return tok_launch<TYPE, 7>(mma, m0, m1, a, grid, smem, st);
+    default: return tok_launch<TYPE, 8>(mma, m0, m1, a, grid, smem, st);
   }
 }
 
@@ -448,8 +774,13 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
               kTokMaxM);
   DSQ_REQUIRE(K % 256 == 0, DSQ_ERR_SHAPE, "%s: K=%lld must be a multiple of 256", name, (long long)K);
   DSQ_REQUIRE(N0 + N1 <= (int64_t(1) << 31), DSQ_ERR_SHAPE, "%s: too many rows", name);
-  const size_t q_bytes = static_cast<size_t>(M) * K;
-  const size_t d_bytes = static_cast<size_t>(M) * (K / 32) * 4;
+  // the tensor-core form keeps 8 (padded) tokens in its own layout; where
+  // that does not fit, the CUDA-core kernel takes the call
+  const size_t per_token = static_cast<size_t>(K) + (K / 32) * 4 * (type == DSQ_Q4_K ? 2 : 1);
+  const bool mma = M >= tok_mma_min_m(type) && 8 * per_token <= kTokMaxActSmem;
+  const int64_t Mk = mma ? 8 : M;
+  const size_t q_bytes = static_cast<size_t>(Mk) * K;
+  const size_t d_bytes = static_cast<size_t>(Mk) * (K / 32) * 4;
   const size_t s_bytes = type == DSQ_Q4_K ? d_bytes : 0;
   DSQ_REQUIRE(q_bytes + d_bytes + s_bytes <= kTokMaxActSmem, DSQ_ERR_SHAPE,
               "%s: %lld tokens of K=%lld exceed the %zu bytes of shared memory kept for activations", name,
@@ -488,11 +819,13 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
   a.xs = xs;
   a.isum = isum;
   a.wait = ctl;
-  // shared memory: activations | ring (W warps x stages x box) | barriers | reduction
+  // shared memory: activations | ring (W warps x stages x box) | barriers |
+  // reduction | Q4_K scale scratch of the tensor-core form
   const size_t act = tok_align(q_bytes + d_bytes + s_bytes, 1024);
   const size_t bars = (1 + kTokWarps * kTokMaxStages + 1) * sizeof(uint64_t);
   const size_t red = 2 * static_cast<size_t>(kTokWarps) * M * 32 * sizeof(float);
-  const size_t fixed = 1024 + act + tok_align(bars, 16) + red;
+  const size_t scr = (mma && type == DSQ_Q4_K) ? static_cast<size_t>(kTokWarps) * kTokRows * kTokScStride * 4 : 0;
+  const size_t fixed = 1024 + act + tok_align(bars, 16) + red + scr;
   const size_t per_stage = static_cast<size_t>(kTokWarps) * a.box_bytes;
   int stages = static_cast<int>((kTokSmemLimit - fixed) / per_stage);
   if (stages > kTokMaxStages) stages = kTokMaxStages;
@@ -502,7 +835,8 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
   a.ring_off = static_cast<uint32_t>(act);
   a.bar_off = static_cast<uint32_t>(act + per_stage * stages);
   a.red_off = static_cast<uint32_t>(a.bar_off + tok_align(bars, 16));
-  const size_t smem = 1024 + a.red_off + red;
+  a.sc_off = static_cast<uint32_t>(a.red_off + red);
+  const size_t smem = 1024 + a.sc_off + scr;
 
   CUtensorMap m0, m1;
   const void *wa = N0 > 0 ? w0 : w1;
@@ -517,11 +851,11 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
   const int64_t slots = sms;
   const unsigned grid = static_cast<unsigned>(a.total_groups < slots ? a.total_groups : slots);
   const int mi = static_cast<int>(M);
-  rc = set_smem_once(type == DSQ_Q8_0 ? tok_kernel<DSQ_Q8_0>(mi) : tok_kernel<DSQ_Q4_K>(mi), static_cast<int>(smem),
-                     name);
+  rc = set_smem_once(type == DSQ_Q8_0 ? tok_kernel<DSQ_Q8_0>(mi, mma) : tok_kernel<DSQ_Q4_K>(mi, mma),
+                     static_cast<int>(smem), name);
   if (rc != DSQ_OK) return rc;
-  const cudaError_t e = type == DSQ_Q8_0 ? tok_dispatch<DSQ_Q8_0>(mi, m0, m1, a, grid, smem, stream)
-                                         : tok_dispatch<DSQ_Q4_K>(mi, m0, m1, a, grid, smem, stream);
+  const cudaError_t e = type == DSQ_Q8_0 ? tok_dispatch<DSQ_Q8_0>(mi, mma, m0, m1, a, grid, smem, stream)
+                                         : tok_dispatch<DSQ_Q4_K>(mi, mma, m0, m1, a, grid, smem, stream);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: %s", name, cudaGetErrorString(e));
   return after_launch(name);
 }
