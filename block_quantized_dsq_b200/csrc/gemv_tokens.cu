@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kTokWarps * 32, 1)
   if (threadIdx.x == 0 && !ok) mbar_wait_for(act_bar, 0, kDrainLimitNs);
 }
 
-// ------------------------------------------------------- 5 to 8 tokens ---
-// From 5 (Q8_0) or 7 (Q4_K) tokens on, the block dots run on the tensor cores: one
+// ------------------------------------------------------- 4 to 8 tokens ---
+// From 4 (Q8_0) or 5 (Q4_K) tokens on, the block dots run on the tensor cores: one
 // mma.sync.m16n8k32 (int8 x int8 -> int32) gives the exact block sums of one
 // 32-element block for 16 weight rows x 8 tokens.  Integer sums are exact
 // whoever forms them, and the lanes then form each fp32 block term and add
@@ -393,11 +393,11 @@ __global__ void __launch_bounds__(kTokWarps * 32, 1)
 //   scales and sums as [unit * 8 + block][token] -- lane reads tokens 2t, 2t+1.
 // The tensor-core form does the work of 8 tokens whatever M is, so it pays
 // only from a type-dependent token count on (interleaved A/B on one B200:
-// paired 2 x 8192 x 4096 Q8_0 at 4 / 6 / 8 tokens 21.9 / 22.9 / 22.7 us
-// against 20.3 / 26.7 / 33.9 on the CUDA cores; Q4_K 4096 x 4096 8.8 / 9.4 /
-// 9.3 us against 7.0 / 8.7 / 10.4).
-constexpr int kTokMmaMinM = 5;   // the smallest count any type takes it at
-__host__ __device__ constexpr int tok_mma_min_m(int type) { return type == DSQ_Q8_0 ? 5 : 7; }
+// paired 2 x 8192 x 4096 Q8_0 takes 18.6 us at any M against 15.8 / 20.3 /
+// 26.7 / 33.9 us for 2 / 4 / 6 / 8 tokens on the CUDA cores; Q4_K 4096 x 4096
+// 7.3 us against 7.0 / 8.7 / 10.4 us for 4 / 6 / 8 tokens).
+constexpr int kTokMmaMinM = 4;   // the smallest count any type takes it at
+__host__ __device__ constexpr int tok_mma_min_m(int type) { return type == DSQ_Q8_0 ? 4 : 5; }
 constexpr int kTokScStride = 18;   // words per row of the Q4_K scale scratch (8 pairs + pad)
 
 __device__ __forceinline__ void mma_s8_m16n8k32(int32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -418,7 +418,7 @@ __device__ __forceinline__ int mma_tok(int v, int t) { return 2 * t + (v & 1); }
 
 // One Q8_0 unit of the warp's 32-row box against unit u of the tokens:
 // part[v] = sum over the 8 blocks, in order, of (d_w * xd) * isum.
-template <int M>
+template <int M, bool ISUM>
 __device__ __forceinline__ void tok_mma_q8_0(const uint8_t *box, const uint32_t *qt, const float *dt, int u,
                                              int lane, float (&part)[8], int32_t *isum, int64_t isum_row,
                                              int64_t isum_tok, int64_t rows_left) {
@@ -444,14 +444,16 @@ __device__ __forceinline__ void tok_mma_q8_0(const uint8_t *box, const uint32_t 
     mma_s8_m16n8k32(D[0], A[0], b0, b1);
     mma_s8_m16n8k32(D[1], A[1], b0, b1);
     const float2 x = *reinterpret_cast<const float2 *>(dt + (u * 8 + b) * 8 + 2 * t);
+    float dw[4];   // rows grp, grp + 8, grp + 16, grp + 24
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      dw[r] = __half2float(*reinterpret_cast<const __half *>(box + (grp + 8 * r) * 272 + 34 * b));
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
-      const int row = mma_row(v, grp);
-      const float dw = __half2float(*reinterpret_cast<const __half *>(box + row * 272 + 34 * b));
       const int32_t sum = D[v >> 2][v & 3];
-      if (isum != nullptr && row < rows_left && mma_tok(v, t) < M)
-        isum[mma_tok(v, t) * isum_tok + row * isum_row + u * 8 + b] = sum;
-      part[v] += __fmul_rn(__fmul_rn(dw, (v & 1) ? x.y : x.x), static_cast<float>(sum));
+      if (ISUM && mma_row(v, grp) < rows_left && mma_tok(v, t) < M)
+        isum[mma_tok(v, t) * isum_tok + mma_row(v, grp) * isum_row + u * 8 + b] = sum;
+      part[v] += __fmul_rn(__fmul_rn(dw[v >> 1], (v & 1) ? x.y : x.x), static_cast<float>(sum));
     }
   }
 }
@@ -460,7 +462,7 @@ __device__ __forceinline__ void tok_mma_q8_0(const uint8_t *box, const uint32_t 
 // sub-blocks j, in order, of xd * ((d*sc_j)*isum_j - (dmin*m_j)*xs_j).  The
 // lanes first decode their own row's eight (d*sc_j, dmin*m_j) into the warp's
 // scratch (lane = row), then read the pairs of the rows they hold.
-template <int M>
+template <int M, bool ISUM>
 __device__ __forceinline__ void tok_mma_q4_k(const uint8_t *box, const uint32_t *qt, const float *dt,
                                              const int32_t *st, float *scr, int u, int lane, float (&part)[8],
                                              int32_t *isum, int64_t isum_row, int64_t isum_tok,
@@ -508,7 +510,7 @@ __device__ __forceinline__ void tok_mma_q4_k(const uint8_t *box, const uint32_t 
       const int row = mma_row(v, grp);
       const float2 sc = *reinterpret_cast<const float2 *>(scr + row * kTokScStride + 2 * j);
       const int32_t sum = D[v >> 2][v & 3];
-      if (isum != nullptr && row < rows_left && mma_tok(v, t) < M)
+      if (ISUM && row < rows_left && mma_tok(v, t) < M)
         isum[mma_tok(v, t) * isum_tok + row * isum_row + u * 8 + j] = sum;
       const float tv = __fmul_rn(sc.x, static_cast<float>(sum));
       const float vv = __fmul_rn(sc.y, static_cast<float>((v & 1) ? xs.y : xs.x));
@@ -518,7 +520,7 @@ __device__ __forceinline__ void tok_mma_q4_k(const uint8_t *box, const uint32_t 
   __syncwarp();   // the scratch is rewritten by the next unit
 }
 
-template <int TYPE, int M>
+template <int TYPE, int M, bool ISUM>
 __global__ void __launch_bounds__(kTokWarps * 32, 1)
     gemv_tokens_mma_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                            const __grid_constant__ TokArgs a) {
@@ -568,34 +570,36 @@ __global__ void __launch_bounds__(kTokWarps * 32, 1)
   }
   {
     // the M tokens' prequantized activations, once, into the layout above
-    // (tokens M..7 zero), while the first weight boxes are in flight.  Each
-    // thread issues all of its 16-byte loads (one per token, unrolled) before
-    // it stores, so the copy costs about one L2 round trip.
-    const uint32_t q16 = static_cast<uint32_t>(a.K / 16), nb = static_cast<uint32_t>(a.K / 32);
-    const uint4 *xq4 = reinterpret_cast<const uint4 *>(a.xq);
-    for (uint32_t w4 = threadIdx.x; w4 < q16; w4 += blockDim.x) {
-      uint4 v[M];
+    // (tokens M..7 zero), while the first weight boxes are in flight.  A
+    // thread takes one 4-code word of every token (coalesced across the
+    // warp) and stores them as two 16-byte words; its loads for four words
+    // are all in flight before it stores.
+    const uint32_t words = static_cast<uint32_t>(a.K / 4), nb = static_cast<uint32_t>(a.K / 32);
+    const uint32_t *xq32 = reinterpret_cast<const uint32_t *>(a.xq);
+#pragma unroll 4
+    for (uint32_t w = threadIdx.x; w < words; w += blockDim.x) {
+      uint32_t v[8];
 #pragma unroll
-      for (int tok = 0; tok < M; ++tok) v[tok] = __ldg(xq4 + tok * q16 + w4);
-#pragma unroll
-      for (int tok = 0; tok < 8; ++tok) {
-        const uint4 z = tok < M ? v[tok < M ? tok : 0] : make_uint4(0u, 0u, 0u, 0u);
-        uint32_t *dst = qt + 4 * w4 * 8 + tok;   // words 4 w4 .. 4 w4 + 3 of this token
-        dst[0] = z.x; dst[8] = z.y; dst[16] = z.z; dst[24] = z.w;
-      }
+      for (int tok = 0; tok < 8; ++tok) v[tok] = tok < M ? __ldg(xq32 + tok * words + w) : 0u;
+      uint4 *dst = reinterpret_cast<uint4 *>(qt + w * 8);
+      dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
     }
     for (uint32_t blk = threadIdx.x; blk < nb; blk += blockDim.x) {
-      float d[M];
-      int32_t sm[M];
-#pragma unroll
-      for (int tok = 0; tok < M; ++tok) {
-        d[tok] = __ldg(a.xd + tok * nb + blk);
-        sm[tok] = TYPE == DSQ_Q4_K ? __ldg(a.xs + tok * nb + blk) : 0;
-      }
+      float d[8];
+      int32_t sm[8];
 #pragma unroll
       for (int tok = 0; tok < 8; ++tok) {
-        dt[blk * 8 + tok] = tok < M ? d[tok < M ? tok : 0] : 0.0f;
-        if (TYPE == DSQ_Q4_K) st[blk * 8 + tok] = tok < M ? sm[tok < M ? tok : 0] : 0;
+        d[tok] = tok < M ? __ldg(a.xd + tok * nb + blk) : 0.0f;
+        sm[tok] = (TYPE == DSQ_Q4_K && tok < M) ? __ldg(a.xs + tok * nb + blk) : 0;
+      }
+      float4 *dd = reinterpret_cast<float4 *>(dt + blk * 8);
+      dd[0] = make_float4(d[0], d[1], d[2], d[3]);
+      dd[1] = make_float4(d[4], d[5], d[6], d[7]);
+      if (TYPE == DSQ_Q4_K) {
+        int4 *ds = reinterpret_cast<int4 *>(st + blk * 8);
+        ds[0] = make_int4(sm[0], sm[1], sm[2], sm[3]);
+        ds[1] = make_int4(sm[4], sm[5], sm[6], sm[7]);
       }
     }
   }
@@ -635,9 +639,9 @@ __global__ void __launch_bounds__(kTokWarps * 32, 1)
           int32_t *isum = a.isum ? a.isum + vbase * nb : nullptr;
           const int64_t rows_left = a.n[sgi] - rbase;
           if constexpr (TYPE == DSQ_Q8_0)
-            tok_mma_q8_0<M>(box, qt, dt, u, lane, part, isum, nb, rows_total * nb, rows_left);
+            tok_mma_q8_0<M, ISUM>(box, qt, dt, u, lane, part, isum, nb, rows_total * nb, rows_left);
           else
-            tok_mma_q4_k<M>(box, qt, dt, st, scr, u, lane, part, isum, nb, rows_total * nb, rows_left);
+            tok_mma_q4_k<M, ISUM>(box, qt, dt, st, scr, u, lane, part, isum, nb, rows_total * nb, rows_left);
 #pragma unroll
           for (int v = 0; v < 8; ++v) acc[i][v] += part[v];
           __syncwarp();
@@ -719,9 +723,11 @@ int tok_map(CUtensorMap *map, const void *w, int type, int64_t N, int64_t K, con
 // The CUDA-core kernel below tok_mma_min_m(type) tokens; from there on the
 // tensor-core one, whenever its padded activation layout fits.
 template <int TYPE, int M>
-const void *tok_kernel_m(bool mma) {
+const void *tok_kernel_m(bool mma, bool isum) {
   if constexpr (M >= kTokMmaMinM)
-    if (mma) return reinterpret_cast<const void *>(gemv_tokens_mma_kernel<TYPE, M>);
+    if (mma)
+      return isum ? reinterpret_cast<const void *>(gemv_tokens_mma_kernel<TYPE, M, true>)
+                  : reinterpret_cast<const void *>(gemv_tokens_mma_kernel<TYPE, M, false>);
   return reinterpret_cast<const void *>(gemv_tokens_kernel<TYPE, M>);
 }
 
@@ -730,21 +736,24 @@ cudaError_t tok_launch(bool mma, const CUtensorMap &m0, const CUtensorMap &m1, c
                        size_t smem, cudaStream_t st) {
   if constexpr (M >= kTokMmaMinM)
     if (mma)
-      return launch_pdl(gemv_tokens_mma_kernel<TYPE, M>, dim3(grid), dim3(kTokWarps * 32), smem, st, m0, m1, a);
+      return a.isum ? launch_pdl(gemv_tokens_mma_kernel<TYPE, M, true>, dim3(grid), dim3(kTokWarps * 32), smem, st,
+                                 m0, m1, a)
+                    : launch_pdl(gemv_tokens_mma_kernel<TYPE, M, false>, dim3(grid), dim3(kTokWarps * 32), smem, st,
+                                 m0, m1, a);
   return launch_pdl(gemv_tokens_kernel<TYPE, M>, dim3(grid), dim3(kTokWarps * 32), smem, st, m0, m1, a);
 }
 
 template <int TYPE>
-const void *tok_kernel(int M, bool mma) {
+const void *tok_kernel(int M, bool mma, bool isum) {
   switch (M) {
-    case 1: return tok_kernel_m<TYPE, 1>(mma);
-    case 2: return tok_kernel_m<TYPE, 2>(mma);
-    case 3: return tok_kernel_m<TYPE, 3>(mma);
-    case 4: return tok_kernel_m<TYPE, 4>(mma);
-    case 5: return tok_kernel_m<TYPE, 5>(mma);
-    case 6: return tok_kernel_m<TYPE, 6>(mma);
-    case 7: return tok_kernel_m<TYPE, 7>(mma);
-    default: return tok_kernel_m<TYPE, 8>(mma);
+    case 1: return tok_kernel_m<TYPE, 1>(mma, isum);
+    case 2: return tok_kernel_m<TYPE, 2>(mma, isum);
+    case 3: return tok_kernel_m<TYPE, 3>(mma, isum);
+    case 4: return tok_kernel_m<TYPE, 4>(mma, isum);
+    case 5: return tok_kernel_m<TYPE, 5>(mma, isum);
+    case 6: return tok_kernel_m<TYPE, 6>(mma, isum);
+    case 7: return tok_kernel_m<TYPE, 7>(mma, isum);
+    default: return tok_kernel_m<TYPE, 8>(mma, isum);
   }
 }
 
@@ -851,7 +860,8 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
   const int64_t slots = sms;
   const unsigned grid = static_cast<unsigned>(a.total_groups < slots ? a.total_groups : slots);
   const int mi = static_cast<int>(M);
-  rc = set_smem_once(type == DSQ_Q8_0 ? tok_kernel<DSQ_Q8_0>(mi, mma) : tok_kernel<DSQ_Q4_K>(mi, mma),
+  rc = set_smem_once(type == DSQ_Q8_0 ? tok_kernel<DSQ_Q8_0>(mi, mma, isum != nullptr)
+                                     : tok_kernel<DSQ_Q4_K>(mi, mma, isum != nullptr),
                      static_cast<int>(smem), name);
   if (rc != DSQ_OK) return rc;
   const cudaError_t e = type == DSQ_Q8_0 ? tok_dispatch<DSQ_Q8_0>(mi, mma, m0, m1, a, grid, smem, stream)

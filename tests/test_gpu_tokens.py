@@ -9,7 +9,7 @@ the oracle's fp64 integer-form GEMV.  Shapes cover one unit per row (G = 1),
 three units (G = 4, idle virtual lanes), several units per virtual lane
 (K = 12288), row counts below and across the 32-row groups, one weight empty,
 and the paired decode workload's full size, on both kernels: the CUDA-core one
-and, from 5 (Q8_0) or 7 (Q4_K) tokens, the tensor-core one.
+and, from 4 (Q8_0) or 5 (Q4_K) tokens, the tensor-core one.
 """
 import numpy as np
 import pytest
@@ -45,7 +45,8 @@ CASES = [(8, 1, 256, 1), (8, 7, 256, 3), (12, 33, 768, 2), (8, 100, 1024, 8), (1
          (8, 515, 4096, 8), (12, 4096, 4096, 8), (8, 129, 12288, 4), (12, 64, 12288, 2), (8, 64, 2048, 6),
          (12, 200, 4096, 7), (8, 8192, 4096, 3), (12, 6000, 2048, 5),   # several row groups per CTA
          (12, 300, 6144, 7),    # tensor-core form, 24 units: four virtual lanes per warp, some idle
-         (8, 300, 7168, 5)]     # 8 padded tokens would not fit: the CUDA-core form takes M = 5
+         (8, 300, 7168, 5),     # 8 padded tokens would not fit: the CUDA-core form takes M = 5
+         (12, 700, 4096, 4)]    # below the Q4_K threshold: the CUDA-core form
 
 
 @pytest.mark.parametrize("qtype,N,K,M", CASES)
