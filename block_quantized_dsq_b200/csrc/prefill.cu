@@ -869,8 +869,10 @@ struct SmallArgs {
   int64_t group0[kMaxGroup + 1];   // first 32-row group of each weight
   int64_t total_groups;
   const float *x;                  // [M][K] fp32
+  const __half *x16;               // mma form: [8][K] rounded activations (rows >= M zero)
+  const int32_t *shift;            // mma form: [M] row shifts
   int nunits, stages;
-  uint32_t box_bytes, ring_off, bar_off, red_off;
+  uint32_t box_bytes, ring_off, bar_off, red_off, sc_off;
   WaitCtl wait;
 };
 
@@ -1103,6 +1105,258 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
     for (int64_t k = n_waited; k < n_issued; ++k)
       mbar_wait_for(&bars[k % S], static_cast<uint32_t>((k / S) & 1), kDrainLimitNs);
   if (threadIdx.x == 0 && !ok) mbar_wait_for(act_bar, 0, kDrainLimitNs);
+}
+
+// ------------------------------------------- 4 to 8 tokens on mma.sync ---
+// Between the CUDA-core bridge and the CTA-pair pipeline.  One launch after
+// the activation rounding multiplies the tensor-core path's binary16 operands
+// -- the converters' formulas, element for element -- on the warp-level
+// tensor-core instruction mma.sync.m16n8k16 (fp16 operands, fp32
+// accumulation).  A warp takes a 32-row box of one K unit: two 16-row
+// m-tiles, 16 k-steps of 16.  Lane 4 grp + t dequantizes exactly the weights
+// its A fragments hold (rows grp and grp + 8 of each m-tile, eight elements
+// of each 32-element block, see mma_box), so every weight is converted once.
+// The activations sit in shared memory as 32-bit words of two binary16 K
+// elements, [k-step][pair][8 tokens] (tokens M..7 zero), so the B fragments
+// load without bank conflicts.  The 8 warps' partials meet in shared memory in a
+// fixed order, then each output is scaled back by 2^-s as in the epilogue of
+// the CTA-pair kernel.
+constexpr int kSmallMmaMaxM = 8;
+constexpr int kScrStride = 18;   // words per row of the Q4_K scale scratch (8 pairs + pad)
+
+__device__ __forceinline__ void mma_f16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                 uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Lane = row of the box: the binary16 range guard of the unit and, for Q4_K,
+// the eight (d*sc_j, -dmin*m_j) of the row into the warp's scratch.
+template <int TYPE>
+__device__ __forceinline__ void mma_row_prep(const uint8_t *row, float *scr, int lane, uint32_t *status) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+    uint32_t worst = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+      worst = max(worst, static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(row + 34 * b)) & 0x7fffu);
+    if (worst >= 0x6008u) record_range(status);
+  } else {
+    PairRegs<DSQ_Q4_K> r;
+    r.hdr = *reinterpret_cast<const uint4 *>(row);
+    if (!(pair_in_range<DSQ_Q4_K, 0>(r) && pair_in_range<DSQ_Q4_K, 1>(r))) record_range(status);
+    const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x & 0xffffu)));
+    const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(r.hdr.x >> 16)));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t scw, mw;
+      if (j < 4) {
+        scw = r.hdr.y & 0x3f3f3f3fu;
+        mw = r.hdr.z & 0x3f3f3f3fu;
+      } else {
+        scw = (r.hdr.w & 0x0f0f0f0fu) | ((r.hdr.y >> 2) & 0x30303030u);
+        mw = ((r.hdr.w >> 4) & 0x0f0f0f0fu) | ((r.hdr.z >> 2) & 0x30303030u);
+      }
+      const int sh = 8 * (j & 3);
+      *reinterpret_cast<float2 *>(scr + lane * kScrStride + 2 * j) =
+          make_float2(__fmul_rn(d, static_cast<float>((scw >> sh) & 0xffu)),
+                      -__fmul_rn(dmin, static_cast<float>((mw >> sh) & 0xffu)));
+    }
+  }
+}
+
+// The K order inside a 32-element block is free as long as both operands
+// follow it.  Lane 4 grp + t takes the block's elements 8t .. 8t+7 (one
+// contiguous run of codes, converted four or eight at a time as the
+// converters do): pairs p0 = (8t, 8t+1) and p1 = (8t+2, 8t+3) feed the first
+// k-step of the block as its (2t, 2t+1) and (2t+8, 2t+9) elements, p2 and p3
+// the second step; the activation layout is permuted to match when it is
+// filled.
+template <int TYPE>
+__device__ __forceinline__ void mma_row_pairs(const uint8_t *box, const float *scr, int r, int blk, int t,
+                                              uint32_t (&p)[4]) {
+  if constexpr (TYPE == DSQ_Q8_0) {
+    const uint8_t *rb = box + r * 272 + 34 * blk;
+    const __half2 d2 = __half2half2(*reinterpret_cast<const __half *>(rb));
+    uint32_t c0, c1;
+    if (blk & 1) {   // codes start word-aligned
+      c0 = *reinterpret_cast<const uint32_t *>(rb + 2 + 8 * t);
+      c1 = *reinterpret_cast<const uint32_t *>(rb + 6 + 8 * t);
+    } else {         // codes start 2 bytes past a word boundary
+      const uint32_t w0 = *reinterpret_cast<const uint32_t *>(rb + 8 * t);
+      const uint32_t w1 = *reinterpret_cast<const uint32_t *>(rb + 4 + 8 * t);
+      const uint32_t w2 = *reinterpret_cast<const uint32_t *>(rb + 8 + 8 * t);
+      c0 = __funnelshift_r(w0, w1, 16);
+      c1 = __funnelshift_r(w1, w2, 16);
+    }
+    q8x4_to_h(c0, d2, p[0], p[1]);
+    q8x4_to_h(c1, d2, p[2], p[3]);
+  } else {
+    const uint2 w = *reinterpret_cast<const uint2 *>(box + r * 144 + 16 + 32 * (blk >> 1) + 8 * t);
+    const bool high = blk & 1;
+    const uint32_t q0 = high ? (w.x >> 4) & 0x0f0f0f0fu : w.x & 0x0f0f0f0fu;
+    const uint32_t q1 = high ? (w.y >> 4) & 0x0f0f0f0fu : w.y & 0x0f0f0f0fu;
+    const float2 an = *reinterpret_cast<const float2 *>(scr + r * kScrStride + 2 * blk);
+    const uint64_t a2 = pack2(an.x, an.x), nb2 = pack2(an.y, an.y);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t q = i < 2 ? q0 : q1;
+      const int e = 2 * (i & 1);
+      const uint64_t f2 = pack2(__uint_as_float(__byte_perm(q, 0x4B000000u, 0x7540 + e)),
+                                __uint_as_float(__byte_perm(q, 0x4B000000u, 0x7540 + e + 1)));
+      const uint64_t v2 = fma2_rn(sub2_rn(f2, kMagic2), a2, nb2);
+      p[i] = h2_bits(__floats2half2_rn(lo_of(v2), hi_of(v2)));
+    }
+  }
+}
+
+// One box (32 rows x unit u) into the accumulators: acc[mt] holds rows
+// grp + 16 mt (+8) x tokens 2t, 2t + 1.
+template <int TYPE>
+__device__ __forceinline__ void mma_box(const uint8_t *box, const float *scr, const uint32_t *xa, int u, int grp,
+                                        int t, float (&acc)[2][4]) {
+#pragma unroll 2
+  for (int blk = 0; blk < 8; ++blk) {
+    uint32_t P[2][2][4];   // [m-tile][row half][pair]
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) mma_row_pairs<TYPE>(box, scr, grp + 8 * h + 16 * mt, blk, t, P[mt][h]);
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      const uint32_t *xk = xa + ((u * 16 + 2 * blk + st) * 8 + t) * 8 + grp;
+      const uint32_t b0 = xk[0], b1 = xk[32];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint32_t A[4] = {P[mt][0][2 * st], P[mt][1][2 * st], P[mt][0][2 * st + 1], P[mt][1][2 * st + 1]};
+        mma_f16_m16n8k16(acc[mt], A, b0, b1);
+      }
+    }
+  }
+}
+
+template <int TYPE, int M>
+__global__ void __launch_bounds__(kSmallWarps * 32, 1)
+    prefill_small_mma_kernel(const __grid_constant__ WeightMaps maps, const __grid_constant__ SmallArgs a) {
+  constexpr int UB = unit_bytes<TYPE>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, t = lane & 3;
+  const int S = a.stages;
+  uint32_t *xa = reinterpret_cast<uint32_t *>(base);   // [K/2][8]
+  uint8_t *ring = base + a.ring_off + static_cast<size_t>(warp) * S * a.box_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + a.bar_off) + warp * 2;
+  volatile uint32_t *abort_flag =
+      reinterpret_cast<volatile uint32_t *>(reinterpret_cast<uint64_t *>(base + a.bar_off) + 2 * kSmallWarps);
+  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][8 warps][M][32]
+  float *scr = reinterpret_cast<float *>(base + a.sc_off) + warp * kSmallRows * kScrStride;
+  __shared__ float scale_back[kSmallMmaMaxM];   // 2^-s_m
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0u;
+    for (int w = 0; w < a.G; ++w) prefetch_tensormap(&maps.m[w]);
+  }
+  if (lane == 0)
+    for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+  fence_barrier_init();
+  SmallCursor issue;
+  issue.first(a, warp);
+  if (lane == 0) {
+    // weights are read-only: this warp's first boxes toward L2 while the
+    // activation rounding before us finishes
+    SmallCursor c = issue;
+    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp)) {
+      const int w = small_weight_of(a, c.g);
+      prefetch_l2_tile_2d(&maps.m[w], c.u * (UB / 4), static_cast<int32_t>((c.g - a.group0[w]) * kSmallRows));
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+
+  int64_t n_issued = 0, n_waited = 0;
+  if (lane == 0)
+    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp), ++n_issued)
+      small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(s) * a.box_bytes, &bars[s]);
+  {
+    // the rounded activations into [k-step][pair][8 tokens] words in the
+    // permuted K order of mma_box: K pair q = 4t + c of a 32-element block
+    // (elements 2q, 2q+1) is pair t + 4 (c & 1) of the block's k-step c >> 1.
+    // A thread takes one pair of every token (coalesced across the warp) and
+    // stores two 16-byte words.
+    const uint32_t kp_n = static_cast<uint32_t>(a.K / 2);
+    const uint32_t *x32 = reinterpret_cast<const uint32_t *>(a.x16);
+#pragma unroll 4
+    for (uint32_t kp = threadIdx.x; kp < kp_n; kp += blockDim.x) {
+      uint32_t v[8];
+#pragma unroll
+      for (int tok = 0; tok < 8; ++tok) v[tok] = tok < M ? __ldg(x32 + tok * kp_n + kp) : 0u;
+      const uint32_t blk32 = kp >> 4, q = kp & 15u, tq = q >> 2, c = q & 3u;   // block of 32 (unit*8 + block)
+      const uint32_t slot = ((2u * blk32 + (c >> 1)) * 8u + tq + 4u * (c & 1u)) * 8u;
+      uint4 *dst = reinterpret_cast<uint4 *>(xa + slot);
+      dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
+    }
+    if (threadIdx.x < M) scale_back[threadIdx.x] = __int_as_float((127 - __ldg(a.shift + threadIdx.x)) << 23);
+  }
+  __syncthreads();
+
+  bool ok = true;
+  int slot = 0;
+  uint32_t parity = 0;
+  int buf = 0;
+  for (int64_t g = blockIdx.x; g < a.total_groups; g += gridDim.x, buf ^= 1) {
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int u = warp; u < a.nunits; u += kSmallWarps) {
+      ok = ok && *abort_flag == 0u;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
+      if (!ok) {
+        if (lane == 0 && *abort_flag == 0u) {
+          *abort_flag = 1u;
+          record_timeout(a.wait);
+        }
+      } else {
+        ++n_waited;
+        const uint8_t *box = ring + static_cast<size_t>(slot) * a.box_bytes;
+        mma_row_prep<TYPE>(box + static_cast<size_t>(lane) * UB, scr, lane, a.wait.status);
+        __syncwarp();
+        mma_box<TYPE>(box, scr, xa, u, grp, t, acc);
+        __syncwarp();
+        if (lane == 0 && issue.valid(a)) {
+          fence_proxy_async_smem();
+          small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(slot) * a.box_bytes, &bars[slot]);
+          issue.next(a, warp);
+          ++n_issued;
+        }
+      }
+      if (++slot == S) {
+        slot = 0;
+        parity ^= 1u;
+      }
+    }
+    float *rb = red + static_cast<size_t>(buf) * kSmallWarps * M * 32;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int tok = 2 * t + (c & 1), row = grp + 8 * (c >> 1) + 16 * mt;
+        if (tok < M) rb[(warp * M + tok) * 32 + row] = acc[mt][c];
+      }
+    __syncthreads();
+    for (int m = warp; m < M; m += kSmallWarps) {
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kSmallWarps; ++w) v += rb[(w * M + m) * 32 + lane];
+      const int wi = small_weight_of(a, g);
+      const int64_t row = (g - a.group0[wi]) * kSmallRows + lane;
+      if (row < a.N[wi] && *abort_flag == 0u) a.y[wi][m * a.N[wi] + row] = __fmul_rn(v, scale_back[m]);
+    }
+  }
+  if (lane == 0)
+    for (int64_t k = n_waited; k < n_issued; ++k)
+      mbar_wait_for(&bars[k % S], static_cast<uint32_t>((k / S) & 1), kDrainLimitNs);
 }
 
 // ------------------------------------------------------------------- host --
@@ -1379,6 +1633,135 @@ int run_prefill_small(const char *name, int type, int G, const void *const *w, c
   return after_launch(name);
 }
 
+// ---- 4 to 8 tokens on mma.sync: plan and launch ----
+// Workspace: the rounded activations [8][K] binary16 (rows >= M zero), then
+// the row shifts.
+size_t small_mma_workspace(int64_t K) { return align_up(static_cast<size_t>(8) * K * 2, 256) + 256; }
+
+// Shared memory of the mma.sync form for `stages` ring slots per warp:
+// activations [K/2][8] words | ring | barriers | reduction [2][8][M][32] |
+// Q4_K scale scratch.
+size_t small_mma_smem(int type, int64_t K, int64_t M, int stages, SmallArgs *a) {
+  const size_t act = align_up(static_cast<size_t>(K) * 16, 1024);
+  const size_t box = static_cast<size_t>(kSmallRows) * (type == DSQ_Q8_0 ? 272 : 144);
+  const size_t bars = align_up((2 * kSmallWarps + 1) * sizeof(uint64_t), 128);
+  const size_t red = 2 * static_cast<size_t>(kSmallWarps) * M * 32 * sizeof(float);
+  const size_t scr = type == DSQ_Q4_K ? static_cast<size_t>(kSmallWarps) * kSmallRows * kScrStride * 4 : 0;
+  if (a) {
+    a->box_bytes = static_cast<uint32_t>(box);
+    a->ring_off = static_cast<uint32_t>(act);
+    a->bar_off = static_cast<uint32_t>(act + kSmallWarps * box * stages);
+    a->red_off = static_cast<uint32_t>(a->bar_off + bars);
+    a->sc_off = static_cast<uint32_t>(a->red_off + red);
+  }
+  return 1024 + act + kSmallWarps * box * stages + bars + red + scr;
+}
+
+// Where the mma.sync form takes the call: above the CUDA-core bridge, up to 8
+// tokens, with two ring slots per warp next to its activations.
+bool small_mma_fits(int type, int64_t K, int64_t M) {
+  return M > small_max_m(type) && M <= kSmallMmaMaxM && small_mma_smem(type, K, M, 2, nullptr) <= kSmallPipeSmem;
+}
+
+template <int TYPE>
+const void *small_mma_kernel_ptr(int M) {
+  switch (M) {
+    case 1: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 1>);
+    case 2: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 2>);
+    case 3: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 3>);
+    case 4: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 4>);
+    case 5: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 5>);
+    case 6: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 6>);
+    case 7: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 7>);
+    default: return reinterpret_cast<const void *>(prefill_small_mma_kernel<TYPE, 8>);
+  }
+}
+
+template <int TYPE, int M>
+cudaError_t small_mma_launch(const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem, cudaStream_t st) {
+  return launch_pdl(prefill_small_mma_kernel<TYPE, M>, dim3(grid), dim3(kSmallWarps * 32), smem, st, maps, a);
+}
+
+template <int TYPE>
+cudaError_t small_mma_dispatch(int M, const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem,
+                               cudaStream_t st) {
+  switch (M) {
+    case 1: return small_mma_launch<TYPE, 1>(maps, a, grid, smem, st);
+    case 2: return small_mma_launch<TYPE, 2>(maps, a, grid, smem, st);
+    case 3: return small_mma_launch<TYPE, 3>(maps, a, grid, smem, st);
+    case 4: return small_mma_launch<TYPE, 4>(maps, a, grid, smem, st);
+    case 5: return small_mma_launch<TYPE, 5>(maps, a, grid, smem, st);
+    case 6: return small_mma_launch<TYPE, 6>(maps, a, grid, smem, st);
+    case 7: return small_mma_launch<TYPE, 7>(maps, a, grid, smem, st);
+    default: return small_mma_launch<TYPE, 8>(maps, a, grid, smem, st);
+  }
+}
+
+int run_prefill_small_mma(const char *name, int type, int G, const void *const *w, const int64_t *N, int64_t K,
+                          const float *x, int64_t M, float *const *y, void *workspace, size_t workspace_bytes,
+                          const WaitCtl &ctl, int sms, cudaStream_t st) {
+  const size_t need = small_mma_workspace(K);
+  DSQ_REQUIRE(workspace != nullptr && workspace_bytes >= need, DSQ_ERR_WORKSPACE,
+              "%s: workspace of %zu bytes needed, %zu given", name, need, workspace_bytes);
+  DSQ_REQUIRE(aligned(workspace, 256), DSQ_ERR_ALIGNMENT, "%s: workspace must be 256-byte aligned", name);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  __half *x16 = reinterpret_cast<__half *>(ws);
+  int32_t *shift = reinterpret_cast<int32_t *>(ws + need - 256);
+  SmallArgs a{};
+  a.K = K;
+  a.M = M;
+  a.G = G;
+  int64_t g0 = 0;
+  for (int g = 0; g < kMaxGroup; ++g) {
+    const bool used = g < G;
+    a.N[g] = used ? N[g] : 1;
+    a.y[g] = used ? y[g] : nullptr;
+    a.group0[g] = g0;
+    if (used) g0 += (N[g] + kSmallRows - 1) / kSmallRows;
+  }
+  a.group0[kMaxGroup] = g0;
+  a.total_groups = g0;
+  a.x16 = x16;
+  a.shift = shift;
+  a.nunits = static_cast<int>(K / 256);
+  a.wait = ctl;
+  a.stages = 2;
+  const size_t smem = small_mma_smem(type, K, M, a.stages, &a);
+  DSQ_REQUIRE(smem <= kSmallPipeSmem, DSQ_ERR_SHAPE, "%s: no pipeline fits next to the activations of K=%lld", name,
+              (long long)K);
+
+  auto enc = encode_fn();
+  DSQ_REQUIRE(enc != nullptr, DSQ_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+  WeightMaps maps;
+  const int64_t rb = static_cast<int64_t>(dsq_row_bytes(type, K));
+  for (int g = 0; g < G; ++g) {
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(rb / 4), static_cast<cuuint64_t>(N[g])};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {type == DSQ_Q8_0 ? 68u : 36u, static_cast<cuuint32_t>(kSmallRows)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&maps.m[g], CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(w[g]), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    DSQ_REQUIRE(cr == CUDA_SUCCESS, DSQ_ERR_CUDA, "%s: weight tensor map %d (%d)", name, g, (int)cr);
+  }
+  for (int g = G; g < kMaxGroup; ++g) maps.m[g] = maps.m[0];
+
+  // the activation rounding of the tensor-core path, row-major, 8 rows
+  cudaError_t e = launch_pdl(x_to_f16_kernel<false>, dim3(8u), dim3(256), 0, st, x, M, K, int64_t(8), x16, shift);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: x_to_f16: %s", name, cudaGetErrorString(e));
+  int rc = after_launch(name);
+  if (rc != DSQ_OK) return rc;
+  const int mi = static_cast<int>(M);
+  rc = set_smem_once(type == DSQ_Q8_0 ? small_mma_kernel_ptr<DSQ_Q8_0>(mi) : small_mma_kernel_ptr<DSQ_Q4_K>(mi),
+                     static_cast<int>(smem), name);
+  if (rc != DSQ_OK) return rc;
+  const unsigned grid = static_cast<unsigned>(a.total_groups < sms ? a.total_groups : sms);
+  e = type == DSQ_Q8_0 ? small_mma_dispatch<DSQ_Q8_0>(mi, maps, a, grid, smem, st)
+                       : small_mma_dispatch<DSQ_Q4_K>(mi, maps, a, grid, smem, st);
+  if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: %s", name, cudaGetErrorString(e));
+  return after_launch(name);
+}
+
 // Argument checks shared by the prefill entry points (nothing launched on
 // failure).
 int validate_group(const char *name, int type, int64_t G, const void *const *w, const int64_t *N, int64_t K,
@@ -1405,6 +1788,7 @@ size_t group_workspace_bytes(int type, int64_t G, const int64_t *N, int64_t K, i
   for (int64_t g = 0; g < G; ++g)
     if (N[g] < 1) return 0;
   if (small_fits(type, K, M)) return kSmallWorkspace;
+  if (small_mma_fits(type, K, M)) return small_mma_workspace(K);
   int sms = 148;
   if (device_ready(nullptr, &sms) != DSQ_OK) sms = 148;
   return make_plan(type, static_cast<int>(G), N, K, M, sms, -1).total;
@@ -1424,6 +1808,8 @@ int run_prefill(const char *name, int type, int64_t G, const void *const *w, con
   const int Gi = static_cast<int>(G);
   if (small_fits(type, K, M))
     return run_prefill_small(name, type, Gi, w, N, K, x, M, y, workspace, workspace_bytes, ctl, sms, st);
+  if (small_mma_fits(type, K, M))
+    return run_prefill_small_mma(name, type, Gi, w, N, K, x, M, y, workspace, workspace_bytes, ctl, sms, st);
   const Plan p = make_plan(type, Gi, N, K, M, sms, -1);
   DSQ_REQUIRE(p.total_tiles < (int64_t(1) << 31), DSQ_ERR_SHAPE, "%s: %lld tiles exceed one launch", name,
               static_cast<long long>(p.total_tiles));
