@@ -885,8 +885,8 @@ struct SmallCursor {
     u = warp;
     if (u >= a.nunits) g = a.total_groups;
   }
-  __device__ __forceinline__ void next(const SmallArgs &a, int warp) {
-    u += kSmallWarps;
+  __device__ __forceinline__ void next(const SmallArgs &a, int warp, int nw = kSmallWarps) {
+    u += nw;
     if (u >= a.nunits) {
       u = warp;
       g += gridDim.x;
@@ -1122,6 +1122,11 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
 // fixed order, then each output is scaled back by 2^-s as in the epilogue of
 // the CTA-pair kernel.
 constexpr int kSmallMmaMaxM = 8;
+// Warps per CTA and ring slots per warp: Q4_K boxes are small enough for 16
+// warps with one slot each (more latency hidden; a 4096-row weight is then
+// one box per warp), Q8_0 keeps 8 warps with two slots.
+__host__ __device__ constexpr int small_mma_warps(int type) { return type == DSQ_Q4_K ? 16 : 8; }
+__host__ __device__ constexpr int small_mma_stages(int type) { return type == DSQ_Q4_K ? 1 : 2; }
 constexpr int kScrStride = 18;   // words per row of the Q4_K scale scratch (8 pairs + pad)
 
 __device__ __forceinline__ void mma_f16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -1238,9 +1243,10 @@ __device__ __forceinline__ void mma_box(const uint8_t *box, const float *scr, co
 }
 
 template <int TYPE, int M>
-__global__ void __launch_bounds__(kSmallWarps * 32, 1)
+__global__ void __launch_bounds__(small_mma_warps(TYPE) * 32, 1)
     prefill_small_mma_kernel(const __grid_constant__ WeightMaps maps, const __grid_constant__ SmallArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
+  constexpr int NW = small_mma_warps(TYPE);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, t = lane & 3;
@@ -1249,8 +1255,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
   uint8_t *ring = base + a.ring_off + static_cast<size_t>(warp) * S * a.box_bytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(base + a.bar_off) + warp * 2;
   volatile uint32_t *abort_flag =
-      reinterpret_cast<volatile uint32_t *>(reinterpret_cast<uint64_t *>(base + a.bar_off) + 2 * kSmallWarps);
-  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][8 warps][M][32]
+      reinterpret_cast<volatile uint32_t *>(reinterpret_cast<uint64_t *>(base + a.bar_off) + 2 * NW);
+  float *red = reinterpret_cast<float *>(base + a.red_off);   // [2][NW warps][M][32]
   float *scr = reinterpret_cast<float *>(base + a.sc_off) + warp * kSmallRows * kScrStride;
   __shared__ float scale_back[kSmallMmaMaxM];   // 2^-s_m
 
@@ -1267,7 +1273,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
     // weights are read-only: this warp's first boxes toward L2 while the
     // activation rounding before us finishes
     SmallCursor c = issue;
-    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp)) {
+    for (int s = 0; s < S && c.valid(a); ++s, c.next(a, warp, NW)) {
       const int w = small_weight_of(a, c.g);
       prefetch_l2_tile_2d(&maps.m[w], c.u * (UB / 4), static_cast<int32_t>((c.g - a.group0[w]) * kSmallRows));
     }
@@ -1278,7 +1284,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
 
   int64_t n_issued = 0, n_waited = 0;
   if (lane == 0)
-    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp), ++n_issued)
+    for (int s = 0; s < S && issue.valid(a); ++s, issue.next(a, warp, NW), ++n_issued)
       small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(s) * a.box_bytes, &bars[s]);
   {
     // the rounded activations into [k-step][pair][8 tokens] words in the
@@ -1309,7 +1315,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
   int buf = 0;
   for (int64_t g = blockIdx.x; g < a.total_groups; g += gridDim.x, buf ^= 1) {
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int u = warp; u < a.nunits; u += kSmallWarps) {
+    for (int u = warp; u < a.nunits; u += NW) {
       ok = ok && *abort_flag == 0u;
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_for(&bars[slot], parity, a.wait.limit_ns));
       if (!ok) {
@@ -1327,7 +1333,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
         if (lane == 0 && issue.valid(a)) {
           fence_proxy_async_smem();
           small_issue<UB>(maps, a, issue, ring + static_cast<size_t>(slot) * a.box_bytes, &bars[slot]);
-          issue.next(a, warp);
+          issue.next(a, warp, NW);
           ++n_issued;
         }
       }
@@ -1336,7 +1342,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
         parity ^= 1u;
       }
     }
-    float *rb = red + static_cast<size_t>(buf) * kSmallWarps * M * 32;
+    float *rb = red + static_cast<size_t>(buf) * NW * M * 32;
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -1345,10 +1351,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
         if (tok < M) rb[(warp * M + tok) * 32 + row] = acc[mt][c];
       }
     __syncthreads();
-    for (int m = warp; m < M; m += kSmallWarps) {
+    for (int m = warp; m < M; m += NW) {
       float v = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kSmallWarps; ++w) v += rb[(w * M + m) * 32 + lane];
+      for (int w = 0; w < NW; ++w) v += rb[(w * M + m) * 32 + lane];
       const int wi = small_weight_of(a, g);
       const int64_t row = (g - a.group0[wi]) * kSmallRows + lane;
       if (row < a.N[wi] && *abort_flag == 0u) a.y[wi][m * a.N[wi] + row] = __fmul_rn(v, scale_back[m]);
@@ -1642,25 +1648,27 @@ size_t small_mma_workspace(int64_t K) { return align_up(static_cast<size_t>(8) *
 // activations [K/2][8] words | ring | barriers | reduction [2][8][M][32] |
 // Q4_K scale scratch.
 size_t small_mma_smem(int type, int64_t K, int64_t M, int stages, SmallArgs *a) {
+  const size_t nw = static_cast<size_t>(small_mma_warps(type));
   const size_t act = align_up(static_cast<size_t>(K) * 16, 1024);
   const size_t box = static_cast<size_t>(kSmallRows) * (type == DSQ_Q8_0 ? 272 : 144);
-  const size_t bars = align_up((2 * kSmallWarps + 1) * sizeof(uint64_t), 128);
-  const size_t red = 2 * static_cast<size_t>(kSmallWarps) * M * 32 * sizeof(float);
-  const size_t scr = type == DSQ_Q4_K ? static_cast<size_t>(kSmallWarps) * kSmallRows * kScrStride * 4 : 0;
+  const size_t bars = align_up((2 * nw + 1) * sizeof(uint64_t), 128);
+  const size_t red = 2 * nw * M * 32 * sizeof(float);
+  const size_t scr = type == DSQ_Q4_K ? nw * kSmallRows * kScrStride * 4 : 0;
   if (a) {
     a->box_bytes = static_cast<uint32_t>(box);
     a->ring_off = static_cast<uint32_t>(act);
-    a->bar_off = static_cast<uint32_t>(act + kSmallWarps * box * stages);
+    a->bar_off = static_cast<uint32_t>(act + nw * box * stages);
     a->red_off = static_cast<uint32_t>(a->bar_off + bars);
     a->sc_off = static_cast<uint32_t>(a->red_off + red);
   }
-  return 1024 + act + kSmallWarps * box * stages + bars + red + scr;
+  return 1024 + act + nw * box * stages + bars + red + scr;
 }
 
 // Where the mma.sync form takes the call: above the CUDA-core bridge, up to 8
-// tokens, with two ring slots per warp next to its activations.
+// tokens, with its ring slots next to its activations.
 bool small_mma_fits(int type, int64_t K, int64_t M) {
-  return M > small_max_m(type) && M <= kSmallMmaMaxM && small_mma_smem(type, K, M, 2, nullptr) <= kSmallPipeSmem;
+  return M > small_max_m(type) && M <= kSmallMmaMaxM &&
+         small_mma_smem(type, K, M, small_mma_stages(type), nullptr) <= kSmallPipeSmem;
 }
 
 template <int TYPE>
@@ -1679,7 +1687,8 @@ const void *small_mma_kernel_ptr(int M) {
 
 template <int TYPE, int M>
 cudaError_t small_mma_launch(const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem, cudaStream_t st) {
-  return launch_pdl(prefill_small_mma_kernel<TYPE, M>, dim3(grid), dim3(kSmallWarps * 32), smem, st, maps, a);
+  return launch_pdl(prefill_small_mma_kernel<TYPE, M>, dim3(grid), dim3(small_mma_warps(TYPE) * 32), smem, st, maps,
+                    a);
 }
 
 template <int TYPE>
@@ -1725,7 +1734,7 @@ int run_prefill_small_mma(const char *name, int type, int G, const void *const *
   a.shift = shift;
   a.nunits = static_cast<int>(K / 256);
   a.wait = ctl;
-  a.stages = 2;
+  a.stages = small_mma_stages(type);
   const size_t smem = small_mma_smem(type, K, M, a.stages, &a);
   DSQ_REQUIRE(smem <= kSmallPipeSmem, DSQ_ERR_SHAPE, "%s: no pipeline fits next to the activations of K=%lld", name,
               (long long)K);
