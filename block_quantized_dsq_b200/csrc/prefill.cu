@@ -839,7 +839,7 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 }
 
 // ------------------------------------------------------ small-M bridge --
-// For one to three tokens the tensor-core pipeline is all fill and drain: the
+// For one or two tokens the tensor-core pipeline is all fill and drain: the
 // weights stream once, but three launches (activation rounding, GEMM, split
 // reduction) and the pair pipeline's start-up dominate.  Those token counts
 // (small_max_m below, chosen from the measured sweep) take this CUDA-core
@@ -1537,12 +1537,12 @@ constexpr size_t kSmallWorkspace = 256;
 
 size_t small_act_bytes(int64_t K, int64_t M) { return static_cast<size_t>(M) * K * 4; }
 
-// Where the small-M kernel beats the tensor-core pipeline (measured on B200
-// with K = 4096: Q4_K up to 3 tokens, 8.6 / 10.6 us against 15.7 us at 1 / 2
-// tokens for 4096 rows; Q8_0 up to 2 tokens, 13.9 / 17.2 us against 19.2 /
-// 19.5 us for 8192 rows; from 4 tokens on its CUDA-core products cost more
-// than the tensor-core pipeline's fixed start-up).
-int small_max_m(int type) { return type == DSQ_Q4_K ? 3 : 2; }   // at most kSmallMaxM
+// Where the CUDA-core kernel beats the mma.sync bridge above it (interleaved
+// A/B on one B200, K = 4096): Q4_K only at 1 token (8.6 us for 4096 rows; at
+// 2 / 3 tokens 10.6 / 12.6 us against 10.1 / 10.2 us, and 30.7 against 26.5
+// us for 16384 rows at 2 tokens); Q8_0 up to 2 tokens (17.3 against 17.0 us
+// for 8192 rows, but 9.6 against 11.0 us for 2048 rows).
+int small_max_m(int type) { return type == DSQ_Q4_K ? 1 : 2; }   // at most kSmallMaxM
 
 bool small_fits(int type, int64_t K, int64_t M) {
   return M >= 1 && M <= small_max_m(type) && small_act_bytes(K, M) <= kSmallMaxActSmem;
