@@ -839,7 +839,7 @@ __global__ void __launch_bounds__(128) w_to_f16_kernel(const uint8_t *__restrict
 }
 
 // ------------------------------------------------------ small-M bridge --
-// For one or two tokens the tensor-core pipeline is all fill and drain: the
+// For a single token the tensor-core pipeline is all fill and drain: the
 // weights stream once, but three launches (activation rounding, GEMM, split
 // reduction) and the pair pipeline's start-up dominate.  Those token counts
 // (small_max_m below, chosen from the measured sweep) take this CUDA-core
@@ -1122,11 +1122,13 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1)
 // fixed order, then each output is scaled back by 2^-s as in the epilogue of
 // the CTA-pair kernel.
 constexpr int kSmallMmaMaxM = 8;
-// Warps per CTA and ring slots per warp: Q4_K boxes are small enough for 16
-// warps with one slot each (more latency hidden; a 4096-row weight is then
-// one box per warp), Q8_0 keeps 8 warps with two slots.
-__host__ __device__ constexpr int small_mma_warps(int type) { return type == DSQ_Q4_K ? 16 : 8; }
-__host__ __device__ constexpr int small_mma_stages(int type) { return type == DSQ_Q4_K ? 1 : 2; }
+// 16 warps per CTA with one ring slot each (more latency hidden than 8 warps
+// with two; a 4096-row weight is one box per warp).  Q8_0's larger boxes
+// leave room for only one reduction buffer, so its CTAs take a second
+// barrier per row group before the buffer is reused.
+__host__ __device__ constexpr int small_mma_warps(int) { return 16; }
+__host__ __device__ constexpr int small_mma_stages(int) { return 1; }
+__host__ __device__ constexpr int small_mma_red_bufs(int type) { return type == DSQ_Q4_K ? 2 : 1; }
 constexpr int kScrStride = 18;   // words per row of the Q4_K scale scratch (8 pairs + pad)
 
 __device__ __forceinline__ void mma_f16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -1342,7 +1344,7 @@ __global__ void __launch_bounds__(small_mma_warps(TYPE) * 32, 1)
         parity ^= 1u;
       }
     }
-    float *rb = red + static_cast<size_t>(buf) * NW * M * 32;
+    float *rb = red + static_cast<size_t>(small_mma_red_bufs(TYPE) == 2 ? buf : 0) * NW * M * 32;
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -1359,6 +1361,7 @@ __global__ void __launch_bounds__(small_mma_warps(TYPE) * 32, 1)
       const int64_t row = (g - a.group0[wi]) * kSmallRows + lane;
       if (row < a.N[wi] && *abort_flag == 0u) a.y[wi][m * a.N[wi] + row] = __fmul_rn(v, scale_back[m]);
     }
+    if (small_mma_red_bufs(TYPE) == 1) __syncthreads();   // the single buffer is rewritten by the next group
   }
   if (lane == 0)
     for (int64_t k = n_waited; k < n_issued; ++k)
@@ -1538,11 +1541,10 @@ constexpr size_t kSmallWorkspace = 256;
 size_t small_act_bytes(int64_t K, int64_t M) { return static_cast<size_t>(M) * K * 4; }
 
 // Where the CUDA-core kernel beats the mma.sync bridge above it (interleaved
-// A/B on one B200, K = 4096): Q4_K only at 1 token (8.6 us for 4096 rows; at
-// 2 / 3 tokens 10.6 / 12.6 us against 10.1 / 10.2 us, and 30.7 against 26.5
-// us for 16384 rows at 2 tokens); Q8_0 up to 2 tokens (17.3 against 17.0 us
-// for 8192 rows, but 9.6 against 11.0 us for 2048 rows).
-int small_max_m(int type) { return type == DSQ_Q4_K ? 1 : 2; }   // at most kSmallMaxM
+// A/B on one B200, K = 4096): one token only.  At 2 tokens the bridge takes
+// Q4_K 4096 rows in 10.1 against 10.6 us (16384 rows: 26.5 against 30.7)
+// and Q8_0 8192 rows in 15.1 against 17.3 us (1024 rows: 9.0 against 9.4).
+int small_max_m(int) { return 1; }   // at most kSmallMaxM
 
 bool small_fits(int type, int64_t K, int64_t M) {
   return M >= 1 && M <= small_max_m(type) && small_act_bytes(K, M) <= kSmallMaxActSmem;
@@ -1553,23 +1555,17 @@ cudaError_t small_launch(const WeightMaps &maps, const SmallArgs &a, unsigned gr
   return launch_pdl(prefill_small_kernel<TYPE, M>, dim3(grid), dim3(kSmallWarps * 32), smem, st, maps, a);
 }
 
+// small_max_m is 1: the kernel is instantiated for a single token (the
+// template takes up to kSmallMaxM).
 template <int TYPE>
-const void *small_kernel_ptr(int M) {
-  switch (M) {
-    case 1: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 1>);
-    case 2: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 2>);
-    default: return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 3>);
-  }
+const void *small_kernel_ptr(int) {
+  return reinterpret_cast<const void *>(prefill_small_kernel<TYPE, 1>);
 }
 
 template <int TYPE>
-cudaError_t small_dispatch(int M, const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem,
+cudaError_t small_dispatch(int, const WeightMaps &maps, const SmallArgs &a, unsigned grid, size_t smem,
                            cudaStream_t st) {
-  switch (M) {
-    case 1: return small_launch<TYPE, 1>(maps, a, grid, smem, st);
-    case 2: return small_launch<TYPE, 2>(maps, a, grid, smem, st);
-    default: return small_launch<TYPE, 3>(maps, a, grid, smem, st);
-  }
+  return small_launch<TYPE, 1>(maps, a, grid, smem, st);
 }
 
 int run_prefill_small(const char *name, int type, int G, const void *const *w, const int64_t *N, int64_t K,
@@ -1652,7 +1648,7 @@ size_t small_mma_smem(int type, int64_t K, int64_t M, int stages, SmallArgs *a) 
   const size_t act = align_up(static_cast<size_t>(K) * 16, 1024);
   const size_t box = static_cast<size_t>(kSmallRows) * (type == DSQ_Q8_0 ? 272 : 144);
   const size_t bars = align_up((2 * nw + 1) * sizeof(uint64_t), 128);
-  const size_t red = 2 * nw * M * 32 * sizeof(float);
+  const size_t red = static_cast<size_t>(small_mma_red_bufs(type)) * nw * M * 32 * sizeof(float);
   const size_t scr = type == DSQ_Q4_K ? nw * kSmallRows * kScrStride * 4 : 0;
   if (a) {
     a->box_bytes = static_cast<uint32_t>(box);

@@ -33,7 +33,7 @@ def run_prefill(dsq, qtype, wg, N, K, xg, M):
 
 CASES = [(8, 128, 256, 1), (8, 256, 512, 5), (12, 300, 512, 33), (8, 128, 4096, 128), (12, 384, 1024, 200),
          (8, 640, 2048, 70), (12, 128, 768, 257), (8, 200, 256, 513), (12, 4096, 4096, 3), (8, 1024, 512, 1100),
-         # M <= 2 (Q8_0) / 1 (Q4_K) takes the small-M kernel, up to 8 the
+         # M = 1 takes the CUDA-core small-M kernel, up to 8 the
          # mma.sync kernel (when its activations fit), then the narrowest
          # tensor-core tile
          (8, 4096, 4096, 8), (12, 1000, 2048, 3), (8, 33, 16384, 2), (12, 300, 512, 9), (8, 256, 512, 17),

@@ -73,11 +73,11 @@ def test_split_partials_are_padded_to_whole_float4s(dsq):
     assert got == _align(32 * K * 2, 1024) + _align(32 * 4, 1024) + 16 * 1164 * 4
 
 
-@pytest.mark.parametrize("qtype,max_m,k128", [(Q8, 2, 16384), (Q4, 1, 32768)])
+@pytest.mark.parametrize("qtype,max_m,k128", [(Q8, 1, 32768), (Q4, 1, 32768)])
 def test_a_few_tokens_take_the_small_kernel(dsq, qtype, max_m, k128):
-    # up to 2 (Q8_0) or 1 (Q4_K) tokens, with M x K x 4 bytes of activations
-    # <= 128 KB, run the CUDA-core kernel, which keeps its activations in
-    # shared memory: the workspace is a token 256 bytes
+    # one token, with M x K x 4 bytes of activations <= 128 KB, runs the
+    # CUDA-core kernel, which keeps its activations in shared memory: the
+    # workspace is a token 256 bytes
     for M in range(1, max_m + 1):
         assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 4096, M) == 256
     assert dsq.dsq_prefill_workspace_bytes(qtype, 4096, 4096, max_m + 1) > 256
@@ -86,7 +86,7 @@ def test_a_few_tokens_take_the_small_kernel(dsq, qtype, max_m, k128):
     assert dsq.dsq_prefill_grouped_workspace_bytes(qtype, [512, 64], 4096, max_m) == 256
 
 
-@pytest.mark.parametrize("qtype,max_m", [(Q8, 2), (Q4, 1)])
+@pytest.mark.parametrize("qtype,max_m", [(Q8, 1), (Q4, 1)])
 def test_up_to_8_tokens_take_the_mma_sync_bridge(dsq, qtype, max_m):
     # above the CUDA-core kernel and up to 8 tokens: the rounded activations
     # [8][K] binary16 plus a 256-byte block of row shifts
