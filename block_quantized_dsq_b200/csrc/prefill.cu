@@ -78,6 +78,16 @@ struct PrefillArgs {
   const int32_t *shift;   // [M] activation row shifts
   int units_per_split;    // 256-element units of K per split
   int splits;
+  // Last-wave split: when the pair tiles fill whole waves and a short last
+  // one, that last wave's tail_tiles tiles are split tail_splits ways in K
+  // (tail_ups units each) into pieces that follow the head_tiles unsplit
+  // tiles; piece j + s * tail_tiles (split s of tail tile j) writes its
+  // partial to tail_part + (j + s * tail_tiles) * tn * 256, token-major
+  // (token * 256 + row), and tail_reduce_kernel sums the splits in order.
+  // head_tiles = total_tiles when nothing is split this way.
+  int64_t head_tiles;
+  int tail_tiles, tail_splits, tail_ups;
+  float *tail_part;
   int tn;                 // tokens per pair tile (MMA N): 32..256, multiple of 32
   int slots;              // pipeline slots: one stage pair each, activations in shared memory
                           // (2 x 64 K x tn/2 tokens) and dequantized weights in TMEM (64 columns); even
@@ -353,26 +363,45 @@ struct Tile {
   int64_t mt, n0;
   int u0, u1, rot;
   int split, g;
+  int piece;   // index of a last-wave piece, -1 for a tile that is not one
 };
 // Every tile index, count and divisor here fits in 32 bits (the host refuses
 // a plan of 2^31 tiles or more), and 32-bit division costs a fraction of
 // 64-bit division, which sits at the start of every role's tile.
+template <bool TAIL>
 __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
   Tile tl;
   const uint32_t t32 = static_cast<uint32_t>(t);
-  const uint32_t tm = static_cast<uint32_t>(a.tiles_m), sp = static_cast<uint32_t>(a.splits);
-  const uint32_t rest = t32 / tm;
-  const uint32_t mt = t32 - rest * tm;
-  const uint32_t nt = rest / sp;
+  const uint32_t tm = static_cast<uint32_t>(a.tiles_m);
+  const uint32_t head = static_cast<uint32_t>(a.head_tiles);
+  uint32_t mt, nt, ups;
+  if (!TAIL || t32 < head) {
+    const uint32_t sp = static_cast<uint32_t>(a.splits);
+    const uint32_t rest = t32 / tm;
+    mt = t32 - rest * tm;
+    nt = rest / sp;
+    tl.split = static_cast<int>(rest - nt * sp);
+    ups = static_cast<uint32_t>(a.units_per_split);
+    tl.piece = -1;
+  } else {
+    // last-wave piece: split s of the (head + j)-th tile in the unsplit order
+    const uint32_t tt = t32 - head, nt_tail = static_cast<uint32_t>(a.tail_tiles);
+    const uint32_t sidx = tt / nt_tail;
+    const uint32_t ut = head + (tt - sidx * nt_tail);
+    nt = ut / tm;
+    mt = ut - nt * tm;
+    tl.split = static_cast<int>(sidx);
+    ups = static_cast<uint32_t>(a.tail_ups);
+    tl.piece = static_cast<int>(tt);
+  }
   tl.mt = mt;
-  tl.split = static_cast<int>(rest - nt * sp);
   int g = 0;
   while (g + 1 < a.G && nt >= static_cast<uint32_t>(a.tile_n0[g + 1])) ++g;
   tl.g = g;
   const uint32_t ntl = nt - static_cast<uint32_t>(a.tile_n0[g]);
   tl.n0 = static_cast<int64_t>(ntl) * kTileN;
-  tl.u0 = tl.split * a.units_per_split;
-  tl.u1 = min(tl.u0 + a.units_per_split, static_cast<int>(a.K / 256));
+  tl.u0 = tl.split * static_cast<int>(ups);
+  tl.u1 = min(tl.u0 + static_cast<int>(ups), static_cast<int>(a.K / 256));
   tl.rot = static_cast<int>((ntl + 7u * mt) % static_cast<uint32_t>(tl.u1 - tl.u0));
   return tl;
 }
@@ -384,7 +413,7 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs &a, int64_t t) {
 // its lane with two tcgen05.st, and one lane per warp arrives on the even
 // CTA's ready barrier of the slot.  The warps of J = 0 fill slots 0, 2, 4, ...
 // of the ring, those of J = 1 slots 1, 3, 5, ...
-template <int TYPE, int J>
+template <int TYPE, int J, bool TAIL>
 __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a, uint32_t tmem_slot0, int rr,
                                              uint32_t ready_even) {
   constexpr uint32_t RAW_BYTES = kRows * unit_bytes<TYPE>();
@@ -396,7 +425,7 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
   int rs = 0;            // raw unit slot and its phase parity
   uint32_t rpar = 0;
   for (int64_t t = blockIdx.x / 2; t < a.total_tiles; t += npairs) {
-    const Tile tl = tile_of(a, t);
+    const Tile tl = tile_of<TAIL>(a, t);
     for (int u = tl.u0; u < tl.u1; ++u) {
       const bool got = wait_or_abort(s, &s.rfull[rs], rpar, a.wait);
       if (__any_sync(0xffffffffu, !got)) return;
@@ -441,7 +470,9 @@ __device__ __forceinline__ void convert_role(const Smem &s, const PrefillArgs &a
 
 // Persistent CTA pair over pair tiles (pair index blockIdx.x / 2, stepping
 // by the number of pairs); rank r = this CTA's rank in the cluster.
-template <int TYPE>
+// TAIL: the plan splits its last wave in K (head_tiles < total_tiles); the
+// instantiation without it carries none of the piece handling.
+template <int TYPE, bool TAIL>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ WeightMaps maps, const __grid_constant__ PrefillArgs a) {
   constexpr int UB = unit_bytes<TYPE>();
@@ -479,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpW && lane == 0 && pair < a.total_tiles) {
     // weights are read-only: start this CTA's first units toward L2 while
     // the activation-rounding kernel before us finishes
-    const Tile tl = tile_of(a, pair);
+    const Tile tl = tile_of<TAIL>(a, pair);
     for (int k = 0; k < 2 && k < tl.u1 - tl.u0; ++k) {
       const int u = tl.u0 + (tl.rot + k) % (tl.u1 - tl.u0);
       prefetch_l2_tile_2d(&maps.m[tl.g], u * (UB / 4), static_cast<int32_t>(tl.n0 + kRows * rank));
@@ -515,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t rnd = 0;
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
-        const Tile tl = tile_of(a, t);
+        const Tile tl = tile_of<TAIL>(a, t);
         const int64_t xt = 2 * tl.mt + rank;   // this CTA's token tile
         int u = tl.u0 + tl.rot;
         for (int k = tl.u0; k < tl.u1 && ok; ++k, u = (u + 1 == tl.u1 ? tl.u0 : u + 1)) {
@@ -549,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t par = 0;
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
-        const Tile tl = tile_of(a, t);
+        const Tile tl = tile_of<TAIL>(a, t);
         for (int g = 0; g < 2 * (tl.u1 - tl.u0); ++g) {
           if (!wait_or_abort(s, &s.ready[sq], par, a.wait)) {
             ok = false;
@@ -573,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pq = 0;   // phase parity of the current round of the slot ring
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs, ++i) {
-        const Tile tl = tile_of(a, t);
+        const Tile tl = tile_of<TAIL>(a, t);
         if (i >= 1 && !wait_or_abort(s, s.accempty, static_cast<uint32_t>((i - 1) & 1), a.wait)) {
           ok = false;
           break;
@@ -617,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t rnd = 0;
       bool ok = true;
       for (int64_t t = pair; t < a.total_tiles && ok; t += npairs) {
-        const Tile tl = tile_of(a, t);
+        const Tile tl = tile_of<TAIL>(a, t);
         const int32_t row0 = static_cast<int32_t>(tl.n0 + kRows * rank);
         int u = tl.u0 + tl.rot;
         for (int k = tl.u0; k < tl.u1; ++k, ++gu, u = (u + 1 == tl.u1 ? tl.u0 : u + 1)) {
@@ -644,8 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;   // TMEM lane quadrant this warp may access
     const uint32_t slot0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + a_col0;
     const uint32_t ready_even = mapa_shared(smem_u32(s.ready), 0);
-    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0>(s, a, slot0, 32 * q + lane, ready_even);
-    else convert_role<TYPE, 1>(s, a, slot0, 32 * q + lane, ready_even);
+    if (warp < kWarpConv0 + 4) convert_role<TYPE, 0, TAIL>(s, a, slot0, 32 * q + lane, ready_even);
+    else convert_role<TYPE, 1, TAIL>(s, a, slot0, 32 * q + lane, ready_even);
   } else {
     // ------------------------------- epilogue: TMEM -> y * 2^-s_m
     const int q = warp & 3;
@@ -654,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nchunks = a.tn / 32;
     int64_t i = 0;
     for (int64_t t = pair; t < a.total_tiles; t += npairs, ++i) {
-      const Tile tl = tile_of(a, t);
+      const Tile tl = tile_of<TAIL>(a, t);
       const int64_t n = tl.n0 + r;
       const int64_t Ng = a.N[tl.g];
       const bool n_ok = n < Ng;
@@ -690,13 +721,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xffffffffu, my_scale[c], j)));
         const int64_t mc = m0 + 32 * c;
         float *yp = a.y[tl.g] + static_cast<int64_t>(tl.split) * a.split_stride[tl.g] + mc * Ng + n;
+        int64_t ys = Ng;
+        if (TAIL && tl.piece >= 0) {
+          // a last-wave piece writes its partial token-major into its own block
+          yp = a.tail_part + (static_cast<int64_t>(tl.piece) * a.tn + 32 * c) * kTileN + r;
+          ys = kTileN;
+        }
         if (n_ok && mc + 32 <= a.M) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) yp[static_cast<int64_t>(j) * Ng] = __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) yp[static_cast<int64_t>(j) * ys] = __uint_as_float(v[j]);
         } else if (n_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (mc + j < a.M) yp[static_cast<int64_t>(j) * Ng] = __uint_as_float(v[j]);
+            if (mc + j < a.M) yp[static_cast<int64_t>(j) * ys] = __uint_as_float(v[j]);
         }
       }
     }
@@ -802,6 +839,47 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
     float acc = part[i];
     for (int s = 1; s < splits; ++s) acc += part[static_cast<int64_t>(s) * sstride + i];
     y[i] = acc;
+  }
+}
+
+// Last-wave pieces -> outputs: for each split tile of the last wave (tile
+// head + j of the unsplit order), token m and weight row n, the pieces'
+// partials are summed in split order (deterministic) and written to y.  One
+// thread per 4 consecutive rows of one token of one tile.
+__global__ void __launch_bounds__(256) tail_reduce_kernel(const __grid_constant__ PrefillArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const uint32_t per_tile = static_cast<uint32_t>(a.tn) * (kTileN / 4);   // float4s per piece
+  const uint32_t total = static_cast<uint32_t>(a.tail_tiles) * per_tile;
+  const int64_t split_stride4 = static_cast<int64_t>(a.tail_tiles) * per_tile;
+  const float4 *p4 = reinterpret_cast<const float4 *>(a.tail_part);
+  const uint32_t tm = static_cast<uint32_t>(a.tiles_m);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const uint32_t j = i / per_tile, rem = i - j * per_tile;
+    const uint32_t ml = rem / (kTileN / 4), r4 = rem - ml * (kTileN / 4);
+    const uint32_t ut = static_cast<uint32_t>(a.head_tiles) + j;
+    const uint32_t nt = ut / tm, mt = ut - nt * tm;
+    const int64_t m = static_cast<int64_t>(mt) * a.tn + ml;
+    if (m >= a.M) continue;
+    int g = 0;
+    while (g + 1 < a.G && nt >= static_cast<uint32_t>(a.tile_n0[g + 1])) ++g;
+    const int64_t Ng = a.N[g];
+    const int64_t n = static_cast<int64_t>(nt - static_cast<uint32_t>(a.tile_n0[g])) * kTileN + 4 * r4;
+    if (n >= Ng) continue;
+    float4 acc = __ldg(p4 + i);
+    for (int sp = 1; sp < a.tail_splits; ++sp) {
+      const float4 v = __ldg(p4 + sp * split_stride4 + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    float *yr = a.y[g] + m * Ng + n;
+    if ((Ng & 3) == 0) {
+      *reinterpret_cast<float4 *>(yr) = acc;   // y is 16-byte aligned and n is a multiple of 4
+    } else {
+      yr[0] = acc.x;
+      if (n + 1 < Ng) yr[1] = acc.y;
+      if (n + 2 < Ng) yr[2] = acc.z;
+      if (n + 3 < Ng) yr[3] = acc.w;
+    }
   }
 }
 
@@ -1372,6 +1450,9 @@ __global__ void __launch_bounds__(small_mma_warps(TYPE) * 32, 1)
 struct Plan {
   int tn, slots, slots_raw, splits, units_per_split;
   int64_t tiles_m, tiles_n, total_tiles, m_pad;
+  int64_t head_tiles;                    // tiles before the last-wave pieces
+  int tail_tiles, tail_splits, tail_ups;   // last-wave split (tail_splits = 1: none)
+  size_t tail_off;                       // byte offset of the last-wave partials
   unsigned grid;   // CTAs (2 per pair)
   size_t smem, x16_bytes, shift_off, part_off, total;
   int64_t split_stride[kMaxGroup];   // floats per split of each weight's partials
@@ -1382,7 +1463,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
-template <int TYPE>
+template <int TYPE, bool TAIL>
 cudaError_t launch_pair(const WeightMaps &maps, const PrefillArgs &args, unsigned grid, size_t smem,
                         cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
@@ -1399,7 +1480,7 @@ cudaError_t launch_pair(const WeightMaps &maps, const PrefillArgs &args, unsigne
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<TYPE>, maps, args);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<TYPE, TAIL>, maps, args);
 }
 
 // How many CTA pairs of the GEMM kernel can be resident at once (clusters
@@ -1416,8 +1497,9 @@ int resident_pairs(int type, int tn, size_t smem, int sms) {
   const int ni = tn / 32 - 1;   // 0..7
   std::lock_guard<std::mutex> lk(mu);
   if (cache[dev][ti][ni] > 0) return cache[dev][ti][ni];
-  const void *kern = type == DSQ_Q8_0 ? reinterpret_cast<const void *>(prefill_kernel<DSQ_Q8_0>)
-                                      : reinterpret_cast<const void *>(prefill_kernel<DSQ_Q4_K>);
+  // both instantiations of a type take the same resources
+  const void *kern = type == DSQ_Q8_0 ? reinterpret_cast<const void *>(prefill_kernel<DSQ_Q8_0, false>)
+                                      : reinterpret_cast<const void *>(prefill_kernel<DSQ_Q4_K, false>);
   if (set_smem_once(kern, static_cast<int>(smem), "prefill") != DSQ_OK) return sms / 2;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(sms / 2 * 2));
@@ -1476,6 +1558,40 @@ Plan make_plan(int type, int G, const int64_t *N, int64_t K, int64_t M, int sms,
   p.units_per_split = (units + p.splits - 1) / p.splits;
   p.splits = (units + p.units_per_split - 1) / p.units_per_split;
   p.total_tiles = tiles * p.splits;
+  p.head_tiles = p.total_tiles;
+  p.tail_tiles = 0;
+  p.tail_splits = 1;
+  p.tail_ups = units;
+  // Last-wave split: tiles that fill whole waves of pairs and a last wave at
+  // most a quarter full leave most pairs idle for a whole tile.  Splitting
+  // the last wave's tiles s ways in K (s * tail <= pairs, so the pieces are
+  // one wave) cuts that wave to ceil(units / s) units, at the price of the
+  // pieces' partials and one more launch to sum them.  Estimates: a unit of
+  // K takes ~1.6 us at 256 tokens per tile (measured, scaled with the
+  // tokens, at least a quarter of it); the sum re-reads the partials at
+  // ~6 TB/s after ~2 us of launch.  A fuller last wave does not pay: with
+  // 34 of 74 pairs busy (Q8_0, 8192 rows, 2048 tokens) its tiles already
+  // finish early, and the split measured 13 % slower; with 12 of 74 (two
+  // Q4_K weights of 4096 + 1024 rows, 2048 tokens) it measured 11 % faster.
+  if (p.splits == 1 && tiles > pairs) {
+    const int64_t tail = tiles % pairs;
+    if (tail > 0 && 4 * tail <= pairs) {
+      int s = static_cast<int>(pairs / tail);
+      if (s > 16) s = 16;
+      if (s > units) s = units;
+      const int ups = (units + s - 1) / s;
+      s = (units + ups - 1) / ups;
+      const double unit_us = 1.6 * (p.tn >= 64 ? p.tn / 256.0 : 0.25);
+      const double part_bytes = static_cast<double>(tail) * s * p.tn * kTileN * 4;
+      if (s > 1 && (units - ups) * unit_us > 2.0 + part_bytes / 6.0e6) {
+        p.head_tiles = tiles - tail;
+        p.tail_tiles = static_cast<int>(tail);
+        p.tail_splits = s;
+        p.tail_ups = ups;
+        p.total_tiles = p.head_tiles + tail * s;
+      }
+    }
+  }
   p.grid = static_cast<unsigned>(2 * (p.total_tiles < pairs ? p.total_tiles : pairs));
   // the fp16 activation buffer is padded with zero rows to whole token tiles
   p.m_pad = p.tiles_m * p.tn;
@@ -1489,6 +1605,10 @@ Plan make_plan(int type, int G, const int64_t *N, int64_t K, int64_t M, int sms,
     p.part_g_off[g] = off;
     if (p.splits > 1) off += static_cast<size_t>(p.splits) * p.split_stride[g] * 4;
   }
+  // last-wave partials: one tn x 256 block per piece
+  p.tail_off = align_up(off, 1024);
+  if (p.tail_splits > 1)
+    off = p.tail_off + static_cast<size_t>(p.tail_tiles) * p.tail_splits * p.tn * kTileN * 4;
   p.total = off;
   return p;
 }
@@ -1517,12 +1637,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int TYPE>
+template <int TYPE, bool TAIL>
 int launch_gemm(const WeightMaps &maps, const PrefillArgs &args, const Plan &p, cudaStream_t stream) {
-  const void *kern = reinterpret_cast<const void *>(prefill_kernel<TYPE>);
+  const void *kern = reinterpret_cast<const void *>(prefill_kernel<TYPE, TAIL>);
   const int rc = set_smem_once(kern, static_cast<int>(p.smem), "prefill");
   if (rc != DSQ_OK) return rc;
-  const cudaError_t e = launch_pair<TYPE>(maps, args, p.grid, p.smem, stream);
+  const cudaError_t e = launch_pair<TYPE, TAIL>(maps, args, p.grid, p.smem, stream);
   if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "dsq_gemm_prefill: gemm: %s", cudaGetErrorString(e));
   return after_launch("dsq_gemm_prefill: gemm");
 }
@@ -1879,8 +1999,18 @@ int run_prefill(const char *name, int type, int64_t G, const void *const *w, con
   args.tiles_m = p.tiles_m;
   args.tiles_n = p.tiles_n;
   args.total_tiles = p.total_tiles;
+  args.head_tiles = p.head_tiles;
+  args.tail_tiles = p.tail_tiles;
+  args.tail_splits = p.tail_splits;
+  args.tail_ups = p.tail_ups;
+  args.tail_part = p.tail_splits > 1 ? reinterpret_cast<float *>(ws + p.tail_off) : nullptr;
   args.wait = ctl;
-  rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0>(maps, args, p, st) : launch_gemm<DSQ_Q4_K>(maps, args, p, st);
+  if (p.tail_splits > 1)
+    rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0, true>(maps, args, p, st)
+                          : launch_gemm<DSQ_Q4_K, true>(maps, args, p, st);
+  else
+    rc = type == DSQ_Q8_0 ? launch_gemm<DSQ_Q8_0, false>(maps, args, p, st)
+                          : launch_gemm<DSQ_Q4_K, false>(maps, args, p, st);
   if (rc != DSQ_OK) return rc;
   if (p.splits > 1) {
     for (int g = 0; g < Gi; ++g) {
@@ -1894,6 +2024,15 @@ int run_prefill(const char *name, int type, int64_t G, const void *const *w, con
       rc = after_launch(name);
       if (rc != DSQ_OK) return rc;
     }
+  }
+  if (p.tail_splits > 1) {
+    const int64_t total4 = static_cast<int64_t>(p.tail_tiles) * p.tn * (kTileN / 4);
+    const int64_t blocks = (total4 + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(blocks < 8 * sms ? blocks : 8 * sms);
+    e = launch_pdl(tail_reduce_kernel, dim3(grid), dim3(256), 0, st, args);
+    if (e != cudaSuccess) return fail(DSQ_ERR_LAUNCH, "%s: last-wave reduce: %s", name, cudaGetErrorString(e));
+    rc = after_launch(name);
+    if (rc != DSQ_OK) return rc;
   }
   return DSQ_OK;
 }

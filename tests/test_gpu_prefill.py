@@ -307,3 +307,74 @@ def test_prefill_two_way_split_is_deterministic(dsq, ref, qtype, N, K, M):
     assert np.array_equal(y1, y2)
     assert rel_l2(y1, ref.prefill_rounded(qtype, w, K, x, "f16")) <= PREFILL_ROUNDED_TOL
     assert rel_l2(y1, ref.prefill_f64(qtype, w, K, x)) <= PREFILL_TOL
+
+
+@pytest.mark.parametrize("qtype", [8, 12])
+@pytest.mark.parametrize("M", [4, 300])          # the mma.sync bridge and the CTA-pair kernel
+def test_prefill_sees_weights_written_just_before(dsq, ref, qtype, M):
+    """Weights quantized on the same stream immediately before the call, with
+    no synchronization between, are the ones multiplied: the kernels that
+    read weights wait for their predecessors before their first weight
+    load."""
+    N, K = 1024, 2048
+    w32 = synth.weights(400 + M, N, K)
+    x = synth.activations(401 + M, M, K)
+    w_ref = ref.quantize(qtype, w32)
+    w = torch.zeros(w_ref.shape, dtype=torch.uint8, device="cuda")
+    w32g, xg = to_dev(w32), to_dev(x)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    nb = dsq.dsq_prefill_workspace_bytes(qtype, N, K, M)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    dsq.dsq_quantize_weights(qtype, w32g, N, K, w)
+    dsq.dsq_gemm_prefill(qtype, w, N, K, xg, M, y, ws, nb)
+    torch.cuda.synchronize()
+    assert np.array_equal(w.cpu().numpy(), w_ref)
+    assert rel_l2(y.cpu().numpy(), ref.prefill_rounded(qtype, w_ref, K, x, "f16")) <= PREFILL_ROUNDED_TOL
+
+
+@pytest.mark.parametrize("qtype,N,K,M", [(12, 10000, 4096, 300), (8, 10000, 2048, 300)])
+def test_prefill_last_wave_split(dsq, ref, qtype, N, K, M):
+    """40 weight tiles x 2 token tiles = 80 pair tiles on 74 SM pairs: the
+    last wave's 6 tiles (weight rows 9472 .. 9999, the last tile ragged, and
+    both token tiles, the second ragged at 300 tokens) are split in K into
+    one wave of pieces whose partials a second kernel sums in split order.
+    Every row of those tiles and a sample of the others against the oracle;
+    two calls give the same bits."""
+    m_pad = -(-M // 256) * 256
+    unsplit = m_pad * K * 2 + -(-m_pad * 4 // 1024) * 1024
+    assert dsq.dsq_prefill_workspace_bytes(qtype, N, K, M) > unsplit   # the plan holds last-wave partials
+    w = ref.quantize(qtype, synth.weights(380 + N, N, K))
+    x = synth.activations(381 + M, M, K)
+    x[1] *= 1e3
+    y1 = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    y2 = run_prefill(dsq, qtype, to_dev(w), N, K, to_dev(x), M)
+    assert np.isfinite(y1).all()
+    assert np.array_equal(y1, y2)
+    rng = np.random.default_rng(382)
+    ns = np.concatenate([np.sort(rng.choice(9472, size=128, replace=False)), np.arange(9472, N)])
+    ys = y1[:, ns]
+    assert rel_l2(ys[:, 128:], ref.prefill_rounded(qtype, w[ns[128:]], K, x, "f16")) <= PREFILL_ROUNDED_TOL
+    assert rel_l2(ys, ref.prefill_rounded(qtype, w[ns], K, x, "f16")) <= PREFILL_ROUNDED_TOL
+    assert rel_l2(ys, ref.prefill_f64(qtype, w[ns], K, x)) <= PREFILL_TOL
+
+
+def test_prefill_grouped_last_wave_split(dsq, ref):
+    """Q4_K weights of 4096 and 1024 rows sharing 2048 tokens: 160 pair tiles
+    = 2 waves of 74 and a last wave of 12 tiles (the second weight's rows
+    512 .. 1023 for tokens from 1024 on, and rows 768 .. 1023 for all), split
+    in K.  Those rows and a sample of the rest against the oracle."""
+    qtype, K, M, Ns = 12, 4096, 2048, [4096, 1024]
+    ws = [ref.quantize(qtype, synth.weights(390 + g, n, K)) for g, n in enumerate(Ns)]
+    x = synth.activations(397, M, K)
+    ys = _grouped(dsq, qtype, [to_dev(w) for w in ws], Ns, K, to_dev(x), M)
+    rng = np.random.default_rng(392)
+    ms = np.sort(np.concatenate([rng.choice(1024, size=16, replace=False),
+                                 1024 + rng.choice(1024, size=32, replace=False)]))
+    for g, (w, y) in enumerate(zip(ws, ys)):
+        yc = y.cpu().numpy()
+        assert np.isfinite(yc).all()
+        ns = np.arange(512, 1024) if g == 1 else np.sort(rng.choice(Ns[g], size=128, replace=False))
+        ys_c = yc[np.ix_(ms, ns)]
+        assert rel_l2(ys_c, ref.prefill_rounded(qtype, w[ns], K, x[ms], "f16")) <= PREFILL_ROUNDED_TOL
+        assert rel_l2(ys_c, ref.prefill_f64(qtype, w[ns], K, x[ms])) <= PREFILL_TOL

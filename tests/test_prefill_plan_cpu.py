@@ -3,7 +3,9 @@ GPU: the planner then assumes 148 SMs, i.e. 74 CTA pairs).
 
 The workspace holds the fp16 activations padded to whole token tiles, the
 per-row shifts, and the fp32 partials when K is split; K is split only while
-the pair tiles leave more than half the pairs idle.
+the pair tiles leave more than half the pairs idle, or, for the tiles of a
+last wave that is at most a quarter full, when the time saved outweighs the
+partials' extra pass.
 """
 import pytest
 
@@ -35,11 +37,42 @@ def test_refusals_return_zero(dsq):
     assert f(Q8, 256, 256, 0) == 0         # M < 1
 
 
-def test_large_problem_has_no_split(dsq):
-    # 8 token tiles (256 tokens each) x 32 weight tiles = 256 pair tiles:
-    # no split, workspace = fp16 activations + shifts
+def test_large_problem_with_a_fuller_last_wave_has_no_split(dsq):
+    # 8 token tiles (256 tokens each) x 32 weight tiles = 256 pair tiles on
+    # 74 pairs: 3 full waves and a last wave of 34 tiles, more than a quarter
+    # of the pairs: no split, workspace = fp16 activations + shifts
     M, N, K = 2048, 8192, 4096
     assert dsq.dsq_prefill_workspace_bytes(Q8, N, K, M) == M * K * 2 + _align(M * 4, 1024)
+
+
+def test_last_wave_more_than_a_quarter_full_is_not_split(dsq):
+    # 128 tiles = 74 + 54
+    M, N, K = 2048, 4096, 4096
+    assert dsq.dsq_prefill_workspace_bytes(Q4, N, K, M) == M * K * 2 + _align(M * 4, 1024)
+
+
+def test_last_wave_of_a_short_k_is_not_split(dsq):
+    # 80 tiles = 74 + 6 as below, but K = 512 is two units: halving the last
+    # wave saves less than the partials' extra pass costs
+    M, N, K = 300, 10000, 512
+    assert dsq.dsq_prefill_workspace_bytes(Q8, N, K, M) == 512 * K * 2 + _align(512 * 4, 1024)
+
+
+def test_last_wave_split_ways_follow_the_idle_pairs(dsq):
+    # 40 weight tiles (ragged: 10000 rows) x 2 token tiles (300 tokens) = 80
+    # tiles = 74 + 6: the 6 are split 12 ways -> 2 units each -> 8 pieces
+    # per tile (K = 4096: 16 units)
+    M, N, K = 300, 10000, 4096
+    base = 512 * K * 2 + _align(512 * 4, 1024)
+    assert dsq.dsq_prefill_workspace_bytes(Q4, N, K, M) == base + 6 * 8 * 256 * 256 * 4
+
+
+def test_grouped_last_wave_split(dsq):
+    # 4096 + 1024 rows at 2048 tokens: 20 x 8 = 160 tiles = 2 x 74 + 12; the
+    # 12 are split 6 ways (3 units each)
+    M, K = 2048, 4096
+    base = M * K * 2 + _align(M * 4, 1024)
+    assert dsq.dsq_prefill_grouped_workspace_bytes(Q4, [4096, 1024], K, M) == base + 12 * 6 * 256 * 256 * 4
 
 
 def test_small_problem_splits_k_and_holds_partials(dsq):
@@ -59,10 +92,12 @@ def test_padding_to_whole_token_tiles(dsq):
 
 @pytest.mark.parametrize("qtype", [Q8, Q4])
 def test_workspace_grows_with_tokens_once_unsplit(dsq, qtype):
+    # 64, 128, 512 and 1024 tiles: none is split (the last waves of 128, 512
+    # and 1024 tiles are 54, 68 and 62 tiles, more than half of 74 pairs)
     N, K = 8192, 4096
-    sizes = [dsq.dsq_prefill_workspace_bytes(qtype, N, K, M) for M in (512, 1024, 2048, 4096)]
-    assert all(a < b for a, b in zip(sizes, sizes[1:]))
-    assert all(s >= M * K * 2 for s, M in zip(sizes, (512, 1024, 2048, 4096)))
+    Ms = (512, 1024, 4096, 8192)
+    sizes = [dsq.dsq_prefill_workspace_bytes(qtype, N, K, M) for M in Ms]
+    assert sizes == [M * K * 2 + _align(M * 4, 1024) for M in Ms]
 
 
 def test_split_partials_are_padded_to_whole_float4s(dsq):
