@@ -816,6 +816,37 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const float *__restrict__
   }
 }
 
+// The n <= kMaxKSplits partials p[0], p[stride], ... summed in index order.
+// Loads go out four at a time before their adds, so up to four latencies
+// overlap instead of adding up, in few enough registers to keep the kernel
+// at full occupancy.
+constexpr int kMaxKSplits = 16;
+__device__ __forceinline__ void add4(float4 &acc, const float4 &v) {
+  acc.x += v.x;
+  acc.y += v.y;
+  acc.z += v.z;
+  acc.w += v.w;
+}
+__device__ __forceinline__ float4 sum_splits(const float4 *p, int64_t stride, int n) {
+  float4 v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (j < n) v[j] = __ldg(p + j * stride);
+  float4 acc = v[0];
+#pragma unroll
+  for (int j = 1; j < 4; ++j)
+    if (j < n) add4(acc, v[j]);
+  for (int s0 = 4; s0 < n; s0 += 4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (s0 + j < n) v[j] = __ldg(p + (s0 + j) * stride);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (s0 + j < n) add4(acc, v[j]);
+  }
+  return acc;
+}
+
 // Split-K partials -> output, summed in split order (deterministic).  Split
 // s's partial of the M x N outputs starts at part + s * sstride, sstride =
 // total rounded up to a multiple of 4, so every split is float4-aligned.
@@ -827,14 +858,8 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
   const float4 *p4 = reinterpret_cast<const float4 *>(part);
   float4 *y4 = reinterpret_cast<float4 *>(y);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    float4 acc = __ldg(p4 + i);
-    for (int s = 1; s < splits; ++s) {
-      const float4 v = __ldg(p4 + static_cast<int64_t>(s) * s4 + i);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    y4[i] = acc;
-  }
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride)
+    y4[i] = sum_splits(p4 + i, s4, splits);
   for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
     float acc = part[i];
     for (int s = 1; s < splits; ++s) acc += part[static_cast<int64_t>(s) * sstride + i];
@@ -866,11 +891,7 @@ __global__ void __launch_bounds__(256) tail_reduce_kernel(const __grid_constant_
     const int64_t Ng = a.N[g];
     const int64_t n = static_cast<int64_t>(nt - static_cast<uint32_t>(a.tile_n0[g])) * kTileN + 4 * r4;
     if (n >= Ng) continue;
-    float4 acc = __ldg(p4 + i);
-    for (int sp = 1; sp < a.tail_splits; ++sp) {
-      const float4 v = __ldg(p4 + sp * split_stride4 + i);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
+    const float4 acc = sum_splits(p4 + i, split_stride4, a.tail_splits);
     float *yr = a.y[g] + m * Ng + n;
     if ((Ng & 3) == 0) {
       *reinterpret_cast<float4 *>(yr) = acc;   // y is 16-byte aligned and n is a multiple of 4
@@ -1554,7 +1575,7 @@ Plan make_plan(int type, int G, const int64_t *N, int64_t K, int64_t M, int sms,
   const int64_t tiles = p.tiles_m * p.tiles_n;
   // split K only when the tiles leave more than half the pairs idle
   p.splits = 1;
-  while (tiles * p.splits * 2 <= pairs && p.splits * 2 <= 16 && p.splits * 2 <= units) p.splits *= 2;
+  while (tiles * p.splits * 2 <= pairs && p.splits * 2 <= kMaxKSplits && p.splits * 2 <= units) p.splits *= 2;
   p.units_per_split = (units + p.splits - 1) / p.splits;
   p.splits = (units + p.units_per_split - 1) / p.units_per_split;
   p.total_tiles = tiles * p.splits;
@@ -1577,7 +1598,7 @@ Plan make_plan(int type, int G, const int64_t *N, int64_t K, int64_t M, int sms,
     const int64_t tail = tiles % pairs;
     if (tail > 0 && 4 * tail <= pairs) {
       int s = static_cast<int>(pairs / tail);
-      if (s > 16) s = 16;
+      if (s > kMaxKSplits) s = kMaxKSplits;
       if (s > units) s = units;
       const int ups = (units + s - 1) / s;
       s = (units + ups - 1) / ups;
