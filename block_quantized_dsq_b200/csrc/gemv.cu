@@ -51,6 +51,14 @@
 #ifndef DSQ_GEMV_CTAS_PER_SM
 #define DSQ_GEMV_CTAS_PER_SM 1
 #endif
+// Long Q4_K matrices: twice the warps (at most 128 registers each), once
+// every CTA has at least this many rows.
+#ifndef DSQ_GEMV_WIDE_WARPS
+#define DSQ_GEMV_WIDE_WARPS 16
+#endif
+#ifndef DSQ_GEMV_WIDE_MIN_ROWS
+#define DSQ_GEMV_WIDE_MIN_ROWS 200
+#endif
 
 namespace dsq {
 namespace {
@@ -328,8 +336,8 @@ __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_
   }
 }
 
-template <int TYPE, int G, bool ISUM, int ACT>
-__global__ void __launch_bounds__(32 * DSQ_GEMV_MAX_WARPS, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
+template <int TYPE, int G, bool ISUM, int ACT, int MAXW>
+__global__ void __launch_bounds__(32 * MAXW, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
   constexpr int RPC = 32 / G;  // rows per slot
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -547,7 +555,7 @@ constexpr size_t kSmemBudget = DSQ_GEMV_SMEM_KB * 1024;
 // scales and int32 sums per 32-block.
 size_t act_smem_bytes(int64_t rows, int64_t K) { return static_cast<size_t>(rows) * (K + 8 * (K / 32)); }
 
-template <int TYPE, int G, bool ISUM, int ACT>
+template <int TYPE, int G, bool ISUM, int ACT, int MAXW>
 int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   constexpr int RPC = 32 / G;
   size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
@@ -557,7 +565,7 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
     a.act_off = static_cast<int>(smem);
     smem += act_smem_bytes(a.act_rows, a.K);
   }
-  auto kern = gemv_kernel<TYPE, G, ISUM, ACT>;
+  auto kern = gemv_kernel<TYPE, G, ISUM, ACT, MAXW>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
   if (rc != DSQ_OK) return rc;
   const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
@@ -568,15 +576,15 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   return after_launch("gemv");
 }
 
-template <int TYPE, bool ISUM, int ACT>
+template <int TYPE, bool ISUM, int ACT, int MAXW = DSQ_GEMV_MAX_WARPS>
 int dispatch_g(GemvArgs &a, int G, int num_sms, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_fast<TYPE, 1, ISUM, ACT>(a, num_sms, stream);
-    case 2: return launch_fast<TYPE, 2, ISUM, ACT>(a, num_sms, stream);
-    case 4: return launch_fast<TYPE, 4, ISUM, ACT>(a, num_sms, stream);
-    case 8: return launch_fast<TYPE, 8, ISUM, ACT>(a, num_sms, stream);
-    case 16: return launch_fast<TYPE, 16, ISUM, ACT>(a, num_sms, stream);
-    default: return launch_fast<TYPE, 32, ISUM, ACT>(a, num_sms, stream);
+    case 1: return launch_fast<TYPE, 1, ISUM, ACT, MAXW>(a, num_sms, stream);
+    case 2: return launch_fast<TYPE, 2, ISUM, ACT, MAXW>(a, num_sms, stream);
+    case 4: return launch_fast<TYPE, 4, ISUM, ACT, MAXW>(a, num_sms, stream);
+    case 8: return launch_fast<TYPE, 8, ISUM, ACT, MAXW>(a, num_sms, stream);
+    case 16: return launch_fast<TYPE, 16, ISUM, ACT, MAXW>(a, num_sms, stream);
+    default: return launch_fast<TYPE, 32, ISUM, ACT, MAXW>(a, num_sms, stream);
   }
 }
 
@@ -665,6 +673,19 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
               "%s: K=%lld rows do not fit the shared-memory pipeline", name, (long long)K);
   a.stages = static_cast<int>(budget / (static_cast<size_t>(a.warps) * a.slot_bytes));
   if (a.stages > DSQ_GEMV_MAX_STAGES) a.stages = DSQ_GEMV_MAX_STAGES;
+  // A long Q4_K matrix is bound by how much unpacking is in flight, not by
+  // its loads (a deeper ring measured slower): twice the warps, each with the
+  // same 2-slot ring.  Shorter matrices keep 8 warps, which start faster.
+  // Interleaved A/B on B200, K = 4096, rows per CTA in brackets: 16,384 rows
+  // (110) 10.5 -> 12.0 us; 32,768 (221) 16.7 -> 16.4; 49,152 (332) 23.3 ->
+  // 21.8; 65,536 (443) 30.1 -> 26.6.
+  if (type == DSQ_Q4_K && act == kActGlobal && !isum && a.warps == kMaxWarps &&
+      total >= static_cast<int64_t>(num_sms) * DSQ_GEMV_CTAS_PER_SM * DSQ_GEMV_WIDE_MIN_ROWS &&
+      static_cast<size_t>(DSQ_GEMV_WIDE_WARPS) * 2 * a.slot_bytes <= budget) {
+    a.warps = DSQ_GEMV_WIDE_WARPS;
+    a.stages = 2;
+    return dispatch_g<DSQ_Q4_K, false, kActGlobal, DSQ_GEMV_WIDE_WARPS>(a, G, num_sms, stream);
+  }
   if (type == DSQ_Q8_0)
     return isum ? dispatch_act<DSQ_Q8_0, true>(a, G, act, num_sms, stream)
                 : dispatch_act<DSQ_Q8_0, false>(a, G, act, num_sms, stream);

@@ -166,3 +166,20 @@ def test_results_are_deterministic(dsq, ref):
         ys.append(y)
     torch.cuda.synchronize()
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+
+
+def test_gemv_q4_k_long_matrix_takes_the_wide_launch(dsq, ref):
+    """38,888 Q4_K rows of K = 4096 (more than 200 rows for each of 148 SMs,
+    ragged): the 16-warp launch.  Each row is still reduced by one warp in the
+    same order, so its first 4096 rows equal a 4096-row call (the 8-warp
+    launch) bit for bit; all rows against the oracle."""
+    N, K = 148 * 256 + 1000, 4096
+    w, xq, xd, xs = _prep(ref, 12, N, K, 64, 65)
+    wg, xqg, xdg, xsg = to_dev(w), to_dev(xq), to_dev(xd), to_dev(xs)
+    y = torch.empty(N, dtype=torch.float32, device="cuda")
+    dsq.dsq_gemv_q4_k(wg, N, K, xqg, xdg, xsg, y)
+    y_head = torch.empty(4096, dtype=torch.float32, device="cuda")
+    dsq.dsq_gemv_q4_k(wg, 4096, K, xqg, xdg, xsg, y_head)
+    torch.cuda.synchronize()
+    assert torch.equal(y[:4096], y_head)
+    _check(ref, 12, w, K, xq, xd, xs, y.cpu().numpy())
