@@ -276,6 +276,13 @@ __device__ __forceinline__ float unit_q8_0(const uint8_t *p, const ActSlice &act
 
 // One Q4_K super-block (144 bytes = 36 words): word 0 = d | dmin << 16,
 // words 1..3 = the 12 scale bytes, words 4..35 = the 128 nibble bytes.
+// Four unsigned bytes of a times four signed bytes of b, added to c.
+__device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c) {
+  int32_t d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 template <bool ISUM>
 __device__ __forceinline__ float unit_q4_k(const uint8_t *p, const ActSlice &act, int32_t *isum_out) {
   uint32_t w[36];
@@ -299,13 +306,16 @@ __device__ __forceinline__ float unit_q4_k(const uint8_t *p, const ActSlice &act
     const int sh = 8 * (j & 3);
     const float sc = static_cast<float>((scw >> sh) & 0xffu);
     const float m = static_cast<float>((mw >> sh) & 0xffu);
+    // The high nibbles stay in place (16 x the code, an unsigned byte) and
+    // the sum is divided by 16 once: Σ 16·q·x is an exact multiple of 16.
     int32_t s = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t byte4 = w[4 + 8 * (j >> 1) + i];
-      const uint32_t nib = (j & 1) ? ((byte4 >> 4) & 0x0f0f0f0fu) : (byte4 & 0x0f0f0f0fu);
-      s = __dp4a(static_cast<int>(nib), static_cast<int>(act.q[8 * j + i]), s);
+      const uint32_t nib = byte4 & ((j & 1) ? 0xf0f0f0f0u : 0x0f0f0f0fu);
+      s = dp4a_us(nib, act.q[8 * j + i], s);
     }
+    if (j & 1) s >>= 4;
     if (ISUM) isum_out[j] = s;
     const float t = __fmul_rn(__fmul_rn(d, sc), static_cast<float>(s));
     const float u = __fmul_rn(__fmul_rn(dmin, m), static_cast<float>(act.s[j]));
