@@ -190,6 +190,11 @@ int dsq_gemv_tokens(int type, const void *w0, int64_t N0, const void *w1, int64_
  *   - the fp32 sum over K is scaled back by 2^-s_m.
  * Error vs the fp64 dequantized reference: relative L2 ~3e-4 on N(0,1)
  * activations and N(0, 0.02^2) weights (gate 2e-3).
+ * Determinism: the sum over K may be cut into pieces computed by different
+ * SMs (all tiles of a small problem, or only the tiles of a short last wave
+ * of a large one); the plan depends only on the shape and the device's SM
+ * count, and the pieces are added in a fixed order, so repeated calls give
+ * the same bits.
  * Weight range: dequantized weights must lie inside the binary16 range.  A
  * block whose scales admit a value of magnitude >= 65520 -- a Q8_0 block
  * with |d|*127 >= 65520, or a Q4_K sub-block whose code-0 or code-15 value
