@@ -51,13 +51,13 @@
 #ifndef DSQ_GEMV_CTAS_PER_SM
 #define DSQ_GEMV_CTAS_PER_SM 1
 #endif
-// Long Q4_K matrices: twice the warps (at most 128 registers each), once
-// every CTA has at least this many rows.
-#ifndef DSQ_GEMV_WIDE_WARPS
-#define DSQ_GEMV_WIDE_WARPS 16
+// Long Q4_K matrices: more warps, once every CTA has at least this many
+// rows (12 warps of at most 168 registers, 16 of at most 128).
+#ifndef DSQ_GEMV_MID_MIN_ROWS
+#define DSQ_GEMV_MID_MIN_ROWS 140
 #endif
 #ifndef DSQ_GEMV_WIDE_MIN_ROWS
-#define DSQ_GEMV_WIDE_MIN_ROWS 200
+#define DSQ_GEMV_WIDE_MIN_ROWS 300
 #endif
 
 namespace dsq {
@@ -684,17 +684,24 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   a.stages = static_cast<int>(budget / (static_cast<size_t>(a.warps) * a.slot_bytes));
   if (a.stages > DSQ_GEMV_MAX_STAGES) a.stages = DSQ_GEMV_MAX_STAGES;
   // A long Q4_K matrix is bound by how much unpacking is in flight, not by
-  // its loads (a deeper ring measured slower): twice the warps, each with the
+  // its loads (a deeper ring measured slower): more warps, each with the
   // same 2-slot ring.  Shorter matrices keep 8 warps, which start faster.
-  // Interleaved A/B on B200, K = 4096, rows per CTA in brackets: 16,384 rows
-  // (110) 10.5 -> 12.0 us; 32,768 (221) 16.7 -> 16.4; 49,152 (332) 23.3 ->
-  // 21.8; 65,536 (443) 30.1 -> 26.6.
-  if (type == DSQ_Q4_K && act == kActGlobal && !isum && a.warps == kMaxWarps &&
-      total >= static_cast<int64_t>(num_sms) * DSQ_GEMV_CTAS_PER_SM * DSQ_GEMV_WIDE_MIN_ROWS &&
-      static_cast<size_t>(DSQ_GEMV_WIDE_WARPS) * 2 * a.slot_bytes <= budget) {
-    a.warps = DSQ_GEMV_WIDE_WARPS;
-    a.stages = 2;
-    return dispatch_g<DSQ_Q4_K, false, kActGlobal, DSQ_GEMV_WIDE_WARPS>(a, G, num_sms, stream);
+  // Interleaved A/B on B200, K = 4096, rows per CTA in brackets, 8 / 12 / 16
+  // warps: 16,384 rows (110) 10.1 / 10.6 / 11.8 us; 24,576 (166) 13.3 /
+  // 12.8 / 14.0; 32,768 (221) 16.7 / 15.5 / 16.1; 65,536 (443) 29.7 / 26.7 /
+  // 26.2-26.6.
+  if (type == DSQ_Q4_K && act == kActGlobal && !isum && a.warps == kMaxWarps) {
+    const int64_t per_cta = total / (static_cast<int64_t>(num_sms) * DSQ_GEMV_CTAS_PER_SM);
+    if (per_cta >= DSQ_GEMV_WIDE_MIN_ROWS && size_t(16) * 2 * a.slot_bytes <= budget) {
+      a.warps = 16;
+      a.stages = 2;
+      return dispatch_g<DSQ_Q4_K, false, kActGlobal, 16>(a, G, num_sms, stream);
+    }
+    if (per_cta >= DSQ_GEMV_MID_MIN_ROWS && size_t(12) * 2 * a.slot_bytes <= budget) {
+      a.warps = 12;
+      a.stages = 2;
+      return dispatch_g<DSQ_Q4_K, false, kActGlobal, 12>(a, G, num_sms, stream);
+    }
   }
   if (type == DSQ_Q8_0)
     return isum ? dispatch_act<DSQ_Q8_0, true>(a, G, act, num_sms, stream)

@@ -168,12 +168,13 @@ def test_results_are_deterministic(dsq, ref):
     assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
 
 
-def test_gemv_q4_k_long_matrix_takes_the_wide_launch(dsq, ref):
-    """38,888 Q4_K rows of K = 4096 (more than 200 rows for each of 148 SMs,
-    ragged): the 16-warp launch.  Each row is still reduced by one warp in the
-    same order, so its first 4096 rows equal a 4096-row call (the 8-warp
-    launch) bit for bit; all rows against the oracle."""
-    N, K = 148 * 256 + 1000, 4096
+@pytest.mark.parametrize("N", [148 * 200 + 7, 148 * 306 + 7])   # 200 and 306 rows per SM: 12 and 16 warps
+def test_gemv_q4_k_long_matrix_takes_the_wide_launch(dsq, ref, N):
+    """Q4_K matrices of K = 4096 long enough for the 12- and 16-warp launches
+    (ragged row counts).  Each row is still reduced by one warp in the same
+    order, so the first 4096 rows equal a 4096-row call (the 8-warp launch)
+    bit for bit; all rows against the oracle."""
+    K = 4096
     w, xq, xd, xs = _prep(ref, 12, N, K, 64, 65)
     wg, xqg, xdg, xsg = to_dev(w), to_dev(xq), to_dev(xd), to_dev(xs)
     y = torch.empty(N, dtype=torch.float32, device="cuda")
