@@ -346,9 +346,14 @@ __device__ __forceinline__ void issue_rows(const GemvArgs &a, int64_t ra, int64_
   }
 }
 
-template <int TYPE, int G, bool ISUM, int ACT, int MAXW>
-__global__ void __launch_bounds__(32 * MAXW, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(const __grid_constant__ GemvArgs a) {
+// MINB = 2: the overlapped launch.  The CTA fits half an SM (registers and
+// shared memory), so the next call's CTA can be resident beside it; it issues
+// its first weight slots before its launch-dependency wait and releases its
+// own dependents only after that wait.
+template <int TYPE, int G, bool ISUM, int ACT, int MAXW, int MINB>
+__global__ void __launch_bounds__(32 * MAXW, MINB) gemv_kernel(const __grid_constant__ GemvArgs a) {
   constexpr int RPC = 32 / G;  // rows per slot
+  constexpr bool EARLY = MINB > 1;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = a.warps, S = a.stages;
@@ -404,17 +409,28 @@ __global__ void __launch_bounds__(32 * MAXW, DSQ_GEMV_CTAS_PER_SM) gemv_kernel(c
       first_key = group * a.nunits + j;
     }
   }
-  pdl_trigger();
-  pdl_wait();
-  if (ACT == kActGlobal && mine == 0) return;
-
-  if (lane == 0 && mine > 0) {
-    for (int64_t k = 0; k < mine && k < S; ++k) {
-      const int64_t c = warp + k * W;
-      const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
-      issue_rows(a, ra, rb, ring + k * a.slot_bytes, &bars[k], policy);
+  auto issue_first = [&]() {
+    if (lane == 0 && mine > 0) {
+      for (int64_t k = 0; k < mine && k < S; ++k) {
+        const int64_t c = warp + k * W;
+        const int64_t ra = r0 + c * RPC, rb = min(ra + RPC, r1);
+        issue_rows(a, ra, rb, ring + k * a.slot_bytes, &bars[k], policy);
+      }
     }
+  };
+  if constexpr (EARLY) {
+    // The weights are read-only for the call, and every kernel of this
+    // library that can precede this one releases it only after its own wait
+    // or writes no weights, so the first slots load before the wait.
+    issue_first();
+    pdl_wait();
+    pdl_trigger();
+  } else {
+    pdl_trigger();
+    pdl_wait();
+    issue_first();
   }
+  if (ACT == kActGlobal && mine == 0) return;
   // activation source: global (two-call path) or quantized here, into shared
   // memory, while the first weight copies are in flight
   const int8_t *xq = a.xq;
@@ -560,12 +576,14 @@ __global__ void __launch_bounds__(256) gemv_q8_0_rowwise_kernel(const __grid_con
 
 constexpr int kMaxWarps = DSQ_GEMV_MAX_WARPS;
 constexpr size_t kSmemBudget = DSQ_GEMV_SMEM_KB * 1024;
+// shared memory of an overlapped-launch CTA: two of them fit one SM
+constexpr size_t kOverlapSmem = 110 * 1024;
 
 // Shared memory of the activation area in fused mode: int8 codes plus fp32
 // scales and int32 sums per 32-block.
 size_t act_smem_bytes(int64_t rows, int64_t K) { return static_cast<size_t>(rows) * (K + 8 * (K / 32)); }
 
-template <int TYPE, int G, bool ISUM, int ACT, int MAXW>
+template <int TYPE, int G, bool ISUM, int ACT, int MAXW, int MINB>
 int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   constexpr int RPC = 32 / G;
   size_t smem = static_cast<size_t>(a.warps) * a.stages * a.slot_bytes +
@@ -575,7 +593,7 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
     a.act_off = static_cast<int>(smem);
     smem += act_smem_bytes(a.act_rows, a.K);
   }
-  auto kern = gemv_kernel<TYPE, G, ISUM, ACT, MAXW>;
+  auto kern = gemv_kernel<TYPE, G, ISUM, ACT, MAXW, MINB>;
   const int rc = set_smem_once(reinterpret_cast<const void *>(kern), static_cast<int>(smem), "gemv");
   if (rc != DSQ_OK) return rc;
   const int64_t chunks = (a.total_rows + RPC - 1) / RPC;
@@ -586,15 +604,15 @@ int launch_fast(GemvArgs &a, int num_sms, cudaStream_t stream) {
   return after_launch("gemv");
 }
 
-template <int TYPE, bool ISUM, int ACT, int MAXW = DSQ_GEMV_MAX_WARPS>
+template <int TYPE, bool ISUM, int ACT, int MAXW = DSQ_GEMV_MAX_WARPS, int MINB = DSQ_GEMV_CTAS_PER_SM>
 int dispatch_g(GemvArgs &a, int G, int num_sms, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_fast<TYPE, 1, ISUM, ACT, MAXW>(a, num_sms, stream);
-    case 2: return launch_fast<TYPE, 2, ISUM, ACT, MAXW>(a, num_sms, stream);
-    case 4: return launch_fast<TYPE, 4, ISUM, ACT, MAXW>(a, num_sms, stream);
-    case 8: return launch_fast<TYPE, 8, ISUM, ACT, MAXW>(a, num_sms, stream);
-    case 16: return launch_fast<TYPE, 16, ISUM, ACT, MAXW>(a, num_sms, stream);
-    default: return launch_fast<TYPE, 32, ISUM, ACT, MAXW>(a, num_sms, stream);
+    case 1: return launch_fast<TYPE, 1, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
+    case 2: return launch_fast<TYPE, 2, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
+    case 4: return launch_fast<TYPE, 4, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
+    case 8: return launch_fast<TYPE, 8, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
+    case 16: return launch_fast<TYPE, 16, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
+    default: return launch_fast<TYPE, 32, ISUM, ACT, MAXW, MINB>(a, num_sms, stream);
   }
 }
 
@@ -702,6 +720,14 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
       a.stages = 2;
       return dispatch_g<DSQ_Q4_K, false, kActGlobal, 12>(a, G, num_sms, stream);
     }
+    // Shorter Q4_K matrices: the overlapped launch, when 8 warps with 2 slots
+    // each fit half an SM's shared memory (Q4_K slots are 4.6 KB at K = 4096).
+    // The next call's first weight slots then load while this call drains
+    // (interleaved A/B on B200: 4096 x 4096 5.57 -> 4.67 us, 16,384 x 4096
+    // 10.0 -> 9.5 us).  Q8_0's 8.7 KB slots would need fewer warps, which
+    // cost more than the overlap gives (8192 x 4096: 8.0 -> 8.7 us).
+    if (a.stages == 2 && size_t(kMaxWarps) * 2 * (a.slot_bytes + sizeof(uint64_t)) <= kOverlapSmem)
+      return dispatch_g<DSQ_Q4_K, false, kActGlobal, DSQ_GEMV_MAX_WARPS, 2>(a, G, num_sms, stream);
   }
   if (type == DSQ_Q8_0)
     return isum ? dispatch_act<DSQ_Q8_0, true>(a, G, act, num_sms, stream)

@@ -43,6 +43,14 @@
  *  - A device-side wait that exceeds its time limit (default 1 s) records
  *    DSQ_ERR_TIMEOUT in a device status word instead of hanging; read it
  *    with dsq_device_status().
+ *  - Kernels are launched with programmatic stream serialization: each one
+ *    waits for its predecessors (griddepcontrol.wait) before it reads
+ *    activations or writes outputs.  Weights are read-only inputs: some
+ *    decode GEMVs (Q4_K) start loading them before that wait.  So weights
+ *    must not be written by a kernel that is still running when the call is
+ *    launched -- a kernel that releases its dependents early
+ *    (griddepcontrol.launch_dependents) before writing them.  Ordinary
+ *    kernels and every kernel of this library meet this.
  */
 #ifndef DSQ_H
 #define DSQ_H

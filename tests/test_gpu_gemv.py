@@ -184,3 +184,32 @@ def test_gemv_q4_k_long_matrix_takes_the_wide_launch(dsq, ref, N):
     torch.cuda.synchronize()
     assert torch.equal(y[:4096], y_head)
     _check(ref, 12, w, K, xq, xd, xs, y.cpu().numpy())
+
+
+def test_gemv_q4_k_overlapped_launches_back_to_back(dsq, ref):
+    """Shorter Q4_K GEMVs take the overlapped launch: a call starts loading its
+    weights before its launch-dependency wait, beside the previous call.
+    Weights quantized on the stream just before, and three back-to-back
+    calls on different weights, activations and outputs with no host
+    synchronization between them, each equal the same call made alone."""
+    N, K = 4096, 4096
+    w32 = [synth.weights(70 + i, N, K) for i in range(3)]
+    acts = [_prep(ref, 12, 1, K, 80, 81 + i)[1:] for i in range(3)]
+    wq = [torch.zeros((N, K // 256 * 144), dtype=torch.uint8, device="cuda") for _ in range(3)]
+    ys = [torch.full((N,), float("nan"), dtype=torch.float32, device="cuda") for _ in range(3)]
+    dev = [(to_dev(xq), to_dev(xd), to_dev(xs)) for xq, xd, xs in acts]
+    w32g = [to_dev(w) for w in w32]
+    torch.cuda.synchronize()
+    for i in range(3):
+        dsq.dsq_quantize_weights(12, w32g[i], N, K, wq[i])
+    for i in range(3):
+        dsq.dsq_gemv_q4_k(wq[i], N, K, *dev[i], ys[i])
+    torch.cuda.synchronize()
+    for i in range(3):
+        y1 = torch.empty(N, dtype=torch.float32, device="cuda")
+        dsq.dsq_gemv_q4_k(wq[i], N, K, *dev[i], y1)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[i], y1)
+        w_ref = ref.quantize(12, w32[i])
+        assert np.array_equal(wq[i].cpu().numpy(), w_ref)
+        _check(ref, 12, w_ref, K, *acts[i], ys[i].cpu().numpy())
