@@ -729,6 +729,20 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
     if (a.stages == 2 && size_t(kMaxWarps) * 2 * (a.slot_bytes + sizeof(uint64_t)) <= kOverlapSmem)
       return dispatch_g<DSQ_Q4_K, false, kActGlobal, DSQ_GEMV_MAX_WARPS, 2>(a, G, num_sms, stream);
   }
+  // Short Q8_0 matrices whose CTAs hold at most two slots per warp even with
+  // the fewer warps that fit half an SM take the overlapped launch too
+  // (1024 x 1024: 2.09 -> 1.98 us, interleaved A/B on B200).
+  if (type == DSQ_Q8_0 && act == kActGlobal && !isum && a.stages == 2) {
+    const int64_t chunks = (total + (32 / G) - 1) / (32 / G);
+    const int64_t slots = static_cast<int64_t>(num_sms) * DSQ_GEMV_CTAS_PER_SM;
+    const int64_t per_cta_chunks = (chunks + (chunks < slots ? chunks : slots) - 1) / (chunks < slots ? chunks : slots);
+    int64_t w_fit = static_cast<int64_t>(kOverlapSmem / (2 * (static_cast<size_t>(a.slot_bytes) + sizeof(uint64_t))));
+    if (w_fit > kMaxWarps) w_fit = kMaxWarps;
+    if (w_fit >= 1 && per_cta_chunks <= 2 * w_fit) {
+      a.warps = static_cast<int>(w_fit);
+      return dispatch_g<DSQ_Q8_0, false, kActGlobal, DSQ_GEMV_MAX_WARPS, 2>(a, G, num_sms, stream);
+    }
+  }
   if (type == DSQ_Q8_0)
     return isum ? dispatch_act<DSQ_Q8_0, true>(a, G, act, num_sms, stream)
                 : dispatch_act<DSQ_Q8_0, false>(a, G, act, num_sms, stream);
