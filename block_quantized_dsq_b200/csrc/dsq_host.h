@@ -34,6 +34,11 @@ int wait_ctl(WaitCtl *ctl, int *num_sms);
 // After a launch: maps a launch error to DSQ_ERR_LAUNCH and counts launches.
 int after_launch(const char *what, int n_kernels = 1);
 
+// One token of a single weight through the multi-token GEMV (gemv_tokens.cu),
+// errors named after `name`.
+int gemv_one_token(const char *name, int type, const void *w, int64_t N, int64_t K, const int8_t *xq,
+                   const float *xd, const int32_t *xs, float *y, cudaStream_t stream);
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, context):
 // the first call in a context configures it; later calls (for example inside
 // a CUDA graph capture) only launch.

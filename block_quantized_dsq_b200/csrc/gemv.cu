@@ -53,6 +53,11 @@
 #endif
 // Long Q4_K matrices: more warps, once every CTA has at least this many
 // rows (12 warps of at most 168 registers, 16 of at most 128).
+// Single matrices from this many rows up to one 32-row group per SM (one
+// token) run the multi-token kernel.
+#ifndef DSQ_GEMV_TOK_MIN_ROWS
+#define DSQ_GEMV_TOK_MIN_ROWS 2048
+#endif
 #ifndef DSQ_GEMV_MID_MIN_ROWS
 #define DSQ_GEMV_MID_MIN_ROWS 140
 #endif
@@ -679,6 +684,16 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   a.x32 = x32;
   a.act_rows = groups;
 
+  // Mid-length single matrices on one token: the multi-token kernel (one CTA
+  // per 32-row group, warps over 256-element units, bit-identical outputs)
+  // is faster while its row groups fill at most one wave of SMs.
+  // Interleaved A/B on B200, K = 4096, this kernel against it: Q4_K 2048 /
+  // 3072 / 4096 rows 3.57 / 4.53 / 4.67 against 3.49 / 3.92 / 4.14 us, Q8_0
+  // 2048 / 4096 rows 3.81 / 6.21 against 3.65 / 4.99 us; past one wave
+  // (Q4_K 5120 rows) 5.47 against 5.82 us.
+  if (s1.rows == 0 && groups == 1 && !isum && !x32 && K % 256 == 0 && total >= DSQ_GEMV_TOK_MIN_ROWS &&
+      (total + 31) / 32 <= num_sms)
+    return gemv_one_token(name, type, s0.w, s0.rows, K, xq, xd, xs, s0.y, stream);
   if (rb % 16 != 0) {  // Q8_0 with K % 256 != 0
     const int64_t blocks = (total + 7) / 8;
     const unsigned grid = static_cast<unsigned>(blocks < 4 * num_sms ? blocks : 4 * num_sms);

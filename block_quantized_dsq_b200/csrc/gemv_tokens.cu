@@ -871,6 +871,13 @@ int run_tokens(const char *name, int type, const void *w0, int64_t N0, const voi
 }
 
 }  // namespace
+
+// One token through the multi-token kernel, with the caller's name in any
+// error message (the decode GEMV entry points route mid-length matrices here).
+int gemv_one_token(const char *name, int type, const void *w, int64_t N, int64_t K, const int8_t *xq,
+                   const float *xd, const int32_t *xs, float *y, cudaStream_t stream) {
+  return run_tokens(name, type, w, N, nullptr, 0, K, 1, xq, xd, xs, y, nullptr, nullptr, stream);
+}
 }  // namespace dsq
 
 extern "C" {

@@ -186,13 +186,14 @@ def test_gemv_q4_k_long_matrix_takes_the_wide_launch(dsq, ref, N):
     _check(ref, 12, w, K, xq, xd, xs, y.cpu().numpy())
 
 
-def test_gemv_q4_k_overlapped_launches_back_to_back(dsq, ref):
+@pytest.mark.parametrize("N", [1024, 8192])   # below and above the multi-token kernel's range
+def test_gemv_q4_k_overlapped_launches_back_to_back(dsq, ref, N):
     """Shorter Q4_K GEMVs take the overlapped launch: a call starts loading its
     weights before its launch-dependency wait, beside the previous call.
     Weights quantized on the stream just before, and three back-to-back
     calls on different weights, activations and outputs with no host
     synchronization between them, each equal the same call made alone."""
-    N, K = 4096, 4096
+    K = 4096
     w32 = [synth.weights(70 + i, N, K) for i in range(3)]
     acts = [_prep(ref, 12, 1, K, 80, 81 + i)[1:] for i in range(3)]
     wq = [torch.zeros((N, K // 256 * 144), dtype=torch.uint8, device="cuda") for _ in range(3)]
@@ -213,3 +214,25 @@ def test_gemv_q4_k_overlapped_launches_back_to_back(dsq, ref):
         w_ref = ref.quantize(12, w32[i])
         assert np.array_equal(wq[i].cpu().numpy(), w_ref)
         _check(ref, 12, w_ref, K, *acts[i], ys[i].cpu().numpy())
+
+
+@pytest.mark.parametrize("qtype,N", [(8, 3000), (12, 2500), (8, 148 * 32), (12, 148 * 32 + 1), (8, 2047)])
+def test_gemv_mid_length_single_token_routes_bit_exactly(dsq, ref, qtype, N):
+    """From 2048 rows up to one 32-row group per SM (4736 rows on 148 SMs) a
+    single-token GEMV runs the multi-token kernel; outside that range the
+    GEMV kernel.  Either way the outputs equal, bit for bit, those of the
+    block-sum hook (always the GEMV kernel), and the oracle's within 1e-5."""
+    K = 4096
+    w, xq, xd, xs = _prep(ref, qtype, N, K, 90 + N, 91)
+    wg, xqg, xdg, xsg = to_dev(w), to_dev(xq), to_dev(xd), to_dev(xs)
+    y = torch.empty(N, dtype=torch.float32, device="cuda")
+    if qtype == 8:
+        dsq.dsq_gemv_q8_0(wg, N, K, xqg, xdg, y)
+    else:
+        dsq.dsq_gemv_q4_k(wg, N, K, xqg, xdg, xsg, y)
+    y_hook = torch.empty(N, dtype=torch.float32, device="cuda")
+    isum = torch.empty((N, K // 32), dtype=torch.int32, device="cuda")
+    dsq.dsq_test_block_sums(qtype, wg, N, K, xqg, xdg, xsg, y_hook, isum)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_hook)
+    _check(ref, qtype, w, K, xq, xd, xs, y.cpu().numpy())
