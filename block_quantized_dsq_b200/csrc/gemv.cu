@@ -691,7 +691,8 @@ int run_gemv(const char *name, int type, Seg s0, Seg s1, int64_t group_rows, int
   // 3072 / 4096 rows 3.57 / 4.53 / 4.67 against 3.49 / 3.92 / 4.14 us, Q8_0
   // 2048 / 4096 rows 3.81 / 6.21 against 3.65 / 4.99 us; past one wave
   // (Q4_K 5120 rows) 5.47 against 5.82 us.
-  if (s1.rows == 0 && groups == 1 && !isum && !x32 && K % 256 == 0 && total >= DSQ_GEMV_TOK_MIN_ROWS &&
+  // (K <= 32768 keeps one token's activation inside that kernel's 64 KB area.)
+  if (s1.rows == 0 && groups == 1 && !isum && !x32 && K % 256 == 0 && K <= 32768 && total >= DSQ_GEMV_TOK_MIN_ROWS &&
       (total + 31) / 32 <= num_sms)
     return gemv_one_token(name, type, s0.w, s0.rows, K, xq, xd, xs, s0.y, stream);
   if (rb % 16 != 0) {  // Q8_0 with K % 256 != 0

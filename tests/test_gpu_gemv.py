@@ -216,13 +216,14 @@ def test_gemv_q4_k_overlapped_launches_back_to_back(dsq, ref, N):
         _check(ref, 12, w_ref, K, *acts[i], ys[i].cpu().numpy())
 
 
-@pytest.mark.parametrize("qtype,N", [(8, 3000), (12, 2500), (8, 148 * 32), (12, 148 * 32 + 1), (8, 2047)])
-def test_gemv_mid_length_single_token_routes_bit_exactly(dsq, ref, qtype, N):
-    """From 2048 rows up to one 32-row group per SM (4736 rows on 148 SMs) a
-    single-token GEMV runs the multi-token kernel; outside that range the
-    GEMV kernel.  Either way the outputs equal, bit for bit, those of the
+@pytest.mark.parametrize("qtype,N,K", [(8, 3000, 4096), (12, 2500, 4096), (8, 148 * 32, 4096),
+                                       (12, 148 * 32 + 1, 4096), (8, 2047, 4096),
+                                       (8, 2048, 36864)])   # K above the multi-token kernel's activation area
+def test_gemv_mid_length_single_token_routes_bit_exactly(dsq, ref, qtype, N, K):
+    """From 2048 rows up to one 32-row group per SM (4736 rows on 148 SMs), and
+    K up to 32768, a single-token GEMV runs the multi-token kernel; outside
+    that range the GEMV kernel.  Either way the outputs equal, bit for bit, those of the
     block-sum hook (always the GEMV kernel), and the oracle's within 1e-5."""
-    K = 4096
     w, xq, xd, xs = _prep(ref, qtype, N, K, 90 + N, 91)
     wg, xqg, xdg, xsg = to_dev(w), to_dev(xq), to_dev(xd), to_dev(xs)
     y = torch.empty(N, dtype=torch.float32, device="cuda")
